@@ -1,0 +1,120 @@
+"""Seeded synthetic tensors shaped like the pages' workloads.
+
+This module only draws random floats and rounds them to the storage format
+(round-to-nearest-even through torch's own casts).  It holds none of the
+codec's arithmetic, so both the CUDA path and the CPU oracle can consume its
+output.  Every generator returns raw bit patterns as numpy arrays: ``uint16``
+for BF16, ``uint8`` for FP8 E4M3.
+
+Workloads (the pages measure on real checkpoints and K/V caches, which are not
+available; these stand in for them):
+
+* ``bf16_1m``   one BF16 1024x1024 tensor, N(0, 0.02^2), seed 0.
+* ``fp8_16m``   one FP8 E4M3 4096x4096 tensor: N(0, 0.02^2) scaled per tensor so
+  that amax maps to 448, then rounded to E4M3, seed 1.
+* ``llama8b_block``  the seven BF16 weight matrices of one Llama-3.1-8B block
+  (q 4096x4096, k 1024x4096, v 1024x4096, o 4096x4096, gate/up 14336x4096,
+  down 4096x14336; 218,103,808 values), Student-t with 5 degrees of freedom
+  scaled to standard deviation 0.02, seed 2.
+* ``kv_layer``  one layer's BF16 K and V caches, [batch 8, tokens 8192,
+  kv heads 8, head dim 128] each: N(0, 1) times a per-channel lognormal(0, 0.5)
+  scale, with 4 outlier channels per head scaled by 20, seed 3.  A 64-token
+  page of one tensor is 64*8*128 = 65,536 values.
+* ``lm_head``   one BF16 128256x4096 tensor, N(0, 0.02^2), seed 4.
+"""
+import math
+
+import numpy as np
+import torch
+
+LLAMA8B_BLOCK_SHAPES = [
+    ("q_proj", (4096, 4096)),
+    ("k_proj", (1024, 4096)),
+    ("v_proj", (1024, 4096)),
+    ("o_proj", (4096, 4096)),
+    ("gate_proj", (14336, 4096)),
+    ("up_proj", (14336, 4096)),
+    ("down_proj", (4096, 14336)),
+]
+
+WORKLOADS = ("bf16_1m", "fp8_16m", "llama8b_block", "kv_layer", "lm_head")
+
+
+def to_bf16_bits(a: np.ndarray) -> np.ndarray:
+    """float32/float64 -> BF16 bit patterns (uint16), round-to-nearest-even."""
+    t = torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32))
+    return t.to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16).reshape(a.shape)
+
+
+def to_fp8_e4m3_bits(a: np.ndarray) -> np.ndarray:
+    """float32 -> FP8 E4M3 (fn variant) bit patterns (uint8), round-to-nearest-even."""
+    t = torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32))
+    return t.to(torch.float8_e4m3fn).view(torch.uint8).numpy().reshape(a.shape)
+
+
+def normal_bf16(n: int, seed: int, std: float = 0.02) -> np.ndarray:
+    rng = np.random.default_rng(seed)
+    w = rng.standard_normal(n, dtype=np.float32)
+    w *= np.float32(std)
+    return to_bf16_bits(w)
+
+
+def normal_fp8(n: int, seed: int, std: float = 0.02) -> np.ndarray:
+    rng = np.random.default_rng(seed)
+    w = rng.standard_normal(n, dtype=np.float32)
+    w *= np.float32(std)
+    w *= np.float32(448.0) / np.abs(w).max()
+    return to_fp8_e4m3_bits(w)
+
+
+def student_t_bf16(shape, rng: np.random.Generator, df: float = 5.0,
+                   std: float = 0.02) -> np.ndarray:
+    # a t(df) draw has variance df/(df-2); rescale to the requested std
+    w = rng.standard_t(df, size=shape).astype(np.float32)
+    w *= np.float32(std / math.sqrt(df / (df - 2.0)))
+    return to_bf16_bits(w)
+
+
+def llama8b_block(seed: int = 2, scale: int = 1):
+    """[(name, bits)] for the seven matrices; ``scale`` divides the row count
+    (scale=1 is the full block)."""
+    rng = np.random.default_rng(seed)
+    out = []
+    for name, (r, c) in LLAMA8B_BLOCK_SHAPES:
+        out.append((name, student_t_bf16((max(1, r // scale), c), rng).reshape(-1)))
+    return out
+
+
+def kv_tensor(rng: np.random.Generator, batch: int, tokens: int, heads: int = 8,
+              head_dim: int = 128, outliers: int = 4) -> np.ndarray:
+    scale = rng.lognormal(0.0, 0.5, size=(heads, head_dim)).astype(np.float32)
+    for h in range(heads):
+        idx = rng.choice(head_dim, outliers, replace=False)
+        scale[h, idx] *= np.float32(20.0)
+    x = rng.standard_normal((batch, tokens, heads, head_dim), dtype=np.float32)
+    x *= scale[None, None, :, :]
+    return to_bf16_bits(x).reshape(-1)
+
+
+def kv_layer(seed: int = 3, batch: int = 8, tokens: int = 8192):
+    """[("k", bits), ("v", bits)], layout [batch, token, head, dim]."""
+    rng = np.random.default_rng(seed)
+    k = kv_tensor(rng, batch, tokens)
+    v = kv_tensor(rng, batch, tokens)
+    return [("k", k), ("v", v)]
+
+
+def workload(name: str, scale: int = 1):
+    """Returns (dtype_name, [(item_name, bits)]).  ``scale`` > 1 shrinks the
+    workload (fewer rows / tokens) for quick parity runs."""
+    if name == "bf16_1m":
+        return "bf16", [("w", normal_bf16((1 << 20) // scale, seed=0))]
+    if name == "fp8_16m":
+        return "fp8_e4m3", [("w", normal_fp8((4096 * 4096) // scale, seed=1))]
+    if name == "llama8b_block":
+        return "bf16", llama8b_block(seed=2, scale=scale)
+    if name == "kv_layer":
+        return "bf16", kv_layer(seed=3, tokens=max(64, 8192 // scale))
+    if name == "lm_head":
+        return "bf16", [("w", normal_bf16((128256 // scale) * 4096, seed=4))]
+    raise KeyError(name)

@@ -1,0 +1,112 @@
+/*
+ * ehref.h -- CPU oracle for the split-exponent Huffman codec.
+ *
+ * TEST INFRASTRUCTURE ONLY.  This library is the plain, slow, single-threaded
+ * statement of what the codec computes.  Only the test suite, the smoke check
+ * and the CPU-baseline leg of the benchmark may load it.  The product library
+ * (libexphuff) shares no source with it and never calls it.
+ *
+ * Sources the steps follow (page title, then section):
+ *  - "70% Size, 100% Accuracy: Lossless LLM Compression for Efficient GPU
+ *    Inference via Dynamic-Length Float" (DFloat11 news article), section
+ *    "方法介绍": the exponent is Huffman-coded from the histogram of all
+ *    exponents, the codes are bit-packed tightly into EncodedExponent, and the
+ *    raw sign and mantissa go to a separate byte array PackedSignMantissa.
+ *  - "Lossless Compression of Neural Network Components ... Low-Precision
+ *    Formats" (paper summary), sections "方法详解" and "实验设计": exponent and
+ *    mantissa are separated; each tensor is coded in fixed-size chunks.
+ *  - "ZipFloat: An Ultra-fast and Lossless Floating-Point Compressor for LLM
+ *    Inference Systems", section 2.1 (Table 2): the BF16 exponent field is the
+ *    exponent plus 127.
+ * Where the pages are silent (tie-breaks, bit order, chunk size, length limit)
+ * the format below fixes one reading; each is listed in the header of
+ * ehref.cpp.
+ *
+ * All pointers are HOST pointers.  Functions return EHREF_OK (0) or a
+ * negative EHREF_E* code.
+ */
+#ifndef EHREF_H
+#define EHREF_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum { EHREF_BF16 = 0, EHREF_FP8_E4M3 = 1 };
+
+enum {
+  EHREF_OK = 0,
+  EHREF_EINVAL = -1,      /* bad argument                                   */
+  EHREF_EINFEASIBLE = -2, /* more distinct symbols than 2^max_code_len      */
+  EHREF_ECAPACITY = -3,   /* output stream buffer too small                 */
+  EHREF_ECORRUPT = -4     /* compressed data inconsistent                   */
+};
+
+/* 256 for BF16 (8-bit exponent field), 16 for FP8 E4M3 (4-bit field). */
+int ehref_alphabet(int dtype);
+
+/* Step S1.  Per element: exponent field e[i] and the raw sign+mantissa
+ * value sm[i] (BF16: (s<<7)|m7, FP8: (s<<3)|m3), one byte each. */
+int ehref_split(int dtype, const void *in, uint64_t n, uint8_t *e, uint8_t *sm);
+
+/* Inverse of ehref_split for one element stream. */
+int ehref_merge(int dtype, const uint8_t *e, const uint8_t *sm, uint64_t n,
+                void *out);
+
+/* Histogram of exponent fields, cnt[A]. */
+int ehref_histogram(int dtype, const void *in, uint64_t n, uint64_t *cnt);
+
+/* Min-variance Huffman leaf depths (0 for absent symbols), before any length
+ * limit or rank assignment.  Returns the maximum depth (>= 0). */
+int ehref_huffman_depths(const uint64_t *cnt, int A, uint8_t *depth);
+
+/* Package-merge lengths limited to Lmax (0 for absent symbols), before rank
+ * assignment.  Needs at least 2 present symbols and at most 2^Lmax. */
+int ehref_package_merge(const uint64_t *cnt, int A, int Lmax, uint8_t *len);
+
+/* The full length rule of the format: Huffman, package-merge when the Huffman
+ * depth exceeds Lmax, then rank assignment. */
+int ehref_code_lengths(const uint64_t *cnt, int A, int Lmax, uint8_t *len);
+
+/* Canonical codes from lengths (0-length symbols get code 0). */
+int ehref_canonical_codes(const uint8_t *len, int A, uint32_t *code);
+
+/* Sign/mantissa array in its stored layout: BF16 one byte per element; FP8
+ * one nibble per element, element 2i in the low nibble of byte i. */
+uint64_t ehref_sm_bytes(int dtype, uint64_t n);
+int ehref_pack_sm(int dtype, const void *in, uint64_t n, uint8_t *sm_packed);
+
+/* Encode the exponent stream with a given code: off[C+1] bit offsets, stream
+ * bytes (zero-filled first, MSB-first bit order), total bits. */
+uint64_t ehref_num_chunks(uint64_t n, uint32_t chunk);
+int ehref_encode(int dtype, const void *in, uint64_t n, uint32_t chunk,
+                 const uint8_t *len, const uint32_t *code, uint64_t *off,
+                 uint8_t *stream, uint64_t stream_cap, uint64_t *total_bits);
+
+/* Steps S1-S5 in order. */
+int ehref_compress(int dtype, const void *in, uint64_t n, uint32_t chunk,
+                   int Lmax, uint8_t *len, uint32_t *code, uint64_t *off,
+                   uint8_t *stream, uint64_t stream_cap, uint8_t *sm_packed,
+                   uint64_t *total_bits);
+
+/* Step S6 for chunks [first, first+count): writes elements
+ * [first*chunk, min(n, (first+count)*chunk)) to out (indexed from element
+ * first*chunk, i.e. out points at the first decoded element). */
+int ehref_decompress_chunks(int dtype, uint64_t n, uint32_t chunk,
+                            const uint8_t *len, const uint32_t *code,
+                            const uint64_t *off, const uint8_t *stream,
+                            uint64_t stream_bytes, const uint8_t *sm_packed,
+                            uint32_t first, uint32_t count, void *out);
+
+/* Step S6 over all chunks. */
+int ehref_decompress(int dtype, uint64_t n, uint32_t chunk, const uint8_t *len,
+                     const uint32_t *code, const uint64_t *off,
+                     const uint8_t *stream, uint64_t stream_bytes,
+                     const uint8_t *sm_packed, void *out);
+
+#ifdef __cplusplus
+}
+#endif
+#endif

@@ -1,0 +1,206 @@
+"""ctypes wrapper around the CPU oracle (libehref.so).
+
+Test infrastructure only.  Inputs and outputs are numpy arrays of raw bit
+patterns: uint16 for BF16, uint8 for FP8 E4M3.  Errors raise OracleError with
+the oracle's code.
+"""
+import ctypes as C
+from dataclasses import dataclass
+
+import numpy as np
+
+from . import build as _build
+
+BF16 = 0
+FP8_E4M3 = 1
+
+OK, EINVAL, EINFEASIBLE, ECAPACITY, ECORRUPT = 0, -1, -2, -3, -4
+_NAMES = {EINVAL: "EINVAL", EINFEASIBLE: "EINFEASIBLE", ECAPACITY: "ECAPACITY",
+          ECORRUPT: "ECORRUPT"}
+
+
+class OracleError(RuntimeError):
+    def __init__(self, code):
+        super().__init__(f"oracle returned {_NAMES.get(code, code)}")
+        self.code = code
+
+
+_lib = None
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        _lib = C.CDLL(_build.build())
+        u64, i32, u32, vp = C.c_uint64, C.c_int, C.c_uint32, C.c_void_p
+        sig = {
+            "ehref_alphabet": (i32, [i32]),
+            "ehref_split": (i32, [i32, vp, u64, vp, vp]),
+            "ehref_merge": (i32, [i32, vp, vp, u64, vp]),
+            "ehref_histogram": (i32, [i32, vp, u64, vp]),
+            "ehref_huffman_depths": (i32, [vp, i32, vp]),
+            "ehref_package_merge": (i32, [vp, i32, i32, vp]),
+            "ehref_code_lengths": (i32, [vp, i32, i32, vp]),
+            "ehref_canonical_codes": (i32, [vp, i32, vp]),
+            "ehref_sm_bytes": (u64, [i32, u64]),
+            "ehref_pack_sm": (i32, [i32, vp, u64, vp]),
+            "ehref_num_chunks": (u64, [u64, u32]),
+            "ehref_encode": (i32, [i32, vp, u64, u32, vp, vp, vp, vp, u64, vp]),
+            "ehref_compress": (i32, [i32, vp, u64, u32, i32, vp, vp, vp, vp, u64, vp, vp]),
+            "ehref_decompress_chunks": (i32, [i32, u64, u32, vp, vp, vp, vp, u64, vp, u32, u32, vp]),
+            "ehref_decompress": (i32, [i32, u64, u32, vp, vp, vp, vp, u64, vp, vp]),
+        }
+        for name, (res, args) in sig.items():
+            f = getattr(_lib, name)
+            f.restype = res
+            f.argtypes = args
+    return _lib
+
+
+def _p(a):
+    return a.ctypes.data_as(C.c_void_p) if a is not None else None
+
+
+def _check(rc):
+    if rc != OK:
+        raise OracleError(rc)
+
+
+def elem_dtype(dtype):
+    return np.uint16 if dtype == BF16 else np.uint8
+
+
+def alphabet(dtype):
+    return lib().ehref_alphabet(dtype)
+
+
+def split(dtype, x):
+    x = np.ascontiguousarray(x, dtype=elem_dtype(dtype))
+    e = np.empty(x.size, np.uint8)
+    sm = np.empty(x.size, np.uint8)
+    _check(lib().ehref_split(dtype, _p(x), x.size, _p(e), _p(sm)))
+    return e, sm
+
+
+def merge(dtype, e, sm):
+    e = np.ascontiguousarray(e, np.uint8)
+    sm = np.ascontiguousarray(sm, np.uint8)
+    out = np.empty(e.size, elem_dtype(dtype))
+    _check(lib().ehref_merge(dtype, _p(e), _p(sm), e.size, _p(out)))
+    return out
+
+
+def histogram(dtype, x):
+    x = np.ascontiguousarray(x, dtype=elem_dtype(dtype))
+    cnt = np.zeros(alphabet(dtype), np.uint64)
+    _check(lib().ehref_histogram(dtype, _p(x), x.size, _p(cnt)))
+    return cnt
+
+
+def huffman_depths(cnt):
+    cnt = np.ascontiguousarray(cnt, np.uint64)
+    d = np.zeros(cnt.size, np.uint8)
+    rc = lib().ehref_huffman_depths(_p(cnt), cnt.size, _p(d))
+    if rc < 0:
+        raise OracleError(rc)
+    return d
+
+
+def package_merge(cnt, lmax):
+    cnt = np.ascontiguousarray(cnt, np.uint64)
+    ln = np.zeros(cnt.size, np.uint8)
+    _check(lib().ehref_package_merge(_p(cnt), cnt.size, lmax, _p(ln)))
+    return ln
+
+
+def code_lengths(cnt, lmax=32):
+    cnt = np.ascontiguousarray(cnt, np.uint64)
+    ln = np.zeros(cnt.size, np.uint8)
+    _check(lib().ehref_code_lengths(_p(cnt), cnt.size, lmax, _p(ln)))
+    return ln
+
+
+def canonical_codes(lengths):
+    ln = np.ascontiguousarray(lengths, np.uint8)
+    code = np.zeros(ln.size, np.uint32)
+    _check(lib().ehref_canonical_codes(_p(ln), ln.size, _p(code)))
+    return code
+
+
+def sm_bytes(dtype, n):
+    return lib().ehref_sm_bytes(dtype, n)
+
+
+def pack_sm(dtype, x):
+    x = np.ascontiguousarray(x, dtype=elem_dtype(dtype))
+    out = np.empty(sm_bytes(dtype, x.size), np.uint8)
+    _check(lib().ehref_pack_sm(dtype, _p(x), x.size, _p(out)))
+    return out
+
+
+def num_chunks(n, chunk):
+    return lib().ehref_num_chunks(n, chunk)
+
+
+@dataclass
+class Compressed:
+    dtype: int
+    n: int
+    chunk: int
+    lmax: int
+    code_len: np.ndarray     # uint8[A]
+    code: np.ndarray         # uint32[A]
+    chunk_bit_off: np.ndarray  # uint64[C+1]
+    stream: np.ndarray       # uint8[ceil(bits/8)]
+    sign_mant: np.ndarray    # uint8[n or ceil(n/2)]
+    bits: int
+
+
+def encode(dtype, x, chunk, lengths, codes):
+    x = np.ascontiguousarray(x, dtype=elem_dtype(dtype))
+    n = x.size
+    ln = np.ascontiguousarray(lengths, np.uint8)
+    cd = np.ascontiguousarray(codes, np.uint32)
+    nc = num_chunks(n, chunk)
+    off = np.zeros(nc + 1, np.uint64)
+    cap = (n * 32 + 7) // 8
+    stream = np.zeros(max(cap, 1), np.uint8)
+    bits = C.c_uint64(0)
+    _check(lib().ehref_encode(dtype, _p(x), n, chunk, _p(ln), _p(cd), _p(off), _p(stream),
+                              cap, C.byref(bits)))
+    return off, stream[: (bits.value + 7) // 8].copy(), bits.value
+
+
+def compress(dtype, x, chunk=65536, lmax=32):
+    x = np.ascontiguousarray(x, dtype=elem_dtype(dtype))
+    n = x.size
+    A = alphabet(dtype)
+    ln = np.zeros(A, np.uint8)
+    code = np.zeros(A, np.uint32)
+    nc = num_chunks(n, chunk)
+    off = np.zeros(nc + 1, np.uint64)
+    cap = (n * lmax + 7) // 8
+    stream = np.zeros(max(cap, 1), np.uint8)
+    sm = np.zeros(max(sm_bytes(dtype, n), 1), np.uint8)
+    bits = C.c_uint64(0)
+    _check(lib().ehref_compress(dtype, _p(x), n, chunk, lmax, _p(ln), _p(code), _p(off),
+                                _p(stream), cap, _p(sm), C.byref(bits)))
+    return Compressed(dtype, n, chunk, lmax, ln, code, off,
+                      stream[: (bits.value + 7) // 8].copy(),
+                      sm[: sm_bytes(dtype, n)].copy(), bits.value)
+
+
+def decompress(c: Compressed, first=None, count=None):
+    nc = num_chunks(c.n, c.chunk)
+    if first is None:
+        first, count = 0, nc
+    i0 = first * c.chunk
+    i1 = min(c.n, (first + count) * c.chunk)
+    out = np.zeros(max(i1 - i0, 0), elem_dtype(c.dtype))
+    stream = np.ascontiguousarray(c.stream, np.uint8)
+    _check(lib().ehref_decompress_chunks(
+        c.dtype, c.n, c.chunk, _p(np.ascontiguousarray(c.code_len, np.uint8)),
+        _p(np.ascontiguousarray(c.code, np.uint32)),
+        _p(np.ascontiguousarray(c.chunk_bit_off, np.uint64)), _p(stream), stream.size,
+        _p(np.ascontiguousarray(c.sign_mant, np.uint8)), first, count, _p(out)))
+    return out
