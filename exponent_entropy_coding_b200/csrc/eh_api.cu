@@ -1,0 +1,314 @@
+// eh_api.cu -- the C ABI of libexphuff (include/exphuff.h): argument checks,
+// workspace layout, kernel launches and status mapping.  No allocation happens
+// here: every buffer, the workspace included, belongs to the caller.
+#include <atomic>
+#include <cstring>
+#include <mutex>
+
+#include "eh_internal.cuh"
+
+using namespace eh;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+  std::once_flag once;
+  int num_sms = 0;
+  cudaError_t err = cudaSuccess;
+};
+DeviceInfo g_dev[kMaxDevices];
+
+// SM count of the current device; configures the kernels once per device.
+cudaError_t device_setup(int *num_sms) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  DeviceInfo &d = g_dev[dev];
+  std::call_once(d.once, [&d, dev]() {
+    d.err = cudaDeviceGetAttribute(&d.num_sms, cudaDevAttrMultiProcessorCount, dev);
+    if (d.err == cudaSuccess) d.err = configure_decode();
+  });
+  *num_sms = d.num_sms;
+  return d.err;
+}
+
+inline bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
+inline uint64_t ceil_div(uint64_t a, uint64_t b) { return (a + b - 1) / b; }
+
+bool plan_ok(const eh_plan_t *p) {
+  return p && (p->dtype == EH_BF16 || p->dtype == EH_FP8_E4M3) && p->chunk_elems >= 1024 &&
+         p->chunk_elems <= (uint32_t)kMaxChunk && p->chunk_elems % 1024 == 0 && p->max_code_len >= 1 &&
+         p->max_code_len <= EH_MAX_CODE_LEN;
+}
+
+uint64_t stream_cap_for(const eh_plan_t *p, uint64_t n) {
+  return ((ceil_div(n * p->max_code_len, 8) + 15) & ~uint64_t(15)) + 16;
+}
+
+uint64_t sm_bytes_for(int dtype, uint64_t n) { return dtype == EH_BF16 ? n : ceil_div(n, 2); }
+
+// ---- compress workspace layout
+//   [0, 256)                 status (u32), ticket (u32), bit totals u64[k]
+//   [256, 256 + 2048k)       per-tensor exponent counts u64[256]
+//   then per tensor, each 256-aligned: package-merge scratch u64[33][256],
+//   per-chunk histograms u32[C][A], per-chunk bits u64[C]
+constexpr uint64_t kHeader = 256;
+constexpr uint64_t kCountsBytes = 256 * sizeof(uint64_t);
+constexpr uint64_t kPmBytes = 33 * 256 * sizeof(uint64_t);
+
+uint64_t compress_ws_bytes(const eh_plan_t *p, int k, const uint64_t *ns) {
+  uint64_t total = align256(kHeader + (uint64_t)k * kCountsBytes);
+  const uint64_t A = alphabet_of(p->dtype);
+  for (int i = 0; i < k; i++) {
+    const uint64_t C = ceil_div(ns[i], p->chunk_elems);
+    total += align256(kPmBytes) + align256(C * A * 4) + align256(C * 8);
+  }
+  return total;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *eh_version(void) { return "libexphuff 0.1 sm_100a"; }
+
+const char *eh_status_str(eh_status s) {
+  switch (s) {
+    case EH_OK: return "ok";
+    case EH_ERR_INVALID_ARG: return "invalid argument";
+    case EH_ERR_UNSUPPORTED: return "unsupported dtype, chunk size or code length limit";
+    case EH_ERR_INFEASIBLE: return "more distinct exponents than the code length limit allows";
+    case EH_ERR_CUDA: return "CUDA runtime error";
+    case EH_ERR_CORRUPT: return "corrupt compressed data or codebook";
+    case EH_ERR_TIMEOUT: return "a bounded wait in a kernel gave up";
+    case EH_ERR_NOMEM: return "workspace too small";
+  }
+  return "unknown status";
+}
+
+eh_status eh_plan(eh_plan_t *plan, int32_t dtype, uint32_t chunk_elems, uint32_t max_code_len) {
+  if (!plan) return EH_ERR_INVALID_ARG;
+  eh_plan_t p;
+  p.dtype = dtype;
+  p.chunk_elems = chunk_elems ? chunk_elems : EH_DEFAULT_CHUNK_ELEMS;
+  p.max_code_len = max_code_len ? max_code_len : EH_MAX_CODE_LEN;
+  p.reserved = 0;
+  if (!plan_ok(&p)) return EH_ERR_UNSUPPORTED;
+  *plan = p;
+  return EH_OK;
+}
+
+eh_status eh_compress_bound(const eh_plan_t *plan, uint64_t n, uint64_t *stream_cap, uint64_t *sm_bytes,
+                            uint64_t *workspace_bytes) {
+  if (!plan_ok(plan)) return EH_ERR_INVALID_ARG;
+  if (n > (1ull << 40)) return EH_ERR_INVALID_ARG;
+  if (stream_cap) *stream_cap = stream_cap_for(plan, n);
+  if (sm_bytes) *sm_bytes = sm_bytes_for(plan->dtype, n);
+  if (workspace_bytes) *workspace_bytes = compress_ws_bytes(plan, 1, &n);
+  return EH_OK;
+}
+
+eh_status eh_compress_batch_workspace(const eh_plan_t *plan, int k, const uint64_t *ns,
+                                      uint64_t *workspace_bytes) {
+  if (!plan_ok(plan) || k < 1 || k > EH_MAX_BATCH || !ns || !workspace_bytes) return EH_ERR_INVALID_ARG;
+  *workspace_bytes = compress_ws_bytes(plan, k, ns);
+  return EH_OK;
+}
+
+eh_status eh_compress_batch(const eh_plan_t *plan, int k, const void *const *ins, eh_compressed_t *outs,
+                            uint64_t *bits_dev, void *workspace, uint64_t workspace_bytes, void *stream) {
+  if (!plan_ok(plan) || k < 1 || k > EH_MAX_BATCH || !ins || !outs || !workspace) return EH_ERR_INVALID_ARG;
+  if (((uintptr_t)workspace & 255u) != 0 || (bits_dev && ((uintptr_t)bits_dev & 7u))) return EH_ERR_INVALID_ARG;
+  uint64_t ns[EH_MAX_BATCH];
+  uint64_t total_chunks = 0;
+  for (int i = 0; i < k; i++) {
+    const eh_compressed_t &o = outs[i];
+    const uint64_t n = o.n;
+    if (o.dtype != plan->dtype || n > (1ull << 40)) return EH_ERR_INVALID_ARG;
+    if (!o.code_len || !o.code || !o.chunk_bit_off) return EH_ERR_INVALID_ARG;
+    if (((uintptr_t)o.code & 3u) || ((uintptr_t)o.chunk_bit_off & 7u)) return EH_ERR_INVALID_ARG;
+    if (n > 0 && (!ins[i] || !o.exp_stream || !o.sign_mant)) return EH_ERR_INVALID_ARG;
+    if (n > 0 && (!aligned16(ins[i]) || !aligned16(o.exp_stream) || !aligned16(o.sign_mant)))
+      return EH_ERR_INVALID_ARG;
+    if (o.exp_stream_cap < stream_cap_for(plan, n) && n > 0) return EH_ERR_INVALID_ARG;
+    ns[i] = n;
+    total_chunks += ceil_div(n, plan->chunk_elems);
+  }
+  if (total_chunks > 0x7FFFFFFFull) return EH_ERR_INVALID_ARG;
+  if (workspace_bytes < compress_ws_bytes(plan, k, ns)) return EH_ERR_NOMEM;
+  int num_sms = 0;
+  cudaError_t e = device_setup(&num_sms);
+  if (e != cudaSuccess) return EH_ERR_CUDA;
+
+  uint8_t *ws = (uint8_t *)workspace;
+  Batch b;
+  std::memset(&b, 0, sizeof(b));
+  b.k = (uint32_t)k;
+  b.chunk_elems = plan->chunk_elems;
+  b.dtype = plan->dtype;
+  b.max_code_len = plan->max_code_len;
+  b.status = (uint32_t *)ws;
+  b.ticket = (uint32_t *)(ws + 4);
+  uint64_t *bits_ws = (uint64_t *)(ws + 8);
+  const uint64_t A = alphabet_of(plan->dtype);
+  uint64_t cursor = align256(kHeader + (uint64_t)k * kCountsBytes);
+  uint32_t chunk0 = 0;
+  for (int i = 0; i < k; i++) {
+    Item &it = b.item[i];
+    const eh_compressed_t &o = outs[i];
+    const uint32_t C = (uint32_t)ceil_div(o.n, plan->chunk_elems);
+    it.in = ins[i];
+    it.n = o.n;
+    it.chunk0 = chunk0;
+    it.nchunks = C;
+    it.first_chunk = 0;
+    it.total_chunks = C;
+    it.code_len = o.code_len;
+    it.code = o.code;
+    it.off = o.chunk_bit_off;
+    it.stream = o.exp_stream;
+    it.stream_cap = o.exp_stream_cap;
+    it.sm = o.sign_mant;
+    it.counts = (uint64_t *)(ws + kHeader + (uint64_t)i * kCountsBytes);
+    it.bits_out = bits_ws + i;
+    it.bits_dev = bits_dev ? bits_dev + i : nullptr;
+    it.pm_scratch = (uint64_t *)(ws + cursor);
+    cursor += align256(kPmBytes);
+    it.chist = (uint32_t *)(ws + cursor);
+    cursor += align256((uint64_t)C * A * 4);
+    it.cbits = (uint64_t *)(ws + cursor);
+    cursor += align256((uint64_t)C * 8);
+    chunk0 += C;
+  }
+  b.total_chunks = chunk0;
+  cudaStream_t s = (cudaStream_t)stream;
+  if ((e = cudaMemsetAsync(ws, 0, kHeader + (uint64_t)k * kCountsBytes, s)) != cudaSuccess) return EH_ERR_CUDA;
+  if ((e = launch_hist(b, s)) != cudaSuccess) return EH_ERR_CUDA;
+  if ((e = launch_book(b, s)) != cudaSuccess) return EH_ERR_CUDA;
+  if ((e = launch_offsets(b, s)) != cudaSuccess) return EH_ERR_CUDA;
+  if ((e = launch_encode(b, s)) != cudaSuccess) return EH_ERR_CUDA;
+  for (int i = 0; i < k; i++) outs[i].n_chunks = b.item[i].nchunks;
+  if (bits_dev) return EH_OK;
+  uint64_t host[1 + EH_MAX_BATCH];
+  if ((e = cudaMemcpyAsync(host, ws, 8 + 8 * (uint64_t)k, cudaMemcpyDeviceToHost, s)) != cudaSuccess)
+    return EH_ERR_CUDA;
+  if ((e = cudaStreamSynchronize(s)) != cudaSuccess) return EH_ERR_CUDA;
+  const uint32_t status = (uint32_t)host[0];
+  for (int i = 0; i < k; i++) outs[i].exp_stream_bits = host[1 + i];
+  if (status & kFlagInfeasible) return EH_ERR_INFEASIBLE;
+  if (status & kFlagTimeout) return EH_ERR_TIMEOUT;
+  if (status & kFlagCorrupt) return EH_ERR_CORRUPT;
+  return EH_OK;
+}
+
+eh_status eh_compress(const eh_plan_t *plan, const void *in, uint64_t n, eh_compressed_t *out, void *workspace,
+                      uint64_t workspace_bytes, void *stream) {
+  if (!out) return EH_ERR_INVALID_ARG;
+  if (out->n != n) return EH_ERR_INVALID_ARG;
+  const void *ins[1] = {in};
+  return eh_compress_batch(plan, 1, ins, out, nullptr, workspace, workspace_bytes, stream);
+}
+
+eh_status eh_decompress_workspace(const eh_plan_t *plan, int k, uint64_t *workspace_bytes) {
+  if (!plan_ok(plan) || k < 1 || k > EH_MAX_BATCH || !workspace_bytes) return EH_ERR_INVALID_ARG;
+  *workspace_bytes = kHeader + (uint64_t)k * kLutBytes;
+  return EH_OK;
+}
+
+}  // extern "C"
+
+namespace {
+
+eh_status decompress_impl(const eh_plan_t *plan, int k, const eh_compressed_t *cs, void *const *outs,
+                          const uint32_t *firsts, const uint32_t *counts, void *workspace,
+                          uint64_t workspace_bytes, void *stream) {
+  if (!plan_ok(plan) || k < 1 || k > EH_MAX_BATCH || !cs || !outs || !workspace) return EH_ERR_INVALID_ARG;
+  if (((uintptr_t)workspace & 255u) != 0) return EH_ERR_INVALID_ARG;
+  if (workspace_bytes < kHeader + (uint64_t)k * kLutBytes) return EH_ERR_NOMEM;
+  uint8_t *ws = (uint8_t *)workspace;
+  Batch b;
+  std::memset(&b, 0, sizeof(b));
+  b.k = (uint32_t)k;
+  b.chunk_elems = plan->chunk_elems;
+  b.dtype = plan->dtype;
+  b.max_code_len = plan->max_code_len;
+  b.status = (uint32_t *)ws;
+  b.ticket = (uint32_t *)(ws + 4);
+  uint64_t chunk0 = 0;
+  for (int i = 0; i < k; i++) {
+    const eh_compressed_t &c = cs[i];
+    if (c.dtype != plan->dtype || c.n > (1ull << 40)) return EH_ERR_INVALID_ARG;
+    const uint64_t C = ceil_div(c.n, plan->chunk_elems);
+    if (c.n_chunks != C) return EH_ERR_INVALID_ARG;
+    const uint32_t first = firsts ? firsts[i] : 0u;
+    const uint32_t count = counts ? counts[i] : (uint32_t)C;
+    if ((uint64_t)first + count > C) return EH_ERR_INVALID_ARG;
+    if (!c.code_len || !c.code || !c.chunk_bit_off || ((uintptr_t)c.chunk_bit_off & 7u)) return EH_ERR_INVALID_ARG;
+    if (count > 0) {
+      if (!outs[i] || !c.exp_stream || !c.sign_mant) return EH_ERR_INVALID_ARG;
+      if (!aligned16(outs[i]) || !aligned16(c.exp_stream) || !aligned16(c.sign_mant)) return EH_ERR_INVALID_ARG;
+    }
+    Item &it = b.item[i];
+    it.out = outs[i];
+    it.n = c.n;
+    it.elem0 = (uint64_t)first * plan->chunk_elems;
+    it.chunk0 = (uint32_t)chunk0;
+    it.nchunks = count;
+    it.first_chunk = first;
+    it.total_chunks = (uint32_t)C;
+    it.code_len = c.code_len;
+    it.code = c.code;
+    it.off = c.chunk_bit_off;
+    it.stream = c.exp_stream;
+    it.stream_cap = c.exp_stream_cap;
+    it.sm = c.sign_mant;
+    it.lut = ws + kHeader + (uint64_t)i * kLutBytes;
+    chunk0 += count;
+  }
+  if (chunk0 > 0x7FFFFFFFull) return EH_ERR_INVALID_ARG;
+  b.total_chunks = (uint32_t)chunk0;
+  int num_sms = 0;
+  if (device_setup(&num_sms) != cudaSuccess) return EH_ERR_CUDA;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (launch_tables(b, s) != cudaSuccess) return EH_ERR_CUDA;
+  if (launch_decode(b, s, num_sms) != cudaSuccess) return EH_ERR_CUDA;
+  return EH_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+eh_status eh_decompress(const eh_plan_t *plan, const eh_compressed_t *c, void *out, void *workspace,
+                        uint64_t workspace_bytes, void *stream) {
+  void *outs[1] = {out};
+  return decompress_impl(plan, 1, c, outs, nullptr, nullptr, workspace, workspace_bytes, stream);
+}
+
+eh_status eh_decompress_batch(const eh_plan_t *plan, int k, const eh_compressed_t *cs, void *const *outs,
+                              void *workspace, uint64_t workspace_bytes, void *stream) {
+  return decompress_impl(plan, k, cs, outs, nullptr, nullptr, workspace, workspace_bytes, stream);
+}
+
+eh_status eh_decompress_chunks(const eh_plan_t *plan, const eh_compressed_t *c, uint32_t first, uint32_t count,
+                               void *out, void *workspace, uint64_t workspace_bytes, void *stream) {
+  void *outs[1] = {out};
+  return decompress_impl(plan, 1, c, outs, &first, &count, workspace, workspace_bytes, stream);
+}
+
+eh_status eh_get_status(void *workspace, void *stream) {
+  if (!workspace) return EH_ERR_INVALID_ARG;
+  uint32_t st = 0;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (cudaMemcpyAsync(&st, workspace, 4, cudaMemcpyDeviceToHost, s) != cudaSuccess) return EH_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return EH_ERR_CUDA;
+  if (st & kFlagInfeasible) return EH_ERR_INFEASIBLE;
+  if (st & kFlagTimeout) return EH_ERR_TIMEOUT;
+  if (st & kFlagCorrupt) return EH_ERR_CORRUPT;
+  return EH_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,513 @@
+// eh_compress.cu -- compression kernels of libexphuff (sm_100a).
+//
+// Steps, in launch order (one launch per step for a whole batch of tensors):
+//   hist     split every value into exponent field and sign+mantissa, write
+//            the packed sign/mantissa array, and count exponents per chunk and
+//            per tensor (DFloat11 article, "方法介绍": the Huffman code is built
+//            from the exponent distribution; sign and mantissa stay raw);
+//   book     one CTA per tensor: code lengths (minimum-variance Huffman,
+//            package-merge when the depth exceeds the limit), rank assignment,
+//            canonical codes;
+//   offsets  code bits per chunk from its histogram, then (last CTA) an
+//            exclusive scan into the chunk bit offsets and the clearing of the
+//            stream words that two chunks share;
+//   encode   one CTA per chunk: code lookup, CTA-wide exclusive scan of code
+//            lengths, bit packing into a shared-memory word ring, coalesced
+//            stores of whole words and atomic OR of the two edge words.
+// Every kernel is HBM-bound; no tensor cores are involved.
+#include "eh_internal.cuh"
+
+namespace eh {
+namespace {
+
+__device__ __forceinline__ uint4 ld_stream(const void *p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+
+__device__ __forceinline__ uint2 ld_stream8(const void *p) {
+  uint2 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "l"(p));
+  return v;
+}
+
+// BF16 pair in one word -> the two sign+mantissa bytes (s<<7 | m7), low
+// element in the low byte.
+__device__ __forceinline__ uint32_t bf16x2_sm(uint32_t x) {
+  return (x & 0x7Fu) | ((x >> 8) & 0x7F80u) | ((x >> 16) & 0x8000u);
+}
+
+// Four FP8 bytes in one word -> four sign+mantissa nibbles (s<<3 | m3),
+// element 0 in the low nibble.
+__device__ __forceinline__ uint32_t fp8x4_sm(uint32_t x) {
+  uint32_t t = (x & 0x07070707u) | ((x >> 4) & 0x08080808u);
+  return (t & 0xFu) | ((t >> 4) & 0xF0u) | ((t >> 8) & 0xF00u) | ((t >> 12) & 0xF000u);
+}
+
+// ---------------------------------------------------------------- hist
+// Exponent counters are replicated per lane: counter (e, lane) lives at
+// h[e*32 + lane], so the 32 lanes of a warp always hit 32 distinct banks and
+// never the same address, however skewed the exponents are.
+template <int DT>
+__global__ void __launch_bounds__(kThreads, 2) hist_kernel(const __grid_constant__ Batch b) {
+  constexpr int A = DT == EH_BF16 ? 256 : 16;
+  __shared__ uint32_t h[A * 32];
+  const uint32_t g = blockIdx.x;
+  const Item &I = b.item[find_item(b, g)];
+  const uint32_t c = g - I.chunk0;
+  const uint64_t i0 = (uint64_t)c * b.chunk_elems;
+  const uint32_t cnt = (uint32_t)min((uint64_t)b.chunk_elems, I.n - i0);
+  const int tid = threadIdx.x, lane = tid & 31;
+  for (int i = tid; i < A * 32; i += kThreads) h[i] = 0;
+  __syncthreads();
+  uint32_t *hl = h + lane;
+  if (DT == EH_BF16) {
+    const uint16_t *in = (const uint16_t *)I.in + i0;
+    uint8_t *smo = I.sm + i0;
+    const uint32_t nvec = cnt / 16;  // 16 values per step: 32 B in, 16 B out
+    #pragma unroll 2
+    for (uint32_t v = tid; v < nvec; v += kThreads) {
+      uint4 p = ld_stream(in + 16 * (uint64_t)v);
+      uint4 q = ld_stream(in + 16 * (uint64_t)v + 8);
+      uint32_t w[8] = {p.x, p.y, p.z, p.w, q.x, q.y, q.z, q.w};
+      uint32_t o[4];
+      #pragma unroll
+      for (int j = 0; j < 8; j++) {
+        atomicAdd(hl + (((w[j] >> 7) & 0xFFu) << 5), 1u);
+        atomicAdd(hl + (((w[j] >> 23) & 0xFFu) << 5), 1u);
+      }
+      #pragma unroll
+      for (int j = 0; j < 4; j++) o[j] = bf16x2_sm(w[2 * j]) | (bf16x2_sm(w[2 * j + 1]) << 16);
+      *(uint4 *)(smo + 16 * (uint64_t)v) = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+    for (uint32_t i = nvec * 16 + tid; i < cnt; i += kThreads) {
+      uint32_t x = in[i];
+      atomicAdd(hl + (((x >> 7) & 0xFFu) << 5), 1u);
+      smo[i] = (uint8_t)bf16x2_sm(x);
+    }
+  } else {
+    const uint8_t *in = (const uint8_t *)I.in + i0;
+    uint8_t *smo = I.sm + i0 / 2;
+    const uint32_t nvec = cnt / 32;  // 32 values per step: 32 B in, 16 B out
+    #pragma unroll 2
+    for (uint32_t v = tid; v < nvec; v += kThreads) {
+      uint4 p = ld_stream(in + 32 * (uint64_t)v);
+      uint4 q = ld_stream(in + 32 * (uint64_t)v + 16);
+      uint32_t w[8] = {p.x, p.y, p.z, p.w, q.x, q.y, q.z, q.w};
+      uint32_t o[4];
+      #pragma unroll
+      for (int j = 0; j < 8; j++) {
+        #pragma unroll
+        for (int k = 0; k < 4; k++) atomicAdd(hl + (((w[j] >> (8 * k + 3)) & 0xFu) << 5), 1u);
+      }
+      #pragma unroll
+      for (int j = 0; j < 4; j++) o[j] = fp8x4_sm(w[2 * j]) | (fp8x4_sm(w[2 * j + 1]) << 16);
+      *(uint4 *)(smo + 16 * (uint64_t)v) = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+    // tail: one sign/mantissa byte (two values) per thread step
+    for (uint32_t pidx = nvec * 16 + tid; 2 * pidx < cnt; pidx += kThreads) {
+      uint32_t x0 = in[2 * pidx];
+      uint32_t x1 = (2 * pidx + 1 < cnt) ? in[2 * pidx + 1] : 0u;
+      atomicAdd(hl + (((x0 >> 3) & 0xFu) << 5), 1u);
+      if (2 * pidx + 1 < cnt) atomicAdd(hl + (((x1 >> 3) & 0xFu) << 5), 1u);
+      uint32_t s = fp8x4_sm(x0 | (x1 << 8));
+      if (2 * pidx + 1 >= cnt) s &= 0xFu;
+      smo[pidx] = (uint8_t)s;
+    }
+  }
+  __syncthreads();
+  if (tid < A) {
+    uint32_t s = 0;
+    #pragma unroll 8
+    for (int l = 0; l < 32; l++) s += h[tid * 32 + ((l + tid) & 31)];
+    I.chist[(uint64_t)c * A + tid] = s;
+    if (s) atomicAdd((unsigned long long *)&I.counts[tid], (unsigned long long)s);
+  }
+}
+
+// ---------------------------------------------------------------- book
+// One CTA of 256 threads per tensor.
+__global__ void __launch_bounds__(256) book_kernel(const __grid_constant__ Batch b) {
+  const Item &I = b.item[blockIdx.x];
+  const int A = alphabet_of(b.dtype);
+  const int Lmax = (int)b.max_code_len;
+  const int tid = threadIdx.x;
+  __shared__ uint64_t cnt[256];
+  __shared__ uint64_t lw[256];      // leaf weights in (count, symbol) order
+  __shared__ uint64_t iw[256];      // internal node weights in creation order
+  __shared__ uint16_t lpar[256], ipar[256];
+  __shared__ uint8_t idep[256];
+  __shared__ uint8_t len[256];
+  __shared__ uint32_t nlen[33], firstc[33];
+  __shared__ uint32_t xsel[33];     // package-merge: leaves selected per level
+  __shared__ uint32_t maxd;
+
+  const uint64_t c = tid < A ? I.counts[tid] : 0ull;
+  cnt[tid] = c;
+  len[tid] = 0;
+  if (tid <= 32) nlen[tid] = 0;
+  if (tid == 0) maxd = 0;
+  const int m = __syncthreads_count(c > 0);
+  if (c > 0) {
+    int r = 0;
+    for (int s2 = 0; s2 < A; s2++) {
+      uint64_t c2 = cnt[s2];
+      r += (c2 > 0) && (c2 < c || (c2 == c && s2 < tid));
+    }
+    lw[r] = c;
+  }
+  bool feasible = m <= 1 || Lmax >= 32 || (uint64_t)m <= (1ull << Lmax);
+  if (!feasible) {
+    if (tid == 0) set_status(b.status, kFlagInfeasible);
+  }
+  __syncthreads();
+
+  uint32_t d = 0;  // raw length of the leaf with rank `tid` in (count, symbol) order
+  if (m >= 2 && feasible) {
+    if (tid == 0) {
+      // two-queue Huffman: leaves sorted by (count, symbol), internal nodes in
+      // creation order; on equal weight the leaf wins (its id is smaller)
+      int i = 0, j = 0, nint = 0;
+      for (int step = 0; step < m - 1; step++) {
+        uint64_t w = 0;
+        #pragma unroll
+        for (int pick = 0; pick < 2; pick++) {
+          if (i < m && (j >= nint || lw[i] <= iw[j])) {
+            w += lw[i];
+            lpar[i++] = (uint16_t)nint;
+          } else {
+            w += iw[j];
+            ipar[j++] = (uint16_t)nint;
+          }
+        }
+        iw[nint++] = w;
+      }
+      idep[nint - 1] = 0;
+      for (int k = nint - 2; k >= 0; k--) idep[k] = (uint8_t)(idep[ipar[k]] + 1);
+    }
+    __syncthreads();
+    if (tid < m) {
+      d = idep[lpar[tid]] + 1u;
+      atomicMax(&maxd, d);
+    }
+    __syncthreads();
+    if ((int)maxd > Lmax) {
+      if (tid == 0) {
+        // package-merge with counts only: list(level) = merge(leaves,
+        // packages(level)), leaf first on equal weight; packages(level) pair
+        // up consecutive items of list(level+1); list(Lmax) = leaves.
+        uint64_t *pk = I.pm_scratch;  // [33][256]
+        uint32_t npk[33];
+        npk[Lmax] = 0;
+        for (int lev = Lmax - 1; lev >= 1; lev--) {
+          const uint64_t *below = pk + (uint64_t)(lev + 1) * 256;
+          uint64_t *cur = pk + (uint64_t)lev * 256;
+          uint32_t nb = npk[lev + 1], li = 0, pi = 0, np = 0;
+          uint64_t pend = 0;
+          bool have = false;
+          for (uint32_t r = 0; r < (uint32_t)m + nb; r++) {
+            uint64_t w;
+            if (li < (uint32_t)m && (pi >= nb || lw[li] <= below[pi])) w = lw[li++];
+            else w = below[pi++];
+            if (have) { cur[np++] = pend + w; have = false; }
+            else { pend = w; have = true; }
+          }
+          npk[lev] = np;
+        }
+        uint32_t sel = 2u * (uint32_t)m - 2u;
+        for (int lev = 1; lev <= Lmax; lev++) {
+          const uint64_t *cur = pk + (uint64_t)lev * 256;
+          uint32_t np = npk[lev], li = 0, pi = 0;
+          for (uint32_t r = 0; r < sel; r++) {
+            if (li < (uint32_t)m && (pi >= np || lw[li] <= cur[pi])) li++;
+            else pi++;
+          }
+          xsel[lev] = li;
+          sel = 2u * pi;
+        }
+      }
+      __syncthreads();
+      if (tid < m) {
+        d = 0;
+        for (int lev = 1; lev <= Lmax; lev++) d += (uint32_t)tid < xsel[lev];
+      }
+    }
+    if (tid < m) atomicAdd(&nlen[d], 1u);
+  } else if (m == 1 && tid < m) {
+    d = 1;
+    atomicAdd(&nlen[1], 1u);
+  }
+  __syncthreads();
+
+  // rank assignment: the r-th shortest length goes to the symbol of rank r in
+  // (count descending, symbol ascending) order
+  if (c > 0 && feasible) {
+    uint32_t r = 0;
+    for (int s2 = 0; s2 < A; s2++) {
+      uint64_t c2 = cnt[s2];
+      r += (c2 > c) || (c2 == c && s2 < tid);
+    }
+    uint32_t cum = 0, L = 1;
+    for (; L <= 32; L++) {
+      cum += nlen[L];
+      if (cum > r) break;
+    }
+    len[tid] = (uint8_t)L;
+  }
+  if (tid == 0) {
+    uint64_t code = 0;
+    for (int L = 1; L <= 32; L++) {
+      firstc[L] = (uint32_t)code;
+      code = (code + nlen[L]) << 1;
+    }
+  }
+  __syncthreads();
+  if (tid < A) {
+    uint32_t l = len[tid], code = 0;
+    if (l) {
+      uint32_t k = 0;
+      for (int s2 = 0; s2 < tid; s2++) k += len[s2] == l;
+      code = firstc[l] + k;
+    }
+    I.code_len[tid] = (uint8_t)l;
+    I.code[tid] = code;
+  }
+}
+
+// ---------------------------------------------------------------- offsets
+__device__ __forceinline__ uint64_t warp_sum64(uint64_t v) {
+  #pragma unroll
+  for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+__global__ void __launch_bounds__(256) offsets_kernel(const __grid_constant__ Batch b) {
+  const int A = alphabet_of(b.dtype);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t g = blockIdx.x * 8 + warp;
+  if (g < b.total_chunks) {
+    const Item &I = b.item[find_item(b, g)];
+    const uint32_t c = g - I.chunk0;
+    uint64_t bits = 0;
+    for (int s = lane; s < A; s += 32) bits += (uint64_t)I.chist[(uint64_t)c * A + s] * I.code_len[s];
+    bits = warp_sum64(bits);
+    if (lane == 0) I.cbits[c] = bits;
+  }
+  __shared__ uint32_t last;
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) last = atomicAdd(b.ticket, 1u) == gridDim.x - 1;
+  __syncthreads();
+  if (!last) return;
+  __threadfence();
+  // last CTA: per-tensor exclusive scan of chunk bits -> offsets
+  __shared__ uint64_t wtot[8];
+  for (uint32_t it = 0; it < b.k; it++) {
+    const Item &I = b.item[it];
+    const uint32_t C = I.nchunks;
+    uint32_t *sw = (uint32_t *)I.stream;
+    uint64_t carry = 0;
+    for (uint32_t base = 0; base < C; base += 256) {
+      const uint32_t ci = base + threadIdx.x;
+      uint64_t v = ci < C ? __ldcg(I.cbits + ci) : 0ull;
+      uint64_t x = v;
+      #pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        uint64_t y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+      }
+      if (lane == 31) wtot[warp] = x;
+      __syncthreads();
+      uint64_t pre = 0, tot = 0;
+      for (int w = 0; w < 8; w++) {
+        if (w < warp) pre += wtot[w];
+        tot += wtot[w];
+      }
+      if (ci < C) {
+        uint64_t off = carry + pre + x - v;
+        I.off[ci] = off;
+        sw[off >> 5] = 0u;  // word shared with the previous chunk: cleared for OR
+      }
+      carry += tot;
+      __syncthreads();
+    }
+    if (threadIdx.x == 0) {
+      I.off[C] = carry;
+      if (carry & 31) sw[carry >> 5] = 0u;
+      I.bits_out[0] = carry;
+      if (I.bits_dev) I.bits_dev[0] = carry;
+    }
+  }
+  if (threadIdx.x == 0) *b.ticket = 0u;  // ready for the next call
+}
+
+// ---------------------------------------------------------------- encode
+constexpr int kEncPerThread = 8;                        // values per thread per tile
+constexpr int kEncTile = kThreads * kEncPerThread;       // 4096 values
+constexpr int kRingWords = 8192;                         // 2 tiles of 32-bit codes
+constexpr uint32_t kRingMask = kRingWords - 1;
+
+__device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t *wsum, uint32_t *total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  uint32_t x = v;
+  #pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) wsum[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    uint32_t t = lane < kThreads / 32 ? wsum[lane] : 0u;
+    #pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      uint32_t y = __shfl_up_sync(0xffffffffu, t, o);
+      if (lane >= o) t += y;
+    }
+    if (lane < kThreads / 32) wsum[lane] = t;
+  }
+  __syncthreads();
+  *total = wsum[kThreads / 32 - 1];
+  return (warp ? wsum[warp - 1] : 0u) + x - v;
+}
+
+template <int DT>
+__global__ void __launch_bounds__(kThreads, 2) encode_kernel(const __grid_constant__ Batch b) {
+  constexpr int A = DT == EH_BF16 ? 256 : 16;
+  extern __shared__ uint32_t ring[];  // kRingWords words, code bits in MSB-first order
+  __shared__ uint2 tab[A];            // (code, length)
+  __shared__ uint32_t wsum[kThreads / 32];
+  const uint32_t g = blockIdx.x;
+  const Item &I = b.item[find_item(b, g)];
+  const uint32_t c = g - I.chunk0;
+  const uint64_t i0 = (uint64_t)c * b.chunk_elems;
+  const uint32_t cnt = (uint32_t)min((uint64_t)b.chunk_elems, I.n - i0);
+  const int tid = threadIdx.x;
+  for (int s = tid; s < A; s += kThreads) tab[s] = make_uint2(I.code[s], I.code_len[s]);
+  for (int i = tid; i < kRingWords; i += kThreads) ring[i] = 0u;
+  const uint64_t bit0 = I.off[c], bit1 = I.off[c + 1];
+  uint32_t *gs = (uint32_t *)I.stream;
+  __syncthreads();
+
+  uint64_t tile_base = bit0;           // stream bit where the current tile starts
+  uint64_t wdone = bit0 >> 5;          // first stream word not yet written out
+  for (uint32_t t0 = 0; t0 < cnt; t0 += kEncTile) {
+    const uint32_t idx = t0 + tid * kEncPerThread;
+    uint32_t e[kEncPerThread];
+    uint32_t nvalid = 0;
+    if (DT == EH_BF16) {
+      const uint16_t *in = (const uint16_t *)I.in + i0;
+      if (idx + kEncPerThread <= cnt) {
+        uint4 p = ld_stream(in + idx);
+        uint32_t w[4] = {p.x, p.y, p.z, p.w};
+        #pragma unroll
+        for (int j = 0; j < 4; j++) {
+          e[2 * j] = (w[j] >> 7) & 0xFFu;
+          e[2 * j + 1] = (w[j] >> 23) & 0xFFu;
+        }
+        nvalid = kEncPerThread;
+      } else {
+        #pragma unroll
+        for (int j = 0; j < kEncPerThread; j++) e[j] = idx + j < cnt ? (in[idx + j] >> 7) & 0xFFu : 0u;
+        nvalid = idx < cnt ? cnt - idx : 0;
+      }
+    } else {
+      const uint8_t *in = (const uint8_t *)I.in + i0;
+      if (idx + kEncPerThread <= cnt) {
+        uint2 p = ld_stream8(in + idx);
+        #pragma unroll
+        for (int j = 0; j < 4; j++) {
+          e[j] = (p.x >> (8 * j + 3)) & 0xFu;
+          e[4 + j] = (p.y >> (8 * j + 3)) & 0xFu;
+        }
+        nvalid = kEncPerThread;
+      } else {
+        #pragma unroll
+        for (int j = 0; j < kEncPerThread; j++) e[j] = idx + j < cnt ? (in[idx + j] >> 3) & 0xFu : 0u;
+        nvalid = idx < cnt ? cnt - idx : 0;
+      }
+    }
+    uint2 cl[kEncPerThread];
+    uint32_t mybits = 0;
+    #pragma unroll
+    for (int j = 0; j < kEncPerThread; j++) {
+      cl[j] = tab[e[j]];
+      if ((uint32_t)j >= nvalid) cl[j].y = 0u;
+      mybits += cl[j].y;
+    }
+    uint32_t total;
+    const uint32_t excl = block_excl_scan(mybits, wsum, &total);
+    if (mybits) {
+      // stream the codes through a 64-bit accumulator aligned to the global
+      // word grid; complete words go to the ring with OR (two neighbours may
+      // share a word)
+      uint64_t pos = tile_base + excl;
+      uint64_t w = pos >> 5;
+      uint32_t nb = (uint32_t)(pos & 31);
+      uint64_t acc = 0;
+      #pragma unroll
+      for (int j = 0; j < kEncPerThread; j++) {
+        const uint32_t l = cl[j].y;
+        if (l) {
+          acc |= (uint64_t)cl[j].x << (64 - nb - l);
+          nb += l;
+          if (nb >= 32) {
+            atomicOr(&ring[w & kRingMask], (uint32_t)(acc >> 32));
+            acc <<= 32;
+            nb -= 32;
+            w++;
+          }
+        }
+      }
+      if (nb) atomicOr(&ring[w & kRingMask], (uint32_t)(acc >> 32));
+    }
+    __syncthreads();
+    tile_base += total;
+    const bool last = t0 + kEncTile >= cnt;
+    const uint64_t wend = last ? (bit1 + 31) >> 5 : tile_base >> 5;
+    for (uint64_t wi = wdone + tid; wi < wend; wi += kThreads) {
+      const uint32_t slot = (uint32_t)(wi & kRingMask);
+      const uint32_t val = bswap32(ring[slot]);
+      ring[slot] = 0u;
+      const bool edge = (wi << 5) < bit0 || ((wi + 1) << 5) > bit1;
+      if (edge) atomicOr(gs + wi, val);
+      else gs[wi] = val;
+    }
+    wdone = wend;
+    __syncthreads();
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_hist(const Batch &b, cudaStream_t s) {
+  if (b.total_chunks == 0) return cudaSuccess;
+  if (b.dtype == EH_BF16) hist_kernel<EH_BF16><<<b.total_chunks, kThreads, 0, s>>>(b);
+  else hist_kernel<EH_FP8_E4M3><<<b.total_chunks, kThreads, 0, s>>>(b);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_book(const Batch &b, cudaStream_t s) {
+  book_kernel<<<b.k, 256, 0, s>>>(b);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_offsets(const Batch &b, cudaStream_t s) {
+  uint32_t grid = (b.total_chunks + 7) / 8;
+  if (grid == 0) grid = 1;  // the last CTA still writes off[0] = 0 and the bit totals
+  offsets_kernel<<<grid, 256, 0, s>>>(b);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_encode(const Batch &b, cudaStream_t s) {
+  if (b.total_chunks == 0) return cudaSuccess;
+  const size_t smem = kRingWords * sizeof(uint32_t);
+  if (b.dtype == EH_BF16) encode_kernel<EH_BF16><<<b.total_chunks, kThreads, smem, s>>>(b);
+  else encode_kernel<EH_FP8_E4M3><<<b.total_chunks, kThreads, smem, s>>>(b);
+  return cudaGetLastError();
+}
+
+}  // namespace eh

@@ -1,0 +1,116 @@
+// eh_internal.cuh -- shared device-side definitions of libexphuff.
+//
+// Launch descriptors, workspace layout, status flags and small device helpers
+// used by the compress and decompress kernels.  The public interface is
+// include/exphuff.h.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/exphuff.h"
+
+namespace eh {
+
+constexpr int kThreads = 512;           // threads per CTA of the chunk kernels
+constexpr int kMaxChunk = 65536;        // largest chunk (elements)
+constexpr int kNumSub = 8;              // second-level decode tables per codebook
+constexpr int kStageBytes = 32 * 1024;  // shared-memory window for one chunk's stream
+
+// status word flags (bitwise OR of everything a call observed)
+constexpr uint32_t kFlagCorrupt = 1u;
+constexpr uint32_t kFlagInfeasible = 2u;
+constexpr uint32_t kFlagTimeout = 4u;
+
+__host__ __device__ inline int alphabet_of(int dtype) { return dtype == EH_BF16 ? 256 : 16; }
+
+// Per-tensor part of a launch.
+struct Item {
+  const void *in;          // compress: raw values
+  void *out;               // decompress: output values
+  uint64_t n;              // element count of the tensor
+  uint64_t elem0;          // decompress_chunks: element index of out[0]
+  uint32_t chunk0;         // global index of this tensor's first chunk in the launch
+  uint32_t nchunks;        // chunks of this tensor processed by the launch
+  uint32_t first_chunk;    // tensor-local index of the first processed chunk
+  uint32_t total_chunks;   // chunks of the whole tensor
+  uint8_t *code_len;       // [A]
+  uint32_t *code;          // [A]
+  uint64_t *off;           // [total_chunks + 1]
+  uint8_t *stream;         // exp_stream
+  uint64_t stream_cap;     // bytes
+  uint8_t *sm;             // sign_mant
+  // workspace views
+  uint64_t *counts;        // compress: [256] global histogram
+  uint32_t *chist;         // compress: [total_chunks][A] per-chunk histograms
+  uint64_t *cbits;         // compress: [total_chunks] code bits per chunk
+  uint64_t *pm_scratch;    // compress: package-merge package weights
+  uint64_t *bits_out;      // compress: total bits (workspace copy)
+  uint64_t *bits_dev;      // compress: optional caller copy (may be null)
+  void *lut;               // decompress: DecodeTables
+};
+
+struct Batch {
+  Item item[EH_MAX_BATCH];
+  uint32_t k;
+  uint32_t total_chunks;   // sum of item[i].nchunks
+  uint32_t chunk_elems;
+  int32_t dtype;
+  uint32_t max_code_len;
+  uint32_t *status;        // workspace status word
+  uint32_t *ticket;        // workspace counter for last-block-done patterns
+};
+
+// Item that owns global chunk g (linear scan; k <= 16).
+__device__ __forceinline__ int find_item(const Batch &b, uint32_t g) {
+  int i = 0;
+  #pragma unroll 1
+  while (i + 1 < (int)b.k && g >= b.item[i + 1].chunk0) i++;
+  return i;
+}
+
+__device__ __forceinline__ uint32_t bswap32(uint32_t x) { return __byte_perm(x, 0, 0x0123); }
+
+__device__ __forceinline__ void set_status(uint32_t *status, uint32_t flag) {
+  atomicOr(status, flag);
+}
+
+// Decode tables for one codebook, built by the table kernel into the
+// workspace and copied to shared memory by each decoding CTA.
+//
+// First level, indexed by the next 8 stream bits.  u64 entry:
+//   bits  0..31  up to four decoded symbols, 8 bits each (first in bits 0..7)
+//   bits 32..35  length of the first code if it is <= 8 bits, else 0
+//   bits 36..39  bits consumed by the `cnt` complete codes in the 8 bits
+//   bits 40..42  cnt: complete codes inside the 8 bits (0..4)
+//   bits 48..55  second-level table of this prefix (0xFF: none -> search)
+// Second level, indexed by the 8 bits after the prefix.  u32 entry:
+//   bits 0..7 symbol, bits 8..13 code length 9..16 (0: longer -> search).
+// The search path handles any length up to 32 with the canonical limits.
+struct DecodeTables {
+  uint64_t l1[256];
+  uint32_t sub[kNumSub][256];
+  uint64_t lim[33];        // (first[L] + count[L]) << (32 - L): left-justified limits
+  uint32_t first[33];      // first canonical code of length L
+  uint32_t base[33];       // index in `sorted` of the first code of length L
+  uint8_t sorted[256];     // symbols in (length, symbol) order
+  uint32_t gcd;            // gcd of the code lengths in use
+  uint32_t maxlen;
+  uint32_t nsym;
+  uint32_t err;            // nonzero: codebook invalid
+};
+
+constexpr uint64_t kLutBytes = (sizeof(DecodeTables) + 255) & ~uint64_t(255);
+
+__host__ __device__ inline uint64_t align256(uint64_t x) { return (x + 255) & ~uint64_t(255); }
+
+// ---- host-side launch wrappers (defined in the .cu files)
+cudaError_t launch_hist(const Batch &b, cudaStream_t s);
+cudaError_t launch_book(const Batch &b, cudaStream_t s);
+cudaError_t launch_offsets(const Batch &b, cudaStream_t s);
+cudaError_t launch_encode(const Batch &b, cudaStream_t s);
+cudaError_t launch_tables(const Batch &b, cudaStream_t s);
+cudaError_t launch_decode(const Batch &b, cudaStream_t s, int num_sms);
+cudaError_t configure_decode();  // once per device, before the first decode launch
+
+}  // namespace eh

@@ -1,0 +1,293 @@
+"""Python binding of libexphuff (include/exphuff.h).
+
+Argument marshalling only: every step of compression and decompression runs
+in the library's CUDA kernels.  PyTorch provides device memory and streams.
+The library must have been built (``python -m exponent_entropy_coding_b200.build``
+or ``__graft_entry__.build()``); if it is missing, loading raises instead of
+falling back to anything else.
+"""
+import ctypes as C
+import os
+from dataclasses import dataclass
+from typing import List, Optional, Sequence
+
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libexphuff.so")
+
+EH_BF16 = 0
+EH_FP8_E4M3 = 1
+EH_DEFAULT_CHUNK_ELEMS = 65536
+EH_MAX_CODE_LEN = 32
+EH_MAX_BATCH = 16
+
+STATUS = {0: "EH_OK", 1: "EH_ERR_INVALID_ARG", 2: "EH_ERR_UNSUPPORTED", 3: "EH_ERR_INFEASIBLE",
+          4: "EH_ERR_CUDA", 5: "EH_ERR_CORRUPT", 6: "EH_ERR_TIMEOUT", 7: "EH_ERR_NOMEM"}
+EH_OK, EH_ERR_INVALID_ARG, EH_ERR_UNSUPPORTED, EH_ERR_INFEASIBLE = 0, 1, 2, 3
+EH_ERR_CUDA, EH_ERR_CORRUPT, EH_ERR_TIMEOUT, EH_ERR_NOMEM = 4, 5, 6, 7
+
+EXPORTED = ["eh_plan", "eh_compress_bound", "eh_compress_batch_workspace", "eh_compress",
+            "eh_compress_batch", "eh_decompress_workspace", "eh_decompress", "eh_decompress_batch",
+            "eh_decompress_chunks", "eh_get_status", "eh_status_str", "eh_version"]
+
+
+class EhError(RuntimeError):
+    def __init__(self, code, what=""):
+        self.code = code
+        super().__init__(f"{what}: {STATUS.get(code, code)}")
+
+
+class eh_plan_t(C.Structure):
+    _fields_ = [("dtype", C.c_int32), ("chunk_elems", C.c_uint32),
+                ("max_code_len", C.c_uint32), ("reserved", C.c_uint32)]
+
+
+class eh_compressed_t(C.Structure):
+    _fields_ = [("dtype", C.c_int32), ("n_chunks", C.c_uint32), ("n", C.c_uint64),
+                ("code_len", C.c_void_p), ("code", C.c_void_p), ("chunk_bit_off", C.c_void_p),
+                ("exp_stream", C.c_void_p), ("exp_stream_cap", C.c_uint64),
+                ("sign_mant", C.c_void_p), ("exp_stream_bits", C.c_uint64)]
+
+
+_lib = None
+
+
+def lib():
+    """Loads libexphuff.so (raises if it was not built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"libexphuff.so not built ({LIB_PATH}); run "
+                               "python -m exponent_entropy_coding_b200.build")
+        L = C.CDLL(LIB_PATH)
+        P, u64, i32, u32, vp = C.POINTER, C.c_uint64, C.c_int32, C.c_uint32, C.c_void_p
+        sig = {
+            "eh_plan": [P(eh_plan_t), i32, u32, u32],
+            "eh_compress_bound": [P(eh_plan_t), u64, P(u64), P(u64), P(u64)],
+            "eh_compress_batch_workspace": [P(eh_plan_t), C.c_int, P(u64), P(u64)],
+            "eh_compress": [P(eh_plan_t), vp, u64, P(eh_compressed_t), vp, u64, vp],
+            "eh_compress_batch": [P(eh_plan_t), C.c_int, P(vp), P(eh_compressed_t), vp, vp, u64, vp],
+            "eh_decompress_workspace": [P(eh_plan_t), C.c_int, P(u64)],
+            "eh_decompress": [P(eh_plan_t), P(eh_compressed_t), vp, vp, u64, vp],
+            "eh_decompress_batch": [P(eh_plan_t), C.c_int, P(eh_compressed_t), P(vp), vp, u64, vp],
+            "eh_decompress_chunks": [P(eh_plan_t), P(eh_compressed_t), u32, u32, vp, vp, u64, vp],
+            "eh_get_status": [vp, vp],
+            "eh_status_str": [C.c_int],
+            "eh_version": [],
+        }
+        for name, args in sig.items():
+            f = getattr(L, name)
+            f.argtypes = args
+            f.restype = C.c_char_p if name in ("eh_status_str", "eh_version") else C.c_int
+        _lib = L
+    return _lib
+
+
+def _check(rc, what):
+    if rc != EH_OK:
+        raise EhError(rc, what)
+
+
+def _stream_ptr(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return C.c_void_p(s.cuda_stream)
+
+
+def dtype_code(torch_dtype) -> int:
+    if torch_dtype in (torch.bfloat16, torch.int16, torch.uint16):
+        return EH_BF16
+    if torch_dtype in (torch.float8_e4m3fn, torch.uint8):
+        return EH_FP8_E4M3
+    raise ValueError(f"unsupported dtype {torch_dtype}")
+
+
+def alphabet(dtype: int) -> int:
+    return 256 if dtype == EH_BF16 else 16
+
+
+def plan(dtype: int, chunk_elems: int = 0, max_code_len: int = 0) -> eh_plan_t:
+    p = eh_plan_t()
+    _check(lib().eh_plan(C.byref(p), dtype, chunk_elems, max_code_len), "eh_plan")
+    return p
+
+
+def compress_bound(p: eh_plan_t, n: int):
+    sc, sm, ws = C.c_uint64(), C.c_uint64(), C.c_uint64()
+    _check(lib().eh_compress_bound(C.byref(p), n, C.byref(sc), C.byref(sm), C.byref(ws)),
+           "eh_compress_bound")
+    return sc.value, sm.value, ws.value
+
+
+def compress_batch_workspace(p: eh_plan_t, ns: Sequence[int]) -> int:
+    arr = (C.c_uint64 * len(ns))(*ns)
+    out = C.c_uint64()
+    _check(lib().eh_compress_batch_workspace(C.byref(p), len(ns), arr, C.byref(out)),
+           "eh_compress_batch_workspace")
+    return out.value
+
+
+def decompress_workspace(p: eh_plan_t, k: int = 1) -> int:
+    out = C.c_uint64()
+    _check(lib().eh_decompress_workspace(C.byref(p), k, C.byref(out)), "eh_decompress_workspace")
+    return out.value
+
+
+@dataclass
+class Compressed:
+    """Device arrays of one compressed tensor (torch tensors own the memory)."""
+    dtype: int
+    n: int
+    code_len: torch.Tensor       # uint8[A]
+    code: torch.Tensor           # int32[A] (uint32 values)
+    chunk_bit_off: torch.Tensor  # int64[C+1] (uint64 values)
+    exp_stream: torch.Tensor     # uint8[cap]
+    sign_mant: torch.Tensor      # uint8[n or ceil(n/2)]
+    exp_stream_bits: int = 0
+
+    @property
+    def n_chunks(self) -> int:
+        return self.chunk_bit_off.numel() - 1
+
+    def stream_bytes(self) -> int:
+        return (self.exp_stream_bits + 7) // 8
+
+    def compressed_bytes(self) -> int:
+        """Stored size: exponent stream + sign/mantissa + offsets + codebook."""
+        return (self.stream_bytes() + self.sign_mant.numel() + 8 * self.chunk_bit_off.numel()
+                + self.code_len.numel())
+
+    def struct(self) -> eh_compressed_t:
+        s = eh_compressed_t()
+        s.dtype = self.dtype
+        s.n_chunks = self.n_chunks
+        s.n = self.n
+        s.code_len = self.code_len.data_ptr()
+        s.code = self.code.data_ptr()
+        s.chunk_bit_off = self.chunk_bit_off.data_ptr()
+        s.exp_stream = self.exp_stream.data_ptr() if self.exp_stream.numel() else None
+        s.exp_stream_cap = self.exp_stream.numel()
+        s.sign_mant = self.sign_mant.data_ptr() if self.sign_mant.numel() else None
+        s.exp_stream_bits = self.exp_stream_bits
+        return s
+
+
+def alloc_compressed(p: eh_plan_t, n: int, device) -> Compressed:
+    cap, smb, _ = compress_bound(p, n)
+    A = alphabet(p.dtype)
+    nc = -(-n // p.chunk_elems)
+    dev = torch.device(device)
+    return Compressed(
+        dtype=p.dtype, n=n,
+        code_len=torch.zeros(A, dtype=torch.uint8, device=dev),
+        code=torch.zeros(A, dtype=torch.int32, device=dev),
+        chunk_bit_off=torch.zeros(nc + 1, dtype=torch.int64, device=dev),
+        exp_stream=torch.empty(cap if n else 0, dtype=torch.uint8, device=dev),
+        sign_mant=torch.empty(smb, dtype=torch.uint8, device=dev))
+
+
+def _raw(x: torch.Tensor) -> torch.Tensor:
+    if not x.is_cuda:
+        raise ValueError("tensor must be on a CUDA device")
+    return x.contiguous()
+
+
+def compress_batch(p: eh_plan_t, xs: List[torch.Tensor], outs: List[Compressed], workspace: torch.Tensor,
+                   bits_dev: Optional[torch.Tensor] = None, stream=None):
+    """Calls eh_compress_batch on device tensors; fills outs[i].exp_stream_bits
+    unless bits_dev (int64[k] on the device) is given."""
+    k = len(xs)
+    xs = [_raw(x) for x in xs]
+    ins = (C.c_void_p * k)(*[x.data_ptr() if x.numel() else None for x in xs])
+    structs = (eh_compressed_t * k)(*[o.struct() for o in outs])
+    rc = lib().eh_compress_batch(C.byref(p), k, ins, structs,
+                                 C.c_void_p(bits_dev.data_ptr()) if bits_dev is not None else None,
+                                 C.c_void_p(workspace.data_ptr()), workspace.numel(), _stream_ptr(stream))
+    _check(rc, "eh_compress_batch")
+    if bits_dev is None:
+        for o, s in zip(outs, structs):
+            o.exp_stream_bits = s.exp_stream_bits
+    return outs
+
+
+def compress(x: torch.Tensor, p: Optional[eh_plan_t] = None, workspace: Optional[torch.Tensor] = None,
+             stream=None) -> Compressed:
+    """Compresses one BF16 / FP8 E4M3 tensor (or its raw uint16 / uint8 bits)."""
+    x = _raw(x)
+    if p is None:
+        p = plan(dtype_code(x.dtype))
+    n = x.numel()
+    out = alloc_compressed(p, n, x.device)
+    if workspace is None:
+        workspace = torch.empty(compress_bound(p, n)[2], dtype=torch.uint8, device=x.device)
+    s = out.struct()
+    rc = lib().eh_compress(C.byref(p), C.c_void_p(x.data_ptr()) if n else None, n, C.byref(s),
+                           C.c_void_p(workspace.data_ptr()), workspace.numel(), _stream_ptr(stream))
+    _check(rc, "eh_compress")
+    out.exp_stream_bits = s.exp_stream_bits
+    return out
+
+
+def _elem_dtype(dtype):
+    return torch.int16 if dtype == EH_BF16 else torch.uint8
+
+
+def decompress_batch(p: eh_plan_t, cs: List[Compressed], outs: List[torch.Tensor], workspace: torch.Tensor,
+                     stream=None):
+    k = len(cs)
+    structs = (eh_compressed_t * k)(*[c.struct() for c in cs])
+    optrs = (C.c_void_p * k)(*[o.data_ptr() if o.numel() else None for o in outs])
+    rc = lib().eh_decompress_batch(C.byref(p), k, structs, optrs, C.c_void_p(workspace.data_ptr()),
+                                   workspace.numel(), _stream_ptr(stream))
+    _check(rc, "eh_decompress_batch")
+    return outs
+
+
+def decompress(c: Compressed, p: Optional[eh_plan_t] = None, out: Optional[torch.Tensor] = None,
+               workspace: Optional[torch.Tensor] = None, stream=None, check: bool = True) -> torch.Tensor:
+    """Decompresses into a raw-bits tensor (int16 for BF16, uint8 for FP8);
+    with check=True waits for the stream and raises on a data error."""
+    dev = c.code_len.device
+    if p is None:
+        p = plan(c.dtype)
+    if out is None:
+        out = torch.empty(c.n, dtype=_elem_dtype(c.dtype), device=dev)
+    if workspace is None:
+        workspace = torch.empty(decompress_workspace(p, 1), dtype=torch.uint8, device=dev)
+    s = c.struct()
+    rc = lib().eh_decompress(C.byref(p), C.byref(s), C.c_void_p(out.data_ptr()) if c.n else None,
+                             C.c_void_p(workspace.data_ptr()), workspace.numel(), _stream_ptr(stream))
+    _check(rc, "eh_decompress")
+    if check:
+        _check(get_status(workspace, stream), "eh_decompress (device status)")
+    return out
+
+
+def decompress_chunks(c: Compressed, first: int, count: int, p: Optional[eh_plan_t] = None,
+                      out: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                      stream=None, check: bool = True) -> torch.Tensor:
+    dev = c.code_len.device
+    if p is None:
+        p = plan(c.dtype)
+    K = p.chunk_elems
+    n_out = max(0, min(c.n, (first + count) * K) - first * K)
+    if out is None:
+        out = torch.empty(n_out, dtype=_elem_dtype(c.dtype), device=dev)
+    if workspace is None:
+        workspace = torch.empty(decompress_workspace(p, 1), dtype=torch.uint8, device=dev)
+    s = c.struct()
+    rc = lib().eh_decompress_chunks(C.byref(p), C.byref(s), first, count,
+                                    C.c_void_p(out.data_ptr()) if n_out else None,
+                                    C.c_void_p(workspace.data_ptr()), workspace.numel(), _stream_ptr(stream))
+    _check(rc, "eh_decompress_chunks")
+    if check:
+        _check(get_status(workspace, stream), "eh_decompress_chunks (device status)")
+    return out
+
+
+def get_status(workspace: torch.Tensor, stream=None) -> int:
+    return lib().eh_get_status(C.c_void_p(workspace.data_ptr()), _stream_ptr(stream))
+
+
+def version() -> str:
+    return lib().eh_version().decode()

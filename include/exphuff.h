@@ -1,0 +1,189 @@
+/*
+ * exphuff.h -- libexphuff: lossless split-exponent Huffman codec for BF16 and
+ * FP8 E4M3 tensors on NVIDIA B200 (sm_100a).
+ *
+ * What the codec computes (page title, then section):
+ *  - "70% Size, 100% Accuracy: Lossless LLM Compression for Efficient GPU
+ *    Inference via Dynamic-Length Float" (DFloat11 article), section
+ *    "方法介绍": a Huffman code is built from the distribution of exponent
+ *    values; the exponent codes are tightly bit-packed into a byte array
+ *    (EncodedExponent) and the sign and mantissa bits are kept raw in a
+ *    separate byte array (PackedSignMantissa).  Decompression rebuilds the
+ *    exact original values on the GPU.
+ *  - "Lossless Compression of Neural Network Components: Weights,
+ *    Checkpoints, and K/V Caches in Low-Precision Formats" (paper summary),
+ *    sections "方法详解" and "实验设计": exponent and mantissa are split, the
+ *    exponent is Huffman-coded, FP8 is covered, and every tensor is coded in
+ *    fixed-size chunks.
+ *  - "ZipFloat: An Ultra-fast and Lossless Floating-Point Compressor for LLM
+ *    Inference Systems", section 2.1: the BF16 exponent field is the exponent
+ *    plus 127.
+ *
+ * Format (one compressed tensor of n elements, chunk size K, C = ceil(n/K)):
+ *  - exponent field e: BF16 bits 14..7 (x>>7 & 0xFF, alphabet 256); FP8 E4M3
+ *    bits 6..3 (x>>3 & 0xF, alphabet 16);
+ *  - code_len[A]: Huffman code lengths, 0 for absent symbols, at most
+ *    max_code_len (<= 32).  Minimum-variance Huffman; package-merge when the
+ *    Huffman depth exceeds the limit; lengths dealt in ascending order to the
+ *    symbols sorted by (count descending, symbol ascending).  A tensor with one
+ *    distinct exponent gets length 1 (code "0");
+ *  - code[A]: canonical codes in (length, symbol) order (RFC 1951 §3.2.2);
+ *  - exp_stream: the codes of all elements in element order, MSB-first (bit
+ *    p is bit 7-(p&7) of byte p>>3), chunks back to back with no padding, the
+ *    last byte zero-padded; ceil(exp_stream_bits/8) meaningful bytes;
+ *  - chunk_bit_off[C+1]: bit offset of each chunk's first code;
+ *    chunk_bit_off[C] = exp_stream_bits;
+ *  - sign_mant: BF16 one byte (s<<7)|m7 per element; FP8 one nibble
+ *    (s<<3)|m3 per element, element 2i in the low nibble of byte i, the unused
+ *    high nibble of an odd-length tensor zero.
+ *
+ * Memory: every pointer passed to a compress/decompress call is a DEVICE
+ * pointer on the current CUDA device, allocated and owned by the CALLER.  The
+ * library allocates nothing on these paths; it needs a caller-provided
+ * workspace whose size the *_workspace / *_bound queries return.  Device
+ * pointers must be 16-byte aligned.  Streams are passed as `void *` holding a
+ * cudaStream_t (NULL = legacy default stream).
+ *
+ * Errors: argument errors are returned immediately (nothing is launched).
+ * Data errors found on the GPU (a corrupt stream, an invalid codebook) are
+ * recorded in a status word inside the workspace; eh_get_status() waits for
+ * the stream and returns it.  Kernels never trap and every wait in them is
+ * bounded.  Functions are thread-safe as long as concurrent calls use
+ * distinct workspaces.
+ */
+#ifndef EXPHUFF_H
+#define EXPHUFF_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define EH_API __attribute__((visibility("default")))
+#else
+#define EH_API
+#endif
+
+#define EH_DEFAULT_CHUNK_ELEMS 65536u /* elements per chunk (one K/V page)   */
+#define EH_MAX_CODE_LEN 32u           /* longest code the format allows     */
+#define EH_MAX_BATCH 16               /* tensors per batched launch         */
+
+typedef enum { EH_BF16 = 0, EH_FP8_E4M3 = 1 } eh_dtype;
+
+typedef enum {
+  EH_OK = 0,
+  EH_ERR_INVALID_ARG = 1, /* bad pointer, size, alignment or capacity      */
+  EH_ERR_UNSUPPORTED = 2, /* dtype / chunk size / limit not supported      */
+  EH_ERR_INFEASIBLE = 3,  /* more distinct exponents than 2^max_code_len   */
+  EH_ERR_CUDA = 4,        /* a CUDA runtime call failed                    */
+  EH_ERR_CORRUPT = 5,     /* compressed data or codebook inconsistent      */
+  EH_ERR_TIMEOUT = 6,     /* a bounded wait inside a kernel gave up        */
+  EH_ERR_NOMEM = 7        /* workspace smaller than required               */
+} eh_status;
+
+/* Fixes the format: dtype, chunk size, length limit. */
+typedef struct {
+  int32_t dtype;         /* eh_dtype                                        */
+  uint32_t chunk_elems;  /* multiple of 1024 in [1024, 65536]               */
+  uint32_t max_code_len; /* 1..32                                           */
+  uint32_t reserved;     /* 0                                               */
+} eh_plan_t;
+
+/* One compressed tensor.  The caller allocates the device arrays (sizes from
+ * eh_compress_bound); eh_compress fills them, n_chunks and exp_stream_bits. */
+typedef struct {
+  int32_t dtype;            /* eh_dtype, must match the plan                 */
+  uint32_t n_chunks;        /* ceil(n / chunk_elems)                         */
+  uint64_t n;               /* element count                                 */
+  uint8_t *code_len;        /* device, [A] (A = 256 BF16, 16 FP8)            */
+  uint32_t *code;           /* device, [A]                                   */
+  uint64_t *chunk_bit_off;  /* device, [n_chunks + 1]                        */
+  uint8_t *exp_stream;      /* device, exp_stream_cap bytes                  */
+  uint64_t exp_stream_cap;  /* bytes; >= eh_compress_bound's stream_cap      */
+  uint8_t *sign_mant;       /* device, n (BF16) or ceil(n/2) (FP8) bytes     */
+  uint64_t exp_stream_bits; /* total code bits (host copy)                   */
+} eh_compressed_t;
+
+/* Fills *plan.  chunk_elems = 0 selects 65536; max_code_len = 0 selects 32.
+ * Returns EH_ERR_UNSUPPORTED for other chunk sizes or limits. */
+EH_API eh_status eh_plan(eh_plan_t *plan, int32_t dtype, uint32_t chunk_elems,
+                  uint32_t max_code_len);
+
+/* Sizes for compressing one tensor of n elements: stream_cap = bytes for
+ * exp_stream (worst case n*max_code_len bits, rounded up to 16 bytes, plus
+ * 16 bytes that the decoder may read past the last code), sm_bytes = bytes
+ * for sign_mant, workspace_bytes = device workspace for eh_compress.
+ * Any output pointer may be NULL. */
+EH_API eh_status eh_compress_bound(const eh_plan_t *plan, uint64_t n,
+                            uint64_t *stream_cap, uint64_t *sm_bytes,
+                            uint64_t *workspace_bytes);
+
+/* Workspace for eh_compress_batch over k tensors of ns[i] elements. */
+EH_API eh_status eh_compress_batch_workspace(const eh_plan_t *plan, int k,
+                                      const uint64_t *ns,
+                                      uint64_t *workspace_bytes);
+
+/* Compresses one tensor (steps: split + histogram + sign/mantissa pack,
+ * codebook, chunk offsets, encode).  `in` holds n raw BF16 (uint16) or FP8
+ * (uint8) values.  `out` is a host struct whose dtype, n and device pointers
+ * the caller has set; the call writes the device arrays, out->n_chunks and
+ * out->exp_stream_bits.  Waits for `stream` once, to return the bit count. */
+EH_API eh_status eh_compress(const eh_plan_t *plan, const void *in, uint64_t n,
+                      eh_compressed_t *out, void *workspace,
+                      uint64_t workspace_bytes, void *stream);
+
+/* Compresses k <= EH_MAX_BATCH tensors with one launch per step, one
+ * codebook per tensor.  ins[i] has outs[i].n elements.  If bits_dev is NULL
+ * the call waits for the stream and fills outs[i].exp_stream_bits; otherwise
+ * it writes the k bit counts to the device array bits_dev[k] and returns
+ * without waiting (outs[i].exp_stream_bits is then left untouched). */
+EH_API eh_status eh_compress_batch(const eh_plan_t *plan, int k,
+                            const void *const *ins, eh_compressed_t *outs,
+                            uint64_t *bits_dev, void *workspace,
+                            uint64_t workspace_bytes, void *stream);
+
+/* Workspace for decompressing up to k tensors in one call. */
+EH_API eh_status eh_decompress_workspace(const eh_plan_t *plan, int k,
+                                  uint64_t *workspace_bytes);
+
+/* Rebuilds the n original values into out (device, n*elem_size bytes).
+ * Fully stream-ordered, no host wait; data errors go to the status word. */
+EH_API eh_status eh_decompress(const eh_plan_t *plan, const eh_compressed_t *c,
+                        void *out, void *workspace, uint64_t workspace_bytes,
+                        void *stream);
+
+/* Block-at-a-time decompression (the DFloat11 article, "方法介绍" and
+ * "消融研究": a whole transformer block is decompressed in one go): k <=
+ * EH_MAX_BATCH tensors, one launch over all of their chunks. */
+EH_API eh_status eh_decompress_batch(const eh_plan_t *plan, int k,
+                              const eh_compressed_t *cs, void *const *outs,
+                              void *workspace, uint64_t workspace_bytes,
+                              void *stream);
+
+/* Decompresses chunks [first, first+count) of one tensor (e.g. K/V pages of
+ * 64 tokens x 8 heads x 128 dims = 65,536 values).  out receives elements
+ * [first*K, min(n, (first+count)*K)). */
+EH_API eh_status eh_decompress_chunks(const eh_plan_t *plan, const eh_compressed_t *c,
+                               uint32_t first, uint32_t count, void *out,
+                               void *workspace, uint64_t workspace_bytes,
+                               void *stream);
+
+/* Waits for `stream` and returns the status word of `workspace`: EH_OK,
+ * EH_ERR_CORRUPT, EH_ERR_INFEASIBLE or EH_ERR_TIMEOUT.  Every compress or
+ * decompress call resets the word when it starts, so it describes the most
+ * recent call that used this workspace. */
+EH_API eh_status eh_get_status(void *workspace, void *stream);
+
+/* Static description of a status code. */
+EH_API const char *eh_status_str(eh_status s);
+
+/* Library version string, e.g. "libexphuff 0.1 sm_100a". */
+EH_API const char *eh_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* EXPHUFF_H */
