@@ -1,0 +1,355 @@
+"""Benchmark of the split-exponent Huffman codec on one Llama-3.1-8B block.
+
+One step = compress the block's seven BF16 weight matrices (one codebook per
+matrix, one batched call) and decompress the whole block back in one batched
+call (block-at-a-time, as in the DFloat11 article's "方法介绍").  `value` is
+BF16 bytes encoded plus BF16 bytes decoded per second, over all ranks (each
+rank codes its own block: weak scaling, no collective on the data path).
+
+python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+--impl reference times the CPU oracle (single-threaded C++) on the host on a
+bounded sample of the same workload, with the same metric.
+"""
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "exhuff decode & encode GB/s (BF16 bytes) on 218M-param block; % HBM; size ratio"
+WORKLOAD = "llama8b_block"
+FALLBACK_HBM_GBS = 6650.0
+
+# DRAM traffic per decode launch on the full block, from one ncu capture
+# (dram__bytes_read.sum + dram__bytes_write.sum), valid only for the decoder
+# source it was taken on.
+DECODE_TRAFFIC = {"bytes": None, "source_sha": None}
+
+
+def decoder_source_sha():
+    h = hashlib.sha256()
+    for f in ("eh_decompress.cu", "eh_internal.cuh"):
+        with open(os.path.join(ROOT, "exponent_entropy_coding_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def hbm_peak():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons during the timed region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, ValueError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for l in getattr(self, "lines", []):
+            f = [x.strip() for x in l.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+            except ValueError:
+                continue
+            for name, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def run_reference(args):
+    """The CPU oracle on the host cores, on a bounded sample of the workload."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    from exponent_entropy_coding_b200 import synth
+    from oracle import ehref
+    items = synth.llama8b_block(seed=2, scale=1, count=2)
+    sample = items[1][1]           # k_proj, 1024x4096 BF16 = 4,194,304 values
+    nbytes = sample.size * 2
+
+    def step():
+        c = ehref.compress(ehref.BF16, sample)
+        y = ehref.decompress(c)
+        return c, y
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        c, y = step()
+    dt = (time.perf_counter() - t0) / args.steps
+    assert np.array_equal(y, sample)
+    v = 2 * nbytes / dt / 1e9
+    desc = "oracle compress+decompress of k_proj (1024x4096 BF16, 8.4 MB) per step"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": v, "unit": "GB/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "u16",
+        "data": "synthetic", "config": {"workload": "llama8b_block (k_proj sample)",
+                                        "dims": "1024x4096", "threads": 1},
+        "cpu_baseline": {"value": v, "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": desc},
+        "e2e": {"value": v, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "size_ratio": (c.stream.size + c.sign_mant.size + 8 * c.chunk_bit_off.size + 256) / nbytes,
+    }
+    print(json.dumps(line))
+    return 0
+
+
+def cpu_baseline_oracle(items, budget_s=12.0):
+    """Single-threaded oracle round trips over the block's matrices until the
+    time budget is used (at least one matrix)."""
+    from oracle import ehref
+    done_bytes, t0, names = 0, time.perf_counter(), []
+    for name, x in items:
+        c = ehref.compress(ehref.BF16, x)
+        y = ehref.decompress(c)
+        assert np.array_equal(y, x)
+        done_bytes += 2 * x.size * 2
+        names.append(name)
+        if time.perf_counter() - t0 > budget_s:
+            break
+    dt = time.perf_counter() - t0
+    return {"value": done_bytes / dt / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": f"one compress+decompress of {'+'.join(names)} ({done_bytes // 2 / 1e6:.1f} MB BF16)"
+                      f" on one host core, {dt:.1f} s"}
+
+
+def run_ncu_case():
+    """Small case for profiler captures: gate_proj alone (117 MB of BF16, more
+    than the 126 MB L2 once its compressed form is counted), compressed once
+    and decompressed once: three codec kernel launches that matter (hist,
+    encode, decode)."""
+    import torch
+
+    from exponent_entropy_coding_b200 import exphuff as eh
+    from exponent_entropy_coding_b200 import synth
+    rng = np.random.default_rng(2)
+    x = synth.student_t_bf16((14336, 4096), rng).reshape(-1)
+    t = torch.from_numpy(x.view(np.int16)).cuda()
+    p = eh.plan(eh.EH_BF16)
+    c = eh.compress(t, p)
+    y = eh.decompress(c, p)
+    torch.cuda.synchronize()
+    assert torch.equal(y, t)
+    print(json.dumps({"case": "gate_proj 14336x4096", "bits": c.exp_stream_bits,
+                      "size_ratio": c.compressed_bytes() / (2 * x.size)}))
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--ncu-case", action="store_true",
+                    help="one compress + one decompress of gate_proj (14336x4096), for ncu captures")
+    args = ap.parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+    if args.ncu_case:
+        return run_ncu_case()
+
+    import torch
+    import torch.distributed as dist
+
+    from exponent_entropy_coding_b200 import exphuff as eh
+    from exponent_entropy_coding_b200 import synth
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300))
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream()
+
+    items = synth.llama8b_block(seed=2, scale=1)
+    ns = [x.size for _, x in items]
+    in_bytes = 2 * sum(ns)
+    xs_host = [torch.from_numpy(x.view(np.int16)).pin_memory() for _, x in items]
+    xs = [h.to(dev) for h in xs_host]
+    p = eh.plan(eh.EH_BF16)
+    outs = [eh.alloc_compressed(p, n, dev) for n in ns]
+    ys = [torch.empty_like(x) for x in xs]
+    wsc = torch.empty(eh.compress_batch_workspace(p, ns), dtype=torch.uint8, device=dev)
+    wsd = torch.empty(eh.decompress_workspace(p, len(xs)), dtype=torch.uint8, device=dev)
+    bits = torch.zeros(len(xs), dtype=torch.int64, device=dev)
+
+    # first pass: exactness and sizes
+    eh.compress_batch(p, xs, outs, wsc)
+    eh.decompress_batch(p, outs, ys, wsd)
+    assert eh.get_status(wsd) == eh.EH_OK
+    assert all(torch.equal(x, y) for x, y in zip(xs, ys)), "round trip mismatch"
+    stream_bytes = sum(o.stream_bytes() for o in outs)
+    comp_bytes = sum(o.compressed_bytes() for o in outs)
+    sm_bytes = sum(o.sign_mant.numel() for o in outs)
+    off_bytes = sum(8 * o.chunk_bit_off.numel() for o in outs)
+
+    n_ev = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(n_ev)]
+
+    def step(i=None):
+        if i is not None:
+            ev[i][0].record(stream)
+        eh.compress_batch(p, xs, outs, wsc, bits_dev=bits)
+        if i is not None:
+            ev[i][1].record(stream)
+        eh.decompress_batch(p, outs, ys, wsd)
+        if i is not None:
+            ev[i][2].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        t_start.record(stream)
+        for i in range(args.steps):
+            step(i)
+        t_end.record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    ms = t_start.elapsed_time(t_end) / args.steps
+    enc_ms = statistics.mean(a.elapsed_time(b) for a, b, _ in ev)
+    dec_ms = statistics.mean(b.elapsed_time(c) for _, b, c in ev)
+    assert eh.get_status(wsd) == eh.EH_OK
+    assert all(torch.equal(x, y) for x, y in zip(xs, ys)), "round trip mismatch after timing"
+    if world > 1:
+        t = torch.tensor([ms, enc_ms, dec_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms, enc_ms, dec_ms = t.tolist()
+
+    # end to end through the public API: pinned host -> device copy of the
+    # block, compress (host wait for the bit counts), decompress, status read
+    e2e_steps = max(1, args.e2e_steps)
+    for _ in range(2):
+        for h, x in zip(xs_host, xs):
+            x.copy_(h, non_blocking=True)
+        eh.compress_batch(p, xs, outs, wsc)
+        eh.decompress_batch(p, outs, ys, wsd)
+        eh.get_status(wsd)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        for h, x in zip(xs_host, xs):
+            x.copy_(h, non_blocking=True)
+        eh.compress_batch(p, xs, outs, wsc)
+        eh.decompress_batch(p, outs, ys, wsd)
+        st = eh.get_status(wsd)
+        assert st == eh.EH_OK
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = t.item()
+        dist.barrier()
+
+    if rank == 0:
+        peak, peak_kind = hbm_peak()
+        value = world * 2 * in_bytes / (ms * 1e-3) / 1e9
+        enc_gbs = in_bytes / (enc_ms * 1e-3) / 1e9
+        dec_gbs = in_bytes / (dec_ms * 1e-3) / 1e9
+        # algorithmic bytes, each byte counted once
+        dec_alg = stream_bytes + sm_bytes + off_bytes + in_bytes
+        enc_alg = in_bytes + sm_bytes + stream_bytes + off_bytes
+        dec_achieved = dec_alg / (dec_ms * 1e-3) / 1e9
+        enc_achieved = enc_alg / (enc_ms * 1e-3) / 1e9
+        traffic = None
+        if DECODE_TRAFFIC["bytes"] and DECODE_TRAFFIC["source_sha"] == decoder_source_sha():
+            traffic = DECODE_TRAFFIC["bytes"]
+        line = {
+            "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "u16",
+            "data": "synthetic",
+            "config": {"workload": "llama8b_block: q,k,v,o 4096/1024x4096, gate/up 14336x4096, "
+                                   "down 4096x14336 BF16, Student-t(5) std 0.02, seed 2",
+                       "elements": sum(ns), "chunk_elems": p.chunk_elems, "max_code_len": p.max_code_len,
+                       "parallelism": f"replicas x{world}",
+                       "l2": "no flush: inputs (436 MB) larger than L2 (126 MB)"},
+            "decode_gbs": dec_gbs, "encode_gbs": enc_gbs,
+            "pct_hbm": {"decode": dec_achieved / peak, "encode": enc_achieved / peak,
+                        "peak_gbs": peak, "peak_kind": peak_kind},
+            "size_ratio": comp_bytes / in_bytes,
+            "bits_per_exponent": 8 * stream_bytes / sum(ns),
+            "roofline": {"bound": "hbm", "kernel": "decode (tables + decode launch)",
+                         "achieved": dec_achieved, "peak": peak, "unit": "GB/s",
+                         "frac": dec_achieved / peak, "traffic": traffic,
+                         "algorithmic_bytes": dec_alg, "peak_kind": peak_kind},
+            "e2e": {"value": world * 2 * in_bytes / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
+                    "h2d_bytes_per_step": in_bytes, "d2h_bytes_per_step": 8 + 8 * len(ns) + 4,
+                    "ms_per_step": e2e_ms},
+            "gpu_launches": 6 * args.steps,
+            "clocks": clk.summary(),
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline_oracle(items)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

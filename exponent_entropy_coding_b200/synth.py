@@ -75,12 +75,12 @@ def student_t_bf16(shape, rng: np.random.Generator, df: float = 5.0,
     return to_bf16_bits(w)
 
 
-def llama8b_block(seed: int = 2, scale: int = 1):
-    """[(name, bits)] for the seven matrices; ``scale`` divides the row count
-    (scale=1 is the full block)."""
+def llama8b_block(seed: int = 2, scale: int = 1, count: int = 7):
+    """[(name, bits)] for the first ``count`` of the seven matrices; ``scale``
+    divides the row count (scale=1 is the full block)."""
     rng = np.random.default_rng(seed)
     out = []
-    for name, (r, c) in LLAMA8B_BLOCK_SHAPES:
+    for name, (r, c) in LLAMA8B_BLOCK_SHAPES[:count]:
         out.append((name, student_t_bf16((max(1, r // scale), c), rng).reshape(-1)))
     return out
 

@@ -230,3 +230,17 @@ def test_corruption_is_reported(eh, oracle):
     c.chunk_bit_off.copy_(good)
     y = eh.decompress(c, p, workspace=ws)
     assert np.array_equal(host_bits(y, 0), x)
+
+
+def test_side_stream(eh, oracle):
+    # calls take the caller's stream (a torch stream handle, not the default)
+    x = synth.normal_bf16(3 * 65536 + 9, seed=12)
+    p = eh.plan(0)
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        t = dev(x)
+        c = eh.compress(t, p, stream=s)
+        y = eh.decompress(c, p, stream=s)
+    s.synchronize()
+    assert_same(c, oracle.compress(0, x))
+    assert torch.equal(y, t)
