@@ -29,10 +29,11 @@
 namespace eh {
 namespace {
 
-constexpr uint32_t kMaskBits = 32;            // boundaries recorded per thread
+constexpr uint32_t kMaskBits = 64;            // code starts recorded per thread
 constexpr uint32_t kSpinLimit = 1u << 26;     // bounded mbarrier wait
 
 // ---------------------------------------------------------------- tables
+// One CTA of 256 threads per codebook.
 __global__ void __launch_bounds__(256) tables_kernel(const __grid_constant__ Batch b) {
   const Item &I = b.item[blockIdx.x];
   DecodeTables *T = (DecodeTables *)I.lut;
@@ -41,15 +42,16 @@ __global__ void __launch_bounds__(256) tables_kernel(const __grid_constant__ Bat
   __shared__ uint32_t cntL[33], firstL[33], baseL[33];
   __shared__ uint64_t limL[33];
   __shared__ uint8_t lens[256];
-  __shared__ unsigned long long kraft;
-  __shared__ uint32_t err, nsub;
-  __shared__ uint32_t subpre[kNumSub];
-  __shared__ uint32_t wcount[8];
   __shared__ uint8_t srt[256];
+  __shared__ unsigned long long kraft;
+  __shared__ uint32_t err;
 
-  if (blockIdx.x == 0 && tid == 0) *b.status = 0u;  // this call's status starts clean
+  if (blockIdx.x == 0 && tid == 0) {
+    *b.status = 0u;  // this call's status starts clean
+    *b.ticket = 0u;
+  }
   if (tid <= 32) cntL[tid] = 0;
-  if (tid == 0) { kraft = 0; err = 0; nsub = 0; }
+  if (tid == 0) { kraft = 0; err = 0; }
   const uint32_t l = tid < A ? I.code_len[tid] : 0u;
   lens[tid] = (uint8_t)l;
   __syncthreads();
@@ -84,7 +86,7 @@ __global__ void __launch_bounds__(256) tables_kernel(const __grid_constant__ Bat
     T->nsym = nsym;
   }
   __syncthreads();
-  // symbol order (length, symbol); stored codes must be the canonical ones
+  // symbol order (length, symbol); the stored codes must be the canonical ones
   if (tid < A && l && l <= 32) {
     uint32_t k = 0;
     for (int s2 = 0; s2 < tid; s2++) k += lens[s2] == l;
@@ -97,50 +99,47 @@ __global__ void __launch_bounds__(256) tables_kernel(const __grid_constant__ Bat
     T->lim[tid] = limL[tid];
   }
   __syncthreads();
+  if (err) {  // invalid codebook: nothing below may index with its values
+    if (tid == 0) T->err = err;
+    return;
+  }
   T->sorted[tid] = tid < (int)nsym ? srt[tid] : (uint8_t)0;
-  const uint8_t *sorted_g = srt;
-  // first level: pattern tid = next 8 bits
-  uint32_t syms = 0, pos = 0, nc = 0, len0 = 0;
-  while (nc < 4) {
-    int found = 0;
-    for (uint32_t L = 1; L + pos <= 8; L++) {
-      uint32_t v = (tid >> (8 - pos - L)) & ((1u << L) - 1u);
-      if (cntL[L] && v >= firstL[L] && v - firstL[L] < cntL[L]) {
-        syms |= (uint32_t)sorted_g[baseL[L] + v - firstL[L]] << (8 * nc);
-        if (nc == 0) len0 = L;
-        pos += L;
-        nc++;
-        found = 1;
-        break;
-      }
+
+  // first level.  Codes longer than kLutBits fill the left-justified range
+  // [lim[kLutBits], lim[32]), so their prefixes are consecutive: the first
+  // kNumSub of them get a second-level table.
+  constexpr uint32_t kShift = 32 - kLutBits;
+  const uint32_t sub0 = (uint32_t)(limL[kLutBits] >> kShift);
+  for (uint32_t p = tid; p < (1u << kLutBits); p += 256) {
+    uint32_t syms = 0, pos = 0, nc = 0, bnd = 0;
+    while (nc < 4 && pos < (uint32_t)kLutBits) {
+      const uint32_t x = (p << kShift) << pos;  // next bits, left-justified, zero-filled
+      uint32_t L = 1;
+      while (L <= 32 && (uint64_t)x >= limL[L]) L++;
+      if (L > (uint32_t)kLutBits - pos) break;  // not complete inside the index bits
+      const uint32_t v = x >> (32 - L);
+      syms |= (uint32_t)srt[baseL[L] + v - firstL[L]] << (8 * nc);
+      bnd |= 1u << pos;
+      pos += L;
+      nc++;
     }
-    if (!found) break;
+    uint32_t sub = kNoSub;
+    if (nc == 0 && ((uint64_t)p << kShift) < limL[32] && p - sub0 < (uint32_t)kNumSub) sub = p - sub0;
+    T->l1sym[p] = syms;
+    T->l1meta[p] = pos | (nc << 4) | (bnd << 7) | (sub << 19);
   }
-  // prefixes of codes longer than 8 bits get a second-level table (in prefix
-  // order, at most kNumSub of them)
-  const bool need_sub = nc == 0 && ((uint64_t)tid << 24) < limL[32];
-  const uint32_t ballot = __ballot_sync(0xffffffffu, need_sub);
-  if ((tid & 31) == 0) wcount[tid >> 5] = __popc(ballot);
-  __syncthreads();
-  uint32_t sidx = __popc(ballot & ((1u << (tid & 31)) - 1u));
-  for (int w = 0; w < (tid >> 5); w++) sidx += wcount[w];
-  uint32_t sub_field = 0xFFu;
-  if (need_sub && sidx < (uint32_t)kNumSub) {
-    sub_field = sidx;
-    subpre[sidx] = tid;
-    atomicMax(&nsub, sidx + 1);
-  }
-  T->l1[tid] = (uint64_t)syms | ((uint64_t)len0 << 32) | ((uint64_t)pos << 36) |
-               ((uint64_t)nc << 40) | ((uint64_t)sub_field << 48);
-  __syncthreads();
+  // second level: codes of kLutBits+1 .. kLutBits+8 bits
   for (uint32_t j = 0; j < (uint32_t)kNumSub; j++) {
     uint32_t e = 0;
-    if (j < nsub) {
-      const uint32_t v16 = (subpre[j] << 8) | (uint32_t)tid;
-      for (uint32_t L = 9; L <= 16; L++) {
-        uint32_t v = v16 >> (16 - L);
-        if (cntL[L] && v >= firstL[L] && v - firstL[L] < cntL[L]) {
-          e = (uint32_t)sorted_g[baseL[L] + v - firstL[L]] | (L << 8);
+    const uint32_t p = sub0 + j;
+    if (((uint64_t)p << kShift) < limL[32]) {
+      const uint32_t x = (p << kShift) | ((uint32_t)tid << (kShift - 8));
+      for (uint32_t L = kLutBits + 1; L <= (uint32_t)kLutBits + 8; L++) {
+        if ((uint64_t)x < limL[L]) {
+          if (x >= (uint32_t)(limL[L - 1])) {
+            const uint32_t v = x >> (32 - L);
+            e = (uint32_t)srt[baseL[L] + v - firstL[L]] | (L << 8);
+          }
           break;
         }
       }
@@ -151,67 +150,118 @@ __global__ void __launch_bounds__(256) tables_kernel(const __grid_constant__ Bat
 }
 
 // ---------------------------------------------------------------- decode
+// Exponent j of a chunk is kept at byte j + 4*(j/128) of the exponent buffer:
+// every 128-byte row is followed by 4 pad bytes, so threads whose outputs
+// start about 128 values apart write to different shared-memory banks.
+constexpr uint32_t kExpBytes = kMaxChunk + 4 * (kMaxChunk / 128);
+__device__ __forceinline__ uint32_t exp_slot(uint32_t j) { return j + ((j >> 7) << 2); }
+
+// Bit reader over the chunk's stream words (stored big-endian): a 64-bit
+// buffer holding the next bits MSB-first, refilled 32 bits at a time.
 template <bool kSmem>
-struct BitSrc {
-  const uint32_t *w;  // shared memory: words already in MSB-first order
-  __device__ __forceinline__ uint32_t word(uint32_t i) const {
-    if (kSmem) return w[i];
-    return bswap32(__ldg(w + i));
+struct Reader {
+  const uint32_t *w;
+  uint64_t buf;    // next bits, MSB first; bits below the valid ones are zero
+  uint32_t avail;  // valid bits in buf, >= 32 between steps
+  uint32_t widx;   // next word to load
+  __device__ __forceinline__ uint32_t word(uint32_t i) const { return bswap32(kSmem ? w[i] : __ldg(w + i)); }
+  __device__ __forceinline__ void seek(uint32_t p) {
+    const uint32_t i = p >> 5, s = p & 31;
+    buf = (((uint64_t)word(i) << 32) | word(i + 1)) << s;
+    avail = 64 - s;
+    widx = i + 2;
   }
-  // 32 bits starting at bit p
-  __device__ __forceinline__ uint32_t peek(uint32_t p) const {
-    const uint32_t i = p >> 5;
-    return __funnelshift_l(word(i + 1), word(i), p & 31);
+  __device__ __forceinline__ void skip(uint32_t nb) {
+    buf <<= nb;
+    avail -= nb;
+    if (avail < 32) {
+      buf |= (uint64_t)word(widx++) << (32 - avail);
+      avail += 32;
+    }
   }
 };
 
-// One decode step at the bit window `peek`.  multi: consume every complete
-// code inside the 8-bit first-level index (up to 4); else only the first.
-// Returns the number of codes (0: invalid code), their symbols in *syms (8
-// bits each) and the bits consumed in *nbits.
-__device__ __forceinline__ uint32_t decode_step(const DecodeTables &T, uint32_t peek, bool multi,
-                                                uint32_t *syms, uint32_t *nbits) {
-  const uint64_t e = T.l1[peek >> 24];
-  const uint32_t hi = (uint32_t)(e >> 32);
-  const uint32_t nc = (hi >> 8) & 7u;
-  if (nc) {
-    if (multi) {
-      *nbits = (hi >> 4) & 15u;
-      *syms = (uint32_t)e;
-      return nc;
-    }
-    *nbits = hi & 15u;
-    *syms = (uint32_t)e & 0xFFu;
-    return 1;
-  }
-  const uint32_t si = (hi >> 16) & 0xFFu;
-  if (si != 0xFFu) {
-    const uint32_t e2 = T.sub[si][(peek >> 16) & 0xFFu];
+__device__ __forceinline__ uint32_t lut_index(uint64_t buf) { return (uint32_t)(buf >> (64 - kLutBits)); }
+
+// Code longer than the first-level index: second-level table, else search of
+// the canonical limits.  Returns 1 and the symbol and length, or 0 for an
+// invalid code.
+__device__ __forceinline__ uint32_t decode_long(const DecodeTables &T, uint64_t buf, uint32_t meta,
+                                                uint32_t &syms, uint32_t &nbits) {
+  const uint32_t peek = (uint32_t)(buf >> 32);
+  const uint32_t si = (meta >> 19) & 63u;
+  if (si != kNoSub) {
+    const uint32_t e2 = T.sub[si][(peek >> (24 - kLutBits)) & 0xFFu];
     const uint32_t l = (e2 >> 8) & 63u;
     if (l) {
-      *nbits = l;
-      *syms = e2 & 0xFFu;
+      nbits = l;
+      syms = e2 & 0xFFu;
       return 1;
     }
   }
-  uint32_t L = 9;
+  uint32_t L = kLutBits + 1;
   #pragma unroll 1
   while (L <= 32 && (uint64_t)peek >= T.lim[L]) L++;
   if (L > 32) return 0;
   const uint32_t v = L == 32 ? peek : peek >> (32 - L);
-  *syms = T.sorted[T.base[L] + (v - T.first[L])];
-  *nbits = L;
+  syms = T.sorted[T.base[L] + (v - T.first[L])];
+  nbits = L;
   return 1;
 }
 
-struct DecodeSmem {
-  alignas(128) uint32_t stage[kStageBytes / 4 + 16];  // bulk-copy target
-  alignas(16) uint8_t exps[kMaxChunk];                // decoded exponents of one chunk
-  alignas(16) DecodeTables tabs;
-  uint32_t ends[kThreads];
-  uint32_t wsum[kThreads / 32];
+// One decode step on the next bits `buf`, taking only codes that start in
+// the next `lim` (>= 1) bits.  Returns the number of codes taken (0: invalid
+// code); their symbols (8 bits each, first in the low byte) when kSyms, the
+// bits up to the end of the last code taken, and the code starts as a bitmap.
+template <bool kSyms>
+__device__ __forceinline__ uint32_t decode_step(const DecodeTables &T, uint64_t buf, uint32_t lim,
+                                                uint32_t &syms, uint32_t &nbits, uint32_t &bnd) {
+  const uint32_t idx = lut_index(buf);
+  const uint32_t meta = T.l1meta[idx];
+  uint32_t k = (meta >> 4) & 7u;
+  if (k) {
+    uint32_t nb = meta & 15u, bm = (meta >> 7) & 0xFFFu;
+    uint32_t sy = kSyms ? T.l1sym[idx] : 0u;
+    if (nb > lim) {
+      // codes starting at or after the limit belong to the next window
+      const uint32_t keep = bm & ((1u << lim) - 1u);
+      const uint32_t rest = bm >> lim;
+      k = __popc(keep);
+      nb = rest ? lim + __ffs(rest) - 1 : nb;
+      bm = keep;
+      if (kSyms && k < 4) sy &= (1u << (8 * k)) - 1u;
+    }
+    nbits = nb;
+    bnd = bm;
+    syms = sy;
+    return k;
+  }
+  bnd = 1u;
+  return decode_long(T, buf, meta, syms, nbits);
+}
+
+// The decoding CTA holds two independent groups of kGroupThreads threads.
+// Each group decodes its own chunk into its own exponent buffer, so one
+// group's memory-bound output pass overlaps the other's decode; the decode
+// tables are shared.
+constexpr uint32_t kGroupThreads = 512;
+constexpr uint32_t kNumGroups = kDecThreads / kGroupThreads;
+constexpr uint32_t kGroupStage = 27136;  // bytes of stream staged per group
+
+struct GroupSmem {
+  alignas(128) uint32_t stage[kGroupStage / 4 + 16];  // bulk-copy target (stream bytes as stored)
+  alignas(16) uint8_t exps[kExpBytes];                // decoded exponents of one chunk (padded rows)
+  uint32_t ends[kGroupThreads];
+  uint32_t wsum[kGroupThreads / 32];
   alignas(8) unsigned long long mbar;
 };
+
+struct DecodeSmem {
+  alignas(16) DecodeTables tabs;
+  GroupSmem grp[kNumGroups];
+  uint32_t abort_flag;
+};
+static_assert(sizeof(DecodeSmem) + 128 <= 232448, "decoder shared memory exceeds the per-CTA limit");
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
   return (uint32_t)__cvta_generic_to_shared(p);
@@ -244,8 +294,39 @@ __device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t by
       : "memory");
 }
 
-__device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t *wsum, uint32_t *total) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+__device__ __forceinline__ uint4 ld_nc16(const void *p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+
+__device__ __forceinline__ uint2 ld_nc8(const void *p) {
+  uint2 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "l"(p));
+  return v;
+}
+
+// Barriers of one group: named barrier `id` over kGroupThreads threads.
+__device__ __forceinline__ void gsync(uint32_t id) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "n"(kGroupThreads) : "memory");
+}
+__device__ __forceinline__ bool gsync_or(uint32_t id, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n .reg .pred pi, po;\n setp.ne.u32 pi, %1, 0;\n bar.red.or.pred po, %2, %3, pi;\n"
+      " selp.u32 %0, 1, 0, po;\n}"
+      : "=r"(r)
+      : "r"((uint32_t)pred), "r"(id), "n"(kGroupThreads)
+      : "memory");
+  return r != 0;
+}
+
+__device__ __forceinline__ uint32_t group_excl_scan(uint32_t v, uint32_t *wsum, uint32_t *total, uint32_t id,
+                                                    uint32_t gtid) {
+  constexpr int kWarps = kGroupThreads / 32;
+  const int lane = gtid & 31, warp = gtid >> 5;
   uint32_t x = v;
   #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
@@ -253,75 +334,175 @@ __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t *wsum, 
     if (lane >= o) x += y;
   }
   if (lane == 31) wsum[warp] = x;
-  __syncthreads();
+  gsync(id);
   if (warp == 0) {
-    uint32_t t = lane < kThreads / 32 ? wsum[lane] : 0u;
+    uint32_t t = lane < kWarps ? wsum[lane] : 0u;
     #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       uint32_t y = __shfl_up_sync(0xffffffffu, t, o);
       if (lane >= o) t += y;
     }
-    if (lane < kThreads / 32) wsum[lane] = t;
+    if (lane < kWarps) wsum[lane] = t;
   }
-  __syncthreads();
-  *total = wsum[kThreads / 32 - 1];
+  gsync(id);
+  *total = wsum[kWarps - 1];
   return (warp ? wsum[warp - 1] : 0u) + x - v;
 }
 
-// Steps 2-5 for one chunk whose bits are [rel0, rel0 + nbits) of `src`.
-// Returns false (CTA-uniform) if the chunk is corrupt.
+// Packs decoded exponents four to a word into the exponent buffer, which
+// is zeroed before each chunk.  Words are combined with OR, so the words a run
+// shares with its neighbours need no special case.
+struct ExpWriter {
+  uint32_t *words;  // exponent buffer as words
+  uint32_t wj;      // output index of the word being filled (multiple of 4)
+  uint32_t na;      // bytes of that word filled so far (those below the run are zero)
+  uint64_t acc;
+  __device__ __forceinline__ void init(uint8_t *e, uint32_t j) {
+    words = (uint32_t *)e;
+    wj = j & ~3u;
+    na = j & 3u;
+    acc = 0;
+  }
+  __device__ __forceinline__ void put(uint32_t syms, uint32_t k) {
+    acc |= (uint64_t)syms << (8 * na);
+    na += k;
+    if (na >= 4) {
+      atomicOr(words + (exp_slot(wj) >> 2), (uint32_t)acc);
+      acc >>= 32;
+      na -= 4;
+      wj += 4;
+    }
+  }
+  __device__ __forceinline__ void finish() {
+    if (na) atomicOr(words + (exp_slot(wj) >> 2), (uint32_t)acc);
+  }
+};
+
+// Steps 2-5 for one chunk whose bits are [rel0, rel0 + nbits) of `words`,
+// decoded by one group.  Returns false (group-uniform) if the chunk is
+// corrupt.
 template <bool kSmem>
-__device__ bool decode_chunk(DecodeSmem &S, const BitSrc<kSmem> src, uint32_t rel0, uint32_t nbits,
-                             uint32_t cnt, uint32_t *timeout) {
-  const DecodeTables &T = S.tabs;
-  const uint32_t tid = threadIdx.x;
+__device__ bool decode_chunk(GroupSmem &G, const DecodeTables &T, const uint32_t *words, uint32_t rel0,
+                             uint32_t nbits, uint32_t cnt, uint32_t id, uint32_t gtid, uint32_t *timeout) {
   // window width: a multiple of the gcd of the code lengths, so that a
   // fixed-length code starts every window on a code boundary
   const uint32_t gq = T.gcd;
-  uint32_t W = (nbits + kThreads - 1) / kThreads;
+  uint32_t W = (nbits + kGroupThreads - 1) / kGroupThreads;
   W = (W + gq - 1) / gq * gq;
-  const uint32_t ws = min(tid * W, nbits), we = min(ws + W, nbits);
+  const uint32_t ws = min(gtid * W, nbits), we = min(ws + W, nbits);
+  Reader<kSmem> r;
+  r.w = words;
+  // Bulk decoding runs while 2 * kLutBits bits of the window remain: two
+  // first-level lookups per refill, no window-end handling.
+  constexpr uint32_t kBulk = 2 * kLutBits;
 
-  // 2. speculative decode of the own window
-  uint32_t pos = ws, n = 0, mask = 0;
+  // 2. speculative decode of the own window; record where codes start in
+  //    its first kMaskBits bits
+  uint32_t pos = ws, n = 0;
+  uint64_t mask = 0;
   bool bad = false;
-  while (pos < we) {
-    const uint32_t off = pos - ws;
-    const bool single = off < kMaskBits || pos + 8 > we;
-    uint32_t syms, nb;
-    const uint32_t k = decode_step(T, src.peek(rel0 + pos), !single, &syms, &nb);
-    if (!k) { bad = true; break; }
-    if (off < kMaskBits) mask |= 1u << off;
-    pos += nb;
-    n += k;
+  if (pos < we) {
+    r.seek(rel0 + pos);
+    while (pos + kBulk <= we && pos - ws < kMaskBits) {
+      const uint32_t off = pos - ws;
+      const uint32_t m1 = T.l1meta[lut_index(r.buf)];
+      const uint32_t k1 = (m1 >> 4) & 7u, nb1 = m1 & 15u;
+      if (!k1) {
+        uint32_t syms, nb;
+        if (!decode_long(T, r.buf, m1, syms, nb)) { bad = true; break; }
+        mask |= 1ull << off;
+        r.skip(nb);
+        pos += nb;
+        n += 1;
+        continue;
+      }
+      mask |= (uint64_t)((m1 >> 7) & 0xFFFu) << off;
+      const uint32_t m2 = T.l1meta[lut_index(r.buf << nb1)];
+      const uint32_t k2 = (m2 >> 4) & 7u, nb2 = m2 & 15u;
+      if (!k2) {
+        r.skip(nb1);
+        pos += nb1;
+        n += k1;
+        continue;
+      }
+      if (off + nb1 < kMaskBits) mask |= (uint64_t)((m2 >> 7) & 0xFFFu) << (off + nb1);
+      r.skip(nb1 + nb2);
+      pos += nb1 + nb2;
+      n += k1 + k2;
+    }
+    while (!bad && pos + kBulk <= we) {
+      const uint32_t m1 = T.l1meta[lut_index(r.buf)];
+      const uint32_t k1 = (m1 >> 4) & 7u, nb1 = m1 & 15u;
+      if (!k1) {
+        uint32_t syms, nb;
+        if (!decode_long(T, r.buf, m1, syms, nb)) { bad = true; break; }
+        r.skip(nb);
+        pos += nb;
+        n += 1;
+        continue;
+      }
+      const uint32_t m2 = T.l1meta[lut_index(r.buf << nb1)];
+      const uint32_t k2 = (m2 >> 4) & 7u, nb2 = m2 & 15u;
+      if (!k2) {
+        r.skip(nb1);
+        pos += nb1;
+        n += k1;
+        continue;
+      }
+      r.skip(nb1 + nb2);
+      pos += nb1 + nb2;
+      n += k1 + k2;
+    }
+    while (!bad && pos < we) {
+      uint32_t syms, nb, bnd;
+      const uint32_t k = decode_step<false>(T, r.buf, we - pos, syms, nb, bnd);
+      if (!k) { bad = true; break; }
+      const uint32_t off = pos - ws;
+      if (off < kMaskBits) mask |= (uint64_t)bnd << off;
+      r.skip(nb);
+      pos += nb;
+      n += k;
+    }
   }
   const uint32_t spec_end = bad ? we : pos, spec_n = n;
-  const uint32_t spec_mask = bad ? 0u : mask;
+  const uint64_t spec_mask = bad ? 0ull : mask;
   uint32_t my_start = ws, my_end = spec_end, my_n = spec_n;
-  S.ends[tid] = my_end;
-  __syncthreads();
+  G.ends[gtid] = my_end;
+  gsync(id);
 
-  // 3. fix-up rounds
+  // 3. fix-up rounds: restart from the predecessor's end until a code starts
+  //    where a speculative one did (from there on the speculative decode is
+  //    right)
   for (uint32_t round = 0;; round++) {
-    const uint32_t pred = tid == 0 ? 0u : S.ends[tid - 1];
+    const uint32_t pred = gtid == 0 ? 0u : G.ends[gtid - 1];
     bool changed = false;
-    if (tid > 0 && pred != my_start) {
+    if (gtid > 0 && pred != my_start) {
       my_start = pred;
       uint32_t p = pred, k = 0;
       bool synced = false, bad2 = false;
+      if (p < we) r.seek(rel0 + p);
       while (p < we) {
-        const uint32_t off = p - ws;
-        if (off < kMaskBits && ((spec_mask >> off) & 1u)) { synced = true; break; }
-        const bool single = off < kMaskBits || p + 8 > we;
-        uint32_t syms, nb;
-        const uint32_t kk = decode_step(T, src.peek(rel0 + p), !single, &syms, &nb);
+        uint32_t syms, nb, bnd;
+        const uint32_t kk = decode_step<false>(T, r.buf, we - p, syms, nb, bnd);
         if (!kk) { bad2 = true; break; }
+        const uint32_t off = p - ws;
+        if (off < kMaskBits) {
+          const uint64_t common = ((uint64_t)bnd << off) & spec_mask;
+          if (common) {
+            const uint32_t q = __ffsll(common) - 1;  // offset from ws, >= off
+            k += __popc(bnd & ((1u << (q - off)) - 1u));
+            p = ws + q;
+            synced = true;
+            break;
+          }
+        }
+        r.skip(nb);
         p += nb;
         k += kk;
       }
       uint32_t new_end;
       if (synced) {
-        my_n = k + spec_n - __popc(spec_mask & ((1u << (p - ws)) - 1u));
+        my_n = k + spec_n - __popcll(spec_mask & ((1ull << (p - ws)) - 1ull));
         new_end = spec_end;
         bad = false;
       } else {
@@ -332,11 +513,11 @@ __device__ bool decode_chunk(DecodeSmem &S, const BitSrc<kSmem> src, uint32_t re
       changed = new_end != my_end;
       my_end = new_end;
     }
-    __syncthreads();
-    if (changed) S.ends[tid] = my_end;
-    if (!__syncthreads_or(changed)) break;
-    if (round > kThreads + 1) {  // cannot happen for consistent data
-      if (tid == 0) *timeout = 1;
+    gsync(id);
+    if (changed) G.ends[gtid] = my_end;
+    if (!gsync_or(id, changed)) break;
+    if (round > kGroupThreads + 1) {  // cannot happen for consistent data
+      if (gtid == 0) *timeout = 1;
       bad = true;
       break;
     }
@@ -344,166 +525,274 @@ __device__ bool decode_chunk(DecodeSmem &S, const BitSrc<kSmem> src, uint32_t re
 
   // 4. output index of every thread's first code
   uint32_t total;
-  const uint32_t o = block_excl_scan(my_n, S.wsum, &total);
-  const bool ok = !__syncthreads_or(bad) && total == cnt && S.ends[kThreads - 1] == nbits;
+  const uint32_t o = group_excl_scan(my_n, G.wsum, &total, id, gtid);
+  const bool ok = !gsync_or(id, bad) && total == cnt && G.ends[kGroupThreads - 1] == nbits;
   if (!ok) return false;
 
   // 5. decode again from the true start, writing exponents
-  uint32_t j = o;
-  pos = tid == 0 ? 0u : S.ends[tid - 1];
-  while (pos < we) {
-    uint32_t syms, nb;
-    const uint32_t k = decode_step(T, src.peek(rel0 + pos), pos + 8 <= we, &syms, &nb);
-    if (!k) break;
-    for (uint32_t q = 0; q < k; q++) {
-      if (j + q < cnt) S.exps[j + q] = (uint8_t)(syms >> (8 * q));
+  ExpWriter out;
+  out.init(G.exps, o);
+  pos = gtid == 0 ? 0u : G.ends[gtid - 1];
+  if (pos < we) {
+    r.seek(rel0 + pos);
+    while (pos + kBulk <= we) {
+      const uint32_t i1 = lut_index(r.buf);
+      const uint32_t m1 = T.l1meta[i1];
+      const uint32_t k1 = (m1 >> 4) & 7u, nb1 = m1 & 15u;
+      if (!k1) {
+        uint32_t syms, nb;
+        if (!decode_long(T, r.buf, m1, syms, nb)) break;
+        r.skip(nb);
+        pos += nb;
+        out.put(syms, 1);
+        continue;
+      }
+      const uint32_t s1 = T.l1sym[i1];
+      const uint32_t i2 = lut_index(r.buf << nb1);
+      const uint32_t m2 = T.l1meta[i2];
+      const uint32_t k2 = (m2 >> 4) & 7u, nb2 = m2 & 15u;
+      out.put(s1, k1);
+      if (!k2) {
+        r.skip(nb1);
+        pos += nb1;
+        continue;
+      }
+      const uint32_t s2 = T.l1sym[i2];
+      r.skip(nb1 + nb2);
+      pos += nb1 + nb2;
+      out.put(s2, k2);
     }
-    j += k;
-    pos += nb;
+    while (pos < we) {
+      uint32_t syms, nb, bnd;
+      const uint32_t k = decode_step<true>(T, r.buf, we - pos, syms, nb, bnd);
+      if (!k) break;
+      r.skip(nb);
+      pos += nb;
+      out.put(syms, k);
+    }
   }
-  __syncthreads();
+  out.finish();
+  gsync(id);
   return true;
 }
 
-// exponent bytes E and sign/mantissa bytes M (4 values) -> 4 BF16 values
+// (sign+mantissa, exponent) byte pairs [s0, e0, s1, e1] -> two BF16 values
 __device__ __forceinline__ uint32_t bf16_merge2(uint32_t p) {
-  // p = [s0, e0, s1, e1] as bytes; value = (s&0x80)<<8 | e<<7 | (s&0x7F)
   return (p & 0x007F007Fu) | ((p >> 1) & 0x7F807F80u) | ((p & 0x00800080u) << 8);
 }
 
+// four sign+mantissa nibbles (16 bits) and four exponent bytes -> 4 FP8 values
+__device__ __forceinline__ uint32_t fp8_merge4(uint32_t nib16, uint32_t e4) {
+  const uint32_t t = (nib16 & 0xFu) | ((nib16 & 0xF0u) << 4) | ((nib16 & 0xF00u) << 8) | ((nib16 & 0xF000u) << 12);
+  return ((t & 0x08080808u) << 4) | ((e4 << 3) & 0x78787878u) | (t & 0x07070707u);
+}
+
+// Where one chunk's bits are and whether they fit a shared-memory stage.
+struct ChunkInfo {
+  int item;
+  uint32_t c;       // tensor-local chunk index
+  uint32_t cnt;     // values in the chunk
+  uint32_t nbits;   // code bits of the chunk
+  uint32_t rel0;    // first bit of the chunk relative to byte `lo`
+  uint32_t bytes;   // stream bytes staged (multiple of 16)
+  uint64_t lo;      // first staged stream byte (multiple of 16)
+  bool ok;          // offsets consistent with the buffer
+  bool fits;        // bits staged in shared memory
+};
+
+__device__ __forceinline__ ChunkInfo chunk_info(const Batch &b, uint32_t g) {
+  ChunkInfo ci;
+  ci.item = find_item(b, g);
+  const Item &I = b.item[ci.item];
+  ci.c = I.first_chunk + (g - I.chunk0);
+  const uint64_t i0 = (uint64_t)ci.c * b.chunk_elems;
+  ci.cnt = (uint32_t)min((uint64_t)b.chunk_elems, I.n - i0);
+  const uint64_t B0 = I.off[ci.c], B1 = I.off[ci.c + 1], Bt = I.off[I.total_chunks];
+  // the stream must hold every chunk's bits plus 16 readable bytes
+  ci.ok = I.off[0] == 0 && B0 <= B1 && B1 <= Bt && (Bt + 7) / 8 + 16 <= I.stream_cap && B1 - B0 >= ci.cnt &&
+          B1 - B0 <= (uint64_t)ci.cnt * 32u;
+  ci.nbits = (uint32_t)(B1 - B0);
+  ci.lo = (B0 >> 3) & ~uint64_t(15);
+  const uint64_t hi = (((B1 + 7) >> 3) + 16 + 15) & ~uint64_t(15);
+  ci.rel0 = (uint32_t)(B0 - ci.lo * 8);
+  ci.fits = ci.ok && hi - ci.lo <= (uint64_t)kGroupStage && hi <= I.stream_cap;
+  ci.bytes = ci.fits ? (uint32_t)(hi - ci.lo) : 0u;
+  return ci;
+}
+
+__device__ __forceinline__ void issue_stage(GroupSmem &G, const Batch &b, const ChunkInfo &ci) {
+  mbar_expect_tx(&G.mbar, ci.bytes);
+  bulk_g2s(G.stage, b.item[ci.item].stream + ci.lo, ci.bytes, &G.mbar);
+}
+
+// Persistent: CTA i of G decodes the contiguous chunk range
+// [i*C/G, (i+1)*C/G), split into runs of one tensor (one codebook); inside a
+// run the two groups take alternate chunks.  Each group copies its next
+// chunk's stream bits while it merges and stores the current one.
 template <int DT>
-__global__ void __launch_bounds__(kThreads, 2) decode_kernel(const __grid_constant__ Batch b) {
+__global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_constant__ Batch b) {
   extern __shared__ __align__(128) uint8_t smem_raw[];
   DecodeSmem &S = *reinterpret_cast<DecodeSmem *>(smem_raw);
   const uint32_t tid = threadIdx.x;
-  if (tid == 0) {
-    mbar_init(&S.mbar, 1);
+  const uint32_t grp = tid / kGroupThreads, gtid = tid % kGroupThreads, id = 1 + grp;
+  GroupSmem &G = S.grp[grp];
+  const uint32_t g0 = (uint32_t)(((uint64_t)b.total_chunks * blockIdx.x) / gridDim.x);
+  const uint32_t g1 = (uint32_t)(((uint64_t)b.total_chunks * (blockIdx.x + 1)) / gridDim.x);
+  if (g0 >= g1) return;
+  if (gtid == 0) {
+    mbar_init(&G.mbar, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
+  if (tid == 0) S.abort_flag = 0;
   __syncthreads();
-  uint32_t parity = 0;
-  int cur = -1;
-  uint32_t timeout = 0;
+  uint32_t parity = 0, timeout = 0;
+  bool pending = false;  // a stage copy of this group is in flight
 
-  for (uint32_t g = blockIdx.x; g < b.total_chunks; g += gridDim.x) {
-    const int it = find_item(b, g);
-    const Item &I = b.item[it];
-    if (it != cur) {
-      __syncthreads();
+  for (uint32_t seg = g0; seg < g1;) {
+    const Item &I = b.item[find_item(b, seg)];
+    const uint32_t seg_end = min(g1, I.chunk0 + I.nchunks);
+    __syncthreads();  // both groups are done with the previous tables
+    {
       const uint4 *src = (const uint4 *)I.lut;
       uint4 *dst = (uint4 *)&S.tabs;
-      for (uint32_t i = tid; i < sizeof(DecodeTables) / 16; i += kThreads) dst[i] = src[i];
-      cur = it;
-      __syncthreads();
-    }
-    if (S.tabs.err) {
-      if (tid == 0) set_status(b.status, kFlagCorrupt);
-      continue;
-    }
-    const uint32_t c = I.first_chunk + (g - I.chunk0);
-    const uint64_t i0 = (uint64_t)c * b.chunk_elems;
-    const uint32_t cnt = (uint32_t)min((uint64_t)b.chunk_elems, I.n - i0);
-    const uint64_t B0 = I.off[c], B1 = I.off[c + 1], Bt = I.off[I.total_chunks];
-    // the stream must hold every chunk's bits plus 16 readable bytes
-    const bool sane = I.off[0] == 0 && B0 <= B1 && B1 <= Bt && (Bt + 7) / 8 + 16 <= I.stream_cap &&
-                      B1 - B0 >= cnt && B1 - B0 <= (uint64_t)cnt * S.tabs.maxlen;
-    if (!sane) {
-      if (tid == 0) set_status(b.status, kFlagCorrupt);
-      continue;
-    }
-    const uint32_t nbits = (uint32_t)(B1 - B0);
-    const uint64_t lo = (B0 >> 3) & ~uint64_t(15);
-    const uint64_t hi = (((B1 + 7) >> 3) + 8 + 15) & ~uint64_t(15);
-    const uint32_t rel0 = (uint32_t)(B0 - lo * 8);
-    bool ok;
-    if (hi - lo <= (uint64_t)kStageBytes && hi <= I.stream_cap) {
-      const uint32_t bytes = (uint32_t)(hi - lo);
-      // order this CTA's earlier generic accesses of the stage before the
-      // asynchronous copy overwrites it
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      __syncthreads();
-      if (tid == 0) {
-        mbar_expect_tx(&S.mbar, bytes);
-        bulk_g2s(S.stage, I.stream + lo, bytes, &S.mbar);
-      }
-      uint32_t spins = 0;
-      while (!mbar_try_wait(&S.mbar, parity) && ++spins < kSpinLimit) {
-      }
-      if (__syncthreads_or(spins >= kSpinLimit)) {
-        // the copy never completed: give it one more bounded wait, then stop
-        spins = 0;
-        while (!mbar_try_wait(&S.mbar, parity) && ++spins < kSpinLimit) {
-        }
-        if (tid == 0) set_status(b.status, kFlagTimeout);
-        return;
-      }
-      parity ^= 1u;
-      const uint32_t nw = bytes / 4;
-      for (uint32_t i = tid; i < nw; i += kThreads) S.stage[i] = bswap32(S.stage[i]);
-      if (tid < 2) S.stage[nw + tid] = 0u;
-      __syncthreads();
-      BitSrc<true> src{S.stage};
-      ok = decode_chunk<true>(S, src, rel0, nbits, cnt, &timeout);
-    } else {
-      BitSrc<false> src{(const uint32_t *)(I.stream + lo)};
-      ok = decode_chunk<false>(S, src, rel0, nbits, cnt, &timeout);
-    }
-    if (!ok) {
-      if (tid == 0) set_status(b.status, timeout ? kFlagTimeout | kFlagCorrupt : kFlagCorrupt);
-      __syncthreads();
-      continue;
-    }
-
-    // 6. merge exponents with sign/mantissa, 16-byte stores
-    if (DT == EH_BF16) {
-      const uint8_t *smp = I.sm + i0;
-      uint16_t *outp = (uint16_t *)I.out + (i0 - I.elem0);
-      const uint32_t nvec = cnt / 16;
-      #pragma unroll 2
-      for (uint32_t v = tid; v < nvec; v += kThreads) {
-        const uint4 m = __ldg((const uint4 *)smp + v);
-        const uint4 e = *(const uint4 *)(S.exps + 16 * v);
-        const uint32_t mw[4] = {m.x, m.y, m.z, m.w}, ew[4] = {e.x, e.y, e.z, e.w};
-        uint32_t o[8];
-        #pragma unroll
-        for (int q = 0; q < 4; q++) {
-          o[2 * q] = bf16_merge2(__byte_perm(mw[q], ew[q], 0x5140));
-          o[2 * q + 1] = bf16_merge2(__byte_perm(mw[q], ew[q], 0x7362));
-        }
-        uint4 *dst = (uint4 *)(outp + 16 * (uint64_t)v);
-        dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
-        dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
-      }
-      for (uint32_t i = nvec * 16 + tid; i < cnt; i += kThreads) {
-        const uint32_t s = smp[i], e = S.exps[i];
-        outp[i] = (uint16_t)(((s & 0x80u) << 8) | (e << 7) | (s & 0x7Fu));
-      }
-    } else {
-      const uint8_t *smp = I.sm + i0 / 2;
-      uint8_t *outp = (uint8_t *)I.out + (i0 - I.elem0);
-      const uint32_t nvec = cnt / 16;
-      #pragma unroll 2
-      for (uint32_t v = tid; v < nvec; v += kThreads) {
-        const uint2 m = __ldg((const uint2 *)smp + v);
-        const uint4 e = *(const uint4 *)(S.exps + 16 * v);
-        const uint32_t mh[4] = {m.x & 0xFFFFu, m.x >> 16, m.y & 0xFFFFu, m.y >> 16};
-        const uint32_t ew[4] = {e.x, e.y, e.z, e.w};
-        uint32_t o[4];
-        #pragma unroll
-        for (int q = 0; q < 4; q++) {
-          const uint32_t x = mh[q];
-          const uint32_t t = (x & 0xFu) | ((x & 0xF0u) << 4) | ((x & 0xF00u) << 8) | ((x & 0xF000u) << 12);
-          o[q] = ((t & 0x08080808u) << 4) | ((ew[q] << 3) & 0x78787878u) | (t & 0x07070707u);
-        }
-        *(uint4 *)(outp + 16 * (uint64_t)v) = make_uint4(o[0], o[1], o[2], o[3]);
-      }
-      for (uint32_t i = nvec * 16 + tid; i < cnt; i += kThreads) {
-        const uint32_t s = (smp[i / 2] >> (4 * (i & 1))) & 0xFu, e = S.exps[i];
-        outp[i] = (uint8_t)(((s & 8u) << 4) | (e << 3) | (s & 7u));
-      }
+      for (uint32_t i = tid; i < sizeof(DecodeTables) / 16; i += kDecThreads) dst[i] = src[i];
     }
     __syncthreads();
+    const bool terr = S.tabs.err != 0;
+    uint32_t g = seg + grp;
+    ChunkInfo ci;
+    ci.fits = false;
+    if (g < seg_end) {
+      ci = chunk_info(b, g);
+      if (ci.fits && gtid == 0) issue_stage(G, b, ci);
+      pending = ci.fits;
+    }
+    for (; g < seg_end; g += kNumGroups) {
+      const uint64_t i0 = (uint64_t)ci.c * b.chunk_elems;
+      const uint32_t cnt = ci.cnt;
+      bool ok = ci.ok && !terr && !S.abort_flag;
+
+      // the exponent words are OR-ed in: clear them
+      for (uint32_t i = gtid; i < kExpBytes / 16; i += kGroupThreads) ((uint4 *)G.exps)[i] = make_uint4(0, 0, 0, 0);
+      if (ci.fits) {
+        uint32_t spins = 0;
+        while (!mbar_try_wait(&G.mbar, parity) && ++spins < kSpinLimit) {
+        }
+        if (gsync_or(id, spins >= kSpinLimit)) {
+          if (gtid == 0) {
+            set_status(b.status, kFlagTimeout);
+            S.abort_flag = 1;
+          }
+          ok = false;
+        } else {
+          parity ^= 1u;
+          pending = false;
+        }
+      } else {
+        gsync(id);  // the cleared exponent buffer is visible to the group
+      }
+      if (ok) {
+        if (ci.fits) ok = decode_chunk<true>(G, S.tabs, G.stage, ci.rel0, ci.nbits, cnt, id, gtid, &timeout);
+        else
+          ok = decode_chunk<false>(G, S.tabs, (const uint32_t *)(I.stream + ci.lo), ci.rel0, ci.nbits, cnt, id,
+                                   gtid, &timeout);
+        if (!ok && gtid == 0) set_status(b.status, timeout ? kFlagTimeout | kFlagCorrupt : kFlagCorrupt);
+      } else if (gtid == 0 && !S.abort_flag) {
+        set_status(b.status, kFlagCorrupt);
+      }
+
+      // the stage is free: start copying the group's next chunk
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      gsync(id);
+      ChunkInfo cn;
+      cn.fits = false;
+      if (g + kNumGroups < seg_end && !pending && !S.abort_flag) {
+        cn = chunk_info(b, g + kNumGroups);
+        if (cn.fits && gtid == 0) issue_stage(G, b, cn);
+        pending = cn.fits;
+      } else if (g + kNumGroups < seg_end) {
+        cn = chunk_info(b, g + kNumGroups);
+        cn.fits = false;
+      }
+
+      // 6. merge exponents with sign/mantissa, 16-byte coalesced stores
+      if (ok) {
+        const uint32_t nvec = cnt / 16;
+        if (DT == EH_BF16) {
+          const uint8_t *smp = I.sm + i0;
+          uint16_t *outp = (uint16_t *)I.out + (i0 - I.elem0);
+          for (uint32_t v0 = gtid; v0 < nvec; v0 += 4 * kGroupThreads) {
+            uint4 m[4];
+            #pragma unroll
+            for (int u = 0; u < 4; u++) {
+              const uint32_t v = v0 + u * kGroupThreads;
+              m[u] = v < nvec ? ld_nc16(smp + 16 * (uint64_t)v) : make_uint4(0, 0, 0, 0);
+            }
+            #pragma unroll
+            for (int u = 0; u < 4; u++) {
+              const uint32_t v = v0 + u * kGroupThreads;
+              if (v < nvec) {
+                const uint32_t *ew = (const uint32_t *)(G.exps + exp_slot(16 * v));
+                const uint32_t mw[4] = {m[u].x, m[u].y, m[u].z, m[u].w};
+                uint32_t o[8];
+                #pragma unroll
+                for (int q = 0; q < 4; q++) {
+                  const uint32_t e = ew[q];
+                  o[2 * q] = bf16_merge2(__byte_perm(mw[q], e, 0x5140));
+                  o[2 * q + 1] = bf16_merge2(__byte_perm(mw[q], e, 0x7362));
+                }
+                uint4 *dst = (uint4 *)(outp + 16 * (uint64_t)v);
+                dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
+                dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
+              }
+            }
+          }
+          for (uint32_t i = nvec * 16 + gtid; i < cnt; i += kGroupThreads) {
+            const uint32_t sm = smp[i], e = G.exps[exp_slot(i)];
+            outp[i] = (uint16_t)(((sm & 0x80u) << 8) | (e << 7) | (sm & 0x7Fu));
+          }
+        } else {
+          const uint8_t *smp = I.sm + i0 / 2;
+          uint8_t *outp = (uint8_t *)I.out + (i0 - I.elem0);
+          for (uint32_t v0 = gtid; v0 < nvec; v0 += 4 * kGroupThreads) {
+            uint2 m[4];
+            #pragma unroll
+            for (int u = 0; u < 4; u++) {
+              const uint32_t v = v0 + u * kGroupThreads;
+              m[u] = v < nvec ? ld_nc8(smp + 8 * (uint64_t)v) : make_uint2(0, 0);
+            }
+            #pragma unroll
+            for (int u = 0; u < 4; u++) {
+              const uint32_t v = v0 + u * kGroupThreads;
+              if (v < nvec) {
+                const uint32_t *ew = (const uint32_t *)(G.exps + exp_slot(16 * v));
+                uint4 o;
+                o.x = fp8_merge4(m[u].x & 0xFFFFu, ew[0]);
+                o.y = fp8_merge4(m[u].x >> 16, ew[1]);
+                o.z = fp8_merge4(m[u].y & 0xFFFFu, ew[2]);
+                o.w = fp8_merge4(m[u].y >> 16, ew[3]);
+                *(uint4 *)(outp + 16 * (uint64_t)v) = o;
+              }
+            }
+          }
+          for (uint32_t i = nvec * 16 + gtid; i < cnt; i += kGroupThreads) {
+            const uint32_t sm = (smp[i / 2] >> (4 * (i & 1))) & 0xFu, e = G.exps[exp_slot(i)];
+            outp[i] = (uint8_t)(((sm & 8u) << 4) | (e << 3) | (sm & 7u));
+          }
+        }
+      }
+      gsync(id);  // the exponent buffer may be cleared for the next chunk
+      ci = cn;
+    }
+    seg = seg_end;
   }
+  // a copy still in flight (only after an abort) must land before the exit
+  if (pending) {
+    uint32_t spins = 0;
+    while (!mbar_try_wait(&G.mbar, parity) && ++spins < kSpinLimit) {
+    }
+  }
+  __syncthreads();
 }
 
 }  // namespace
@@ -516,10 +805,10 @@ cudaError_t launch_tables(const Batch &b, cudaStream_t s) {
 cudaError_t launch_decode(const Batch &b, cudaStream_t s, int num_sms) {
   if (b.total_chunks == 0) return cudaSuccess;
   const size_t smem = sizeof(DecodeSmem) + 128;
-  uint32_t grid = (uint32_t)num_sms * 2;
+  uint32_t grid = (uint32_t)num_sms;
   if (grid > b.total_chunks) grid = b.total_chunks;
-  if (b.dtype == EH_BF16) decode_kernel<EH_BF16><<<grid, kThreads, smem, s>>>(b);
-  else decode_kernel<EH_FP8_E4M3><<<grid, kThreads, smem, s>>>(b);
+  if (b.dtype == EH_BF16) decode_kernel<EH_BF16><<<grid, kDecThreads, smem, s>>>(b);
+  else decode_kernel<EH_FP8_E4M3><<<grid, kDecThreads, smem, s>>>(b);
   return cudaGetLastError();
 }
 

@@ -8,13 +8,14 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
-#include "../../include/exphuff.h"
+#include "exphuff.h"
 
 namespace eh {
 
-constexpr int kThreads = 512;           // threads per CTA of the chunk kernels
+constexpr int kThreads = 512;           // threads per CTA of the compress kernels
+constexpr int kDecThreads = 1024;       // threads per CTA of the decoder (one CTA per SM)
 constexpr int kMaxChunk = 65536;        // largest chunk (elements)
-constexpr int kNumSub = 8;              // second-level decode tables per codebook
+constexpr int kNumSub = 4;              // second-level decode tables per codebook
 constexpr int kStageBytes = 32 * 1024;  // shared-memory window for one chunk's stream
 
 // status word flags (bitwise OR of everything a call observed)
@@ -78,17 +79,20 @@ __device__ __forceinline__ void set_status(uint32_t *status, uint32_t flag) {
 // Decode tables for one codebook, built by the table kernel into the
 // workspace and copied to shared memory by each decoding CTA.
 //
-// First level, indexed by the next 8 stream bits.  u64 entry:
-//   bits  0..31  up to four decoded symbols, 8 bits each (first in bits 0..7)
-//   bits 32..35  length of the first code if it is <= 8 bits, else 0
-//   bits 36..39  bits consumed by the `cnt` complete codes in the 8 bits
-//   bits 40..42  cnt: complete codes inside the 8 bits (0..4)
-//   bits 48..55  second-level table of this prefix (0xFF: none -> search)
+// First level, indexed by the next kLutBits stream bits, as two u32 arrays:
+//   l1sym:  up to four decoded symbols, 8 bits each (first in bits 0..7)
+//   l1meta: bits  0..3  bits consumed by the `cnt` complete codes in the index
+//           bits  4..6  cnt: complete codes inside the index bits (0..4)
+//           bits  7..18 bit i set when one of those codes starts at offset i
+//           bits 19..24 second-level table of this prefix (kNoSub: none)
 // Second level, indexed by the 8 bits after the prefix.  u32 entry:
-//   bits 0..7 symbol, bits 8..13 code length 9..16 (0: longer -> search).
+//   bits 0..7 symbol, bits 8..13 code length (0: longer -> search).
 // The search path handles any length up to 32 with the canonical limits.
+constexpr int kLutBits = 12;
+constexpr uint32_t kNoSub = 63;
 struct DecodeTables {
-  uint64_t l1[256];
+  uint32_t l1meta[1 << kLutBits];
+  uint32_t l1sym[1 << kLutBits];
   uint32_t sub[kNumSub][256];
   uint64_t lim[33];        // (first[L] + count[L]) << (32 - L): left-justified limits
   uint32_t first[33];      // first canonical code of length L
