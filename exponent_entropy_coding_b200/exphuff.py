@@ -21,6 +21,7 @@ EH_FP8_E4M3 = 1
 EH_DEFAULT_CHUNK_ELEMS = 65536
 EH_MAX_CODE_LEN = 32
 EH_MAX_BATCH = 16
+EH_NOALLOC_MAX_BATCH = 8
 
 STATUS = {0: "EH_OK", 1: "EH_ERR_INVALID_ARG", 2: "EH_ERR_UNSUPPORTED", 3: "EH_ERR_INFEASIBLE",
           4: "EH_ERR_CUDA", 5: "EH_ERR_CORRUPT", 6: "EH_ERR_TIMEOUT", 7: "EH_ERR_NOMEM"}
@@ -29,7 +30,8 @@ EH_ERR_CUDA, EH_ERR_CORRUPT, EH_ERR_TIMEOUT, EH_ERR_NOMEM = 4, 5, 6, 7
 
 EXPORTED = ["eh_plan", "eh_compress_bound", "eh_compress_batch_workspace", "eh_compress",
             "eh_compress_batch", "eh_decompress_workspace", "eh_decompress", "eh_decompress_batch",
-            "eh_decompress_chunks", "eh_get_status", "eh_status_str", "eh_version"]
+            "eh_decompress_chunks", "eh_decompress_batch_noalloc", "eh_get_status", "eh_status_str",
+            "eh_version"]
 
 
 class EhError(RuntimeError):
@@ -72,6 +74,7 @@ def lib():
             "eh_decompress": [P(eh_plan_t), P(eh_compressed_t), vp, vp, u64, vp],
             "eh_decompress_batch": [P(eh_plan_t), C.c_int, P(eh_compressed_t), P(vp), vp, u64, vp],
             "eh_decompress_chunks": [P(eh_plan_t), P(eh_compressed_t), u32, u32, vp, vp, u64, vp],
+            "eh_decompress_batch_noalloc": [P(eh_plan_t), C.c_int, P(eh_compressed_t), P(vp), vp],
             "eh_get_status": [vp, vp],
             "eh_status_str": [C.c_int],
             "eh_version": [],
@@ -241,6 +244,15 @@ def decompress_batch(p: eh_plan_t, cs: List[Compressed], outs: List[torch.Tensor
                                    workspace.numel(), _stream_ptr(stream))
     _check(rc, "eh_decompress_batch")
     return outs
+
+
+def decompress_batch_noalloc(p: eh_plan_t, cs: List[Compressed], outs: List[torch.Tensor], stream=None) -> int:
+    """Block decompression with the library's fixed scratch (no workspace, no
+    allocation); waits for the stream and returns the call's status code."""
+    k = len(cs)
+    structs = (eh_compressed_t * k)(*[c.struct() for c in cs])
+    optrs = (C.c_void_p * k)(*[o.data_ptr() if o.numel() else None for o in outs])
+    return lib().eh_decompress_batch_noalloc(C.byref(p), k, structs, optrs, _stream_ptr(stream))
 
 
 def decompress(c: Compressed, p: Optional[eh_plan_t] = None, out: Optional[torch.Tensor] = None,

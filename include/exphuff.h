@@ -70,6 +70,7 @@ extern "C" {
 #define EH_DEFAULT_CHUNK_ELEMS 65536u /* elements per chunk (one K/V page)   */
 #define EH_MAX_CODE_LEN 32u           /* longest code the format allows     */
 #define EH_MAX_BATCH 16               /* tensors per batched launch         */
+#define EH_NOALLOC_MAX_BATCH 8        /* tensors per eh_decompress_batch_noalloc */
 
 typedef enum { EH_BF16 = 0, EH_FP8_E4M3 = 1 } eh_dtype;
 
@@ -170,6 +171,22 @@ EH_API eh_status eh_decompress_chunks(const eh_plan_t *plan, const eh_compressed
                                uint32_t first, uint32_t count, void *out,
                                void *workspace, uint64_t workspace_bytes,
                                void *stream);
+
+/* eh_decompress_batch without a workspace, for callers that cannot allocate
+ * device memory (code running during CUDA graph capture, runtimes that plan
+ * all device memory ahead of time, allocator callbacks).  There is no
+ * counterpart on the pages: it is a packaging variant of block decompression.
+ * The decoder's scratch lives in a fixed device array inside the library
+ * (256 + EH_NOALLOC_MAX_BATCH * 37,888 bytes, held by every GPU that uses the
+ * library until the process exits); nothing is allocated.  k must be in
+ * [1, EH_NOALLOC_MAX_BATCH], else EH_ERR_INVALID_ARG.  The first call on a
+ * device looks up the array's device address, so make that first call
+ * before any stream capture.  The call waits for `stream` and returns the
+ * call's status (EH_OK or a data error).  All calls share the array: calls
+ * that overlap on the GPU race and must not be issued. */
+EH_API eh_status eh_decompress_batch_noalloc(const eh_plan_t *plan, int k,
+                                             const eh_compressed_t *cs,
+                                             void *const *outs, void *stream);
 
 /* Waits for `stream` and returns the status word of `workspace`: EH_OK,
  * EH_ERR_CORRUPT, EH_ERR_INFEASIBLE or EH_ERR_TIMEOUT.  Every compress or
