@@ -30,6 +30,7 @@ cudaError_t device_setup(int *num_sms) {
   std::call_once(d.once, [&d, dev]() {
     d.err = cudaDeviceGetAttribute(&d.num_sms, cudaDevAttrMultiProcessorCount, dev);
     if (d.err == cudaSuccess) d.err = configure_decode();
+    if (d.err == cudaSuccess) d.err = configure_encode();
   });
   *num_sms = d.num_sms;
   return d.err;

@@ -28,12 +28,6 @@ __device__ __forceinline__ uint4 ld_stream(const void *p) {
   return v;
 }
 
-__device__ __forceinline__ uint2 ld_stream8(const void *p) {
-  uint2 v;
-  asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "l"(p));
-  return v;
-}
-
 // BF16 pair in one word -> the two sign+mantissa bytes (s<<7 | m7), low
 // element in the low byte.
 __device__ __forceinline__ uint32_t bf16x2_sm(uint32_t x) {
@@ -345,9 +339,9 @@ __global__ void __launch_bounds__(256) offsets_kernel(const __grid_constant__ Ba
 }
 
 // ---------------------------------------------------------------- encode
-constexpr int kEncPerThread = 8;                        // values per thread per tile
-constexpr int kEncTile = kThreads * kEncPerThread;       // 4096 values
-constexpr int kRingWords = 8192;                         // 2 tiles of 32-bit codes
+constexpr int kEncPerThread = 16;                       // values per thread per tile
+constexpr int kEncTile = kThreads * kEncPerThread;       // 8192 values
+constexpr int kRingWords = 16384;                        // > one tile of 32-bit codes + carry
 constexpr uint32_t kRingMask = kRingWords - 1;
 
 __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t *wsum, uint32_t *total) {
@@ -374,11 +368,68 @@ __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t *wsum, 
   return (warp ? wsum[warp - 1] : 0u) + x - v;
 }
 
+// Loads the exponent fields of this thread's 16 values of a tile (fewer at
+// the end of the chunk; missing values get exponent 0 and are masked by the
+// caller).
+template <int DT>
+__device__ __forceinline__ void load_exps(const void *in, uint32_t idx, uint32_t cnt, uint4 &p, uint4 &q) {
+  if (DT == EH_BF16) {
+    const uint16_t *x = (const uint16_t *)in;
+    if (idx + 16 <= cnt) {
+      p = ld_stream(x + idx);
+      q = ld_stream(x + idx + 8);
+    } else {
+      uint32_t w[8];
+      #pragma unroll
+      for (int j = 0; j < 8; j++) {
+        const uint32_t a = idx + 2 * j < cnt ? x[idx + 2 * j] : 0u;
+        const uint32_t b2 = idx + 2 * j + 1 < cnt ? x[idx + 2 * j + 1] : 0u;
+        w[j] = a | (b2 << 16);
+      }
+      p = make_uint4(w[0], w[1], w[2], w[3]);
+      q = make_uint4(w[4], w[5], w[6], w[7]);
+    }
+  } else {
+    const uint8_t *x = (const uint8_t *)in;
+    if (idx + 16 <= cnt) {
+      p = ld_stream(x + idx);
+    } else {
+      uint32_t w[4] = {0, 0, 0, 0};
+      #pragma unroll
+      for (int j = 0; j < 16; j++)
+        if (idx + j < cnt) w[j / 4] |= (uint32_t)x[idx + j] << (8 * (j & 3));
+      p = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+    q = make_uint4(0, 0, 0, 0);
+  }
+}
+
+template <int DT>
+__device__ __forceinline__ uint32_t exp_of(const uint4 &p, const uint4 &q, int j) {
+  if (DT == EH_BF16) {
+    const uint32_t w[8] = {p.x, p.y, p.z, p.w, q.x, q.y, q.z, q.w};
+    return (w[j >> 1] >> ((j & 1) ? 23 : 7)) & 0xFFu;
+  } else {
+    const uint32_t w[4] = {p.x, p.y, p.z, p.w};
+    return (w[j >> 2] >> (8 * (j & 3) + 3)) & 0xFu;
+  }
+}
+
+// ORs the `nbits` (<= 32) code bits held right-aligned in `acc` into the
+// ring at stream bit `pos`.
+__device__ __forceinline__ void ring_or(uint32_t *ring, uint64_t pos, uint32_t acc, uint32_t nbits) {
+  const uint32_t s = (uint32_t)(pos & 31);
+  const uint64_t w = pos >> 5;
+  const uint64_t y = (uint64_t)acc << (64 - s - nbits);
+  atomicOr(&ring[w & kRingMask], (uint32_t)(y >> 32));
+  if (s + nbits > 32) atomicOr(&ring[(w + 1) & kRingMask], (uint32_t)y);
+}
+
 template <int DT>
 __global__ void __launch_bounds__(kThreads, 2) encode_kernel(const __grid_constant__ Batch b) {
   constexpr int A = DT == EH_BF16 ? 256 : 16;
   extern __shared__ uint32_t ring[];  // kRingWords words, code bits in MSB-first order
-  __shared__ uint2 tab[A];            // (code, length)
+  __shared__ uint2 tab[A];            // (code left-aligned in 32 bits, length)
   __shared__ uint32_t wsum[kThreads / 32];
   const uint32_t g = blockIdx.x;
   const Item &I = b.item[find_item(b, g)];
@@ -386,83 +437,52 @@ __global__ void __launch_bounds__(kThreads, 2) encode_kernel(const __grid_consta
   const uint64_t i0 = (uint64_t)c * b.chunk_elems;
   const uint32_t cnt = (uint32_t)min((uint64_t)b.chunk_elems, I.n - i0);
   const int tid = threadIdx.x;
-  for (int s = tid; s < A; s += kThreads) tab[s] = make_uint2(I.code[s], I.code_len[s]);
+  for (int s2 = tid; s2 < A; s2 += kThreads) {
+    const uint32_t l = I.code_len[s2];
+    tab[s2] = make_uint2(l ? I.code[s2] << (32 - l) : 0u, l);
+  }
   for (int i = tid; i < kRingWords; i += kThreads) ring[i] = 0u;
   const uint64_t bit0 = I.off[c], bit1 = I.off[c + 1];
   uint32_t *gs = (uint32_t *)I.stream;
+  const uint8_t *in = (const uint8_t *)I.in + i0 * (DT == EH_BF16 ? 2 : 1);
   __syncthreads();
 
   uint64_t tile_base = bit0;           // stream bit where the current tile starts
   uint64_t wdone = bit0 >> 5;          // first stream word not yet written out
+  uint4 np, nq;
+  load_exps<DT>(in, tid * kEncPerThread, cnt, np, nq);
   for (uint32_t t0 = 0; t0 < cnt; t0 += kEncTile) {
     const uint32_t idx = t0 + tid * kEncPerThread;
-    uint32_t e[kEncPerThread];
-    uint32_t nvalid = 0;
-    if (DT == EH_BF16) {
-      const uint16_t *in = (const uint16_t *)I.in + i0;
-      if (idx + kEncPerThread <= cnt) {
-        uint4 p = ld_stream(in + idx);
-        uint32_t w[4] = {p.x, p.y, p.z, p.w};
-        #pragma unroll
-        for (int j = 0; j < 4; j++) {
-          e[2 * j] = (w[j] >> 7) & 0xFFu;
-          e[2 * j + 1] = (w[j] >> 23) & 0xFFu;
-        }
-        nvalid = kEncPerThread;
-      } else {
-        #pragma unroll
-        for (int j = 0; j < kEncPerThread; j++) e[j] = idx + j < cnt ? (in[idx + j] >> 7) & 0xFFu : 0u;
-        nvalid = idx < cnt ? cnt - idx : 0;
-      }
-    } else {
-      const uint8_t *in = (const uint8_t *)I.in + i0;
-      if (idx + kEncPerThread <= cnt) {
-        uint2 p = ld_stream8(in + idx);
-        #pragma unroll
-        for (int j = 0; j < 4; j++) {
-          e[j] = (p.x >> (8 * j + 3)) & 0xFu;
-          e[4 + j] = (p.y >> (8 * j + 3)) & 0xFu;
-        }
-        nvalid = kEncPerThread;
-      } else {
-        #pragma unroll
-        for (int j = 0; j < kEncPerThread; j++) e[j] = idx + j < cnt ? (in[idx + j] >> 3) & 0xFu : 0u;
-        nvalid = idx < cnt ? cnt - idx : 0;
-      }
-    }
-    uint2 cl[kEncPerThread];
-    uint32_t mybits = 0;
+    const uint4 p = np, q = nq;
+    if (t0 + kEncTile < cnt) load_exps<DT>(in, idx + kEncTile, cnt, np, nq);
+    // two groups of 8 codes, each concatenated in a 32-bit accumulator when
+    // it fits (the usual case); longer groups take the per-code path
+    uint32_t acc[2] = {0u, 0u}, tot[2] = {0u, 0u};
     #pragma unroll
     for (int j = 0; j < kEncPerThread; j++) {
-      cl[j] = tab[e[j]];
-      if ((uint32_t)j >= nvalid) cl[j].y = 0u;
-      mybits += cl[j].y;
+      uint2 cl = tab[exp_of<DT>(p, q, j)];
+      if (idx + j >= cnt) cl = make_uint2(0u, 0u);
+      acc[j >> 3] = __funnelshift_lc(cl.x, acc[j >> 3], cl.y);
+      tot[j >> 3] += cl.y;
     }
     uint32_t total;
-    const uint32_t excl = block_excl_scan(mybits, wsum, &total);
-    if (mybits) {
-      // stream the codes through a 64-bit accumulator aligned to the global
-      // word grid; complete words go to the ring with OR (two neighbours may
-      // share a word)
-      uint64_t pos = tile_base + excl;
-      uint64_t w = pos >> 5;
-      uint32_t nb = (uint32_t)(pos & 31);
-      uint64_t acc = 0;
-      #pragma unroll
-      for (int j = 0; j < kEncPerThread; j++) {
-        const uint32_t l = cl[j].y;
-        if (l) {
-          acc |= (uint64_t)cl[j].x << (64 - nb - l);
-          nb += l;
-          if (nb >= 32) {
-            atomicOr(&ring[w & kRingMask], (uint32_t)(acc >> 32));
-            acc <<= 32;
-            nb -= 32;
-            w++;
-          }
+    const uint32_t excl = block_excl_scan(tot[0] + tot[1], wsum, &total);
+    uint64_t pos = tile_base + excl;
+    #pragma unroll
+    for (int h = 0; h < 2; h++) {
+      if (tot[h] == 0) continue;
+      if (tot[h] <= 32) {
+        ring_or(ring, pos, acc[h], tot[h]);
+      } else {
+        uint64_t pp = pos;
+        for (int j = 8 * h; j < 8 * h + 8; j++) {
+          uint2 cl = tab[exp_of<DT>(p, q, j)];
+          if (idx + j >= cnt || cl.y == 0) continue;
+          ring_or(ring, pp, cl.x >> (32 - cl.y), cl.y);
+          pp += cl.y;
         }
       }
-      if (nb) atomicOr(&ring[w & kRingMask], (uint32_t)(acc >> 32));
+      pos += tot[h];
     }
     __syncthreads();
     tile_base += total;
@@ -477,7 +497,6 @@ __global__ void __launch_bounds__(kThreads, 2) encode_kernel(const __grid_consta
       else gs[wi] = val;
     }
     wdone = wend;
-    __syncthreads();
   }
 }
 
@@ -500,6 +519,13 @@ cudaError_t launch_offsets(const Batch &b, cudaStream_t s) {
   if (grid == 0) grid = 1;  // the last CTA still writes off[0] = 0 and the bit totals
   offsets_kernel<<<grid, 256, 0, s>>>(b);
   return cudaGetLastError();
+}
+
+cudaError_t configure_encode() {
+  const int smem = kRingWords * (int)sizeof(uint32_t);
+  cudaError_t e = cudaFuncSetAttribute(encode_kernel<EH_BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  return cudaFuncSetAttribute(encode_kernel<EH_FP8_E4M3>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
 }
 
 cudaError_t launch_encode(const Batch &b, cudaStream_t s) {

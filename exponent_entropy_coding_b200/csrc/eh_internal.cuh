@@ -116,5 +116,6 @@ cudaError_t launch_encode(const Batch &b, cudaStream_t s);
 cudaError_t launch_tables(const Batch &b, cudaStream_t s);
 cudaError_t launch_decode(const Batch &b, cudaStream_t s, int num_sms);
 cudaError_t configure_decode();  // once per device, before the first decode launch
+cudaError_t configure_encode();  // once per device, before the first encode launch
 
 }  // namespace eh
