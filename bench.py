@@ -32,7 +32,7 @@ FALLBACK_HBM_GBS = 6650.0
 # DRAM traffic per decode launch on the full block, from one ncu capture
 # (dram__bytes_read.sum + dram__bytes_write.sum), valid only for the decoder
 # source it was taken on.
-DECODE_TRAFFIC = {"bytes": None, "source_sha": None}
+DECODE_TRAFFIC = {"bytes": 293231616 + 374882304, "source_sha": "531e4b32324d2310"}
 
 
 def decoder_source_sha():
