@@ -119,8 +119,14 @@ eh_status eh_compress_batch_workspace(const eh_plan_t *plan, int k, const uint64
   return EH_OK;
 }
 
-eh_status eh_compress_batch(const eh_plan_t *plan, int k, const void *const *ins, eh_compressed_t *outs,
-                            uint64_t *bits_dev, void *workspace, uint64_t workspace_bytes, void *stream) {
+}  // extern "C"
+
+namespace {
+
+// Checks the arguments of a compress call and lays out its launch
+// descriptor and workspace.
+eh_status prepare_compress(const eh_plan_t *plan, int k, const void *const *ins, eh_compressed_t *outs,
+                           uint64_t *bits_dev, void *workspace, uint64_t workspace_bytes, Batch *bp) {
   if (!plan_ok(plan) || k < 1 || k > EH_MAX_BATCH || !ins || !outs || !workspace) return EH_ERR_INVALID_ARG;
   if (((uintptr_t)workspace & 255u) != 0 || (bits_dev && ((uintptr_t)bits_dev & 7u))) return EH_ERR_INVALID_ARG;
   uint64_t ns[EH_MAX_BATCH];
@@ -140,12 +146,9 @@ eh_status eh_compress_batch(const eh_plan_t *plan, int k, const void *const *ins
   }
   if (total_chunks > 0x7FFFFFFFull) return EH_ERR_INVALID_ARG;
   if (workspace_bytes < compress_ws_bytes(plan, k, ns)) return EH_ERR_NOMEM;
-  int num_sms = 0;
-  cudaError_t e = device_setup(&num_sms);
-  if (e != cudaSuccess) return EH_ERR_CUDA;
 
   uint8_t *ws = (uint8_t *)workspace;
-  Batch b;
+  Batch &b = *bp;
   std::memset(&b, 0, sizeof(b));
   b.k = (uint32_t)k;
   b.chunk_elems = plan->chunk_elems;
@@ -185,24 +188,76 @@ eh_status eh_compress_batch(const eh_plan_t *plan, int k, const void *const *ins
     chunk0 += C;
   }
   b.total_chunks = chunk0;
-  cudaStream_t s = (cudaStream_t)stream;
-  if ((e = cudaMemsetAsync(ws, 0, kHeader + (uint64_t)k * kCountsBytes, s)) != cudaSuccess) return EH_ERR_CUDA;
-  if ((e = launch_hist(b, s)) != cudaSuccess) return EH_ERR_CUDA;
-  if ((e = launch_book(b, s)) != cudaSuccess) return EH_ERR_CUDA;
-  if ((e = launch_offsets(b, s)) != cudaSuccess) return EH_ERR_CUDA;
-  if ((e = launch_encode(b, s)) != cudaSuccess) return EH_ERR_CUDA;
   for (int i = 0; i < k; i++) outs[i].n_chunks = b.item[i].nchunks;
-  if (bits_dev) return EH_OK;
+  return EH_OK;
+}
+
+// Codebook, offsets and encode launches, then (without bits_dev) the wait
+// for the bit counts and the status.
+eh_status finish_compress(const Batch &b, int k, eh_compressed_t *outs, bool wait, void *workspace,
+                          cudaStream_t s) {
+  if (launch_book(b, s) != cudaSuccess) return EH_ERR_CUDA;
+  if (launch_offsets(b, s) != cudaSuccess) return EH_ERR_CUDA;
+  if (launch_encode(b, s) != cudaSuccess) return EH_ERR_CUDA;
+  if (!wait) return EH_OK;
   uint64_t host[1 + EH_MAX_BATCH];
-  if ((e = cudaMemcpyAsync(host, ws, 8 + 8 * (uint64_t)k, cudaMemcpyDeviceToHost, s)) != cudaSuccess)
+  if (cudaMemcpyAsync(host, workspace, 8 + 8 * (uint64_t)k, cudaMemcpyDeviceToHost, s) != cudaSuccess)
     return EH_ERR_CUDA;
-  if ((e = cudaStreamSynchronize(s)) != cudaSuccess) return EH_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return EH_ERR_CUDA;
   const uint32_t status = (uint32_t)host[0];
   for (int i = 0; i < k; i++) outs[i].exp_stream_bits = host[1 + i];
   if (status & kFlagInfeasible) return EH_ERR_INFEASIBLE;
   if (status & kFlagTimeout) return EH_ERR_TIMEOUT;
   if (status & kFlagCorrupt) return EH_ERR_CORRUPT;
   return EH_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+eh_status eh_compress_batch(const eh_plan_t *plan, int k, const void *const *ins, eh_compressed_t *outs,
+                            uint64_t *bits_dev, void *workspace, uint64_t workspace_bytes, void *stream) {
+  Batch b;
+  eh_status st = prepare_compress(plan, k, ins, outs, bits_dev, workspace, workspace_bytes, &b);
+  if (st != EH_OK) return st;
+  int num_sms = 0;
+  if (device_setup(&num_sms) != cudaSuccess) return EH_ERR_CUDA;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (cudaMemsetAsync(workspace, 0, kHeader + (uint64_t)k * kCountsBytes, s) != cudaSuccess) return EH_ERR_CUDA;
+  if (launch_hist(b, s) != cudaSuccess) return EH_ERR_CUDA;
+  return finish_compress(b, k, outs, bits_dev == nullptr, workspace, s);
+}
+
+eh_status eh_compress_shard_begin(const eh_plan_t *plan, const void *in, eh_compressed_t *out, uint64_t *counts,
+                                  void *workspace, uint64_t workspace_bytes, void *stream) {
+  if (!counts || ((uintptr_t)counts & 7u)) return EH_ERR_INVALID_ARG;
+  const void *ins[1] = {in};
+  Batch b;
+  eh_status st = prepare_compress(plan, 1, ins, out, nullptr, workspace, workspace_bytes, &b);
+  if (st != EH_OK) return st;
+  b.item[0].counts = counts;
+  int num_sms = 0;
+  if (device_setup(&num_sms) != cudaSuccess) return EH_ERR_CUDA;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (cudaMemsetAsync(workspace, 0, kHeader, s) != cudaSuccess) return EH_ERR_CUDA;
+  if (cudaMemsetAsync(counts, 0, sizeof(uint64_t) * alphabet_of(plan->dtype), s) != cudaSuccess) return EH_ERR_CUDA;
+  if (launch_hist(b, s) != cudaSuccess) return EH_ERR_CUDA;
+  return EH_OK;
+}
+
+eh_status eh_compress_shard_finish(const eh_plan_t *plan, const void *in, eh_compressed_t *out,
+                                   const uint64_t *counts, uint64_t *bits_dev, void *workspace,
+                                   uint64_t workspace_bytes, void *stream) {
+  if (!counts || ((uintptr_t)counts & 7u)) return EH_ERR_INVALID_ARG;
+  const void *ins[1] = {in};
+  Batch b;
+  eh_status st = prepare_compress(plan, 1, ins, out, bits_dev, workspace, workspace_bytes, &b);
+  if (st != EH_OK) return st;
+  b.item[0].counts = const_cast<uint64_t *>(counts);
+  int num_sms = 0;
+  if (device_setup(&num_sms) != cudaSuccess) return EH_ERR_CUDA;
+  return finish_compress(b, 1, out, bits_dev == nullptr, workspace, (cudaStream_t)stream);
 }
 
 eh_status eh_compress(const eh_plan_t *plan, const void *in, uint64_t n, eh_compressed_t *out, void *workspace,

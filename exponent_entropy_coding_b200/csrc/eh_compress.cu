@@ -138,18 +138,32 @@ __global__ void __launch_bounds__(256) book_kernel(const __grid_constant__ Batch
   __shared__ uint32_t nlen[33], firstc[33];
   __shared__ uint32_t xsel[33];     // package-merge: leaves selected per level
   __shared__ uint32_t maxd;
+  __shared__ uint8_t ps[256];       // present symbols, increasing
+  __shared__ uint32_t wpres[8];
 
   const uint64_t c = tid < A ? I.counts[tid] : 0ull;
   cnt[tid] = c;
   len[tid] = 0;
   if (tid <= 32) nlen[tid] = 0;
   if (tid == 0) maxd = 0;
-  const int m = __syncthreads_count(c > 0);
+  // compact list of the present symbols (loops below run over it only)
+  const uint32_t pb = __ballot_sync(0xffffffffu, c > 0);
+  if ((tid & 31) == 0) wpres[tid >> 5] = __popc(pb);
+  __syncthreads();
+  uint32_t pidx = __popc(pb & ((1u << (tid & 31)) - 1u));
+  int m = 0;
+  for (int w = 0; w < 8; w++) {
+    if (w < (tid >> 5)) pidx += wpres[w];
+    m += wpres[w];
+  }
+  if (c > 0) ps[pidx] = (uint8_t)tid;
+  __syncthreads();
   if (c > 0) {
     int r = 0;
-    for (int s2 = 0; s2 < A; s2++) {
-      uint64_t c2 = cnt[s2];
-      r += (c2 > 0) && (c2 < c || (c2 == c && s2 < tid));
+    for (int j = 0; j < m; j++) {
+      const int s2 = ps[j];
+      const uint64_t c2 = cnt[s2];
+      r += c2 < c || (c2 == c && s2 < tid);
     }
     lw[r] = c;
   }
@@ -240,8 +254,9 @@ __global__ void __launch_bounds__(256) book_kernel(const __grid_constant__ Batch
   // (count descending, symbol ascending) order
   if (c > 0 && feasible) {
     uint32_t r = 0;
-    for (int s2 = 0; s2 < A; s2++) {
-      uint64_t c2 = cnt[s2];
+    for (int j = 0; j < m; j++) {
+      const int s2 = ps[j];
+      const uint64_t c2 = cnt[s2];
       r += (c2 > c) || (c2 == c && s2 < tid);
     }
     uint32_t cum = 0, L = 1;
@@ -263,7 +278,10 @@ __global__ void __launch_bounds__(256) book_kernel(const __grid_constant__ Batch
     uint32_t l = len[tid], code = 0;
     if (l) {
       uint32_t k = 0;
-      for (int s2 = 0; s2 < tid; s2++) k += len[s2] == l;
+      for (int j = 0; j < m; j++) {
+        const int s2 = ps[j];
+        k += s2 < tid && len[s2] == l;
+      }
       code = firstc[l] + k;
     }
     I.code_len[tid] = (uint8_t)l;
@@ -278,10 +296,14 @@ __device__ __forceinline__ uint64_t warp_sum64(uint64_t v) {
   return v;
 }
 
-__global__ void __launch_bounds__(256) offsets_kernel(const __grid_constant__ Batch b) {
+constexpr int kOffThreads = 1024;          // one warp per chunk
+constexpr int kOffPerThread = 4;           // chunks per thread in the final scan
+constexpr int kOffTile = kOffThreads * kOffPerThread;
+
+__global__ void __launch_bounds__(kOffThreads) offsets_kernel(const __grid_constant__ Batch b) {
   const int A = alphabet_of(b.dtype);
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const uint32_t g = blockIdx.x * 8 + warp;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const uint32_t g = blockIdx.x * (kOffThreads / 32) + warp;
   if (g < b.total_chunks) {
     const Item &I = b.item[find_item(b, g)];
     const uint32_t c = g - I.chunk0;
@@ -293,49 +315,98 @@ __global__ void __launch_bounds__(256) offsets_kernel(const __grid_constant__ Ba
   __shared__ uint32_t last;
   __threadfence();
   __syncthreads();
-  if (threadIdx.x == 0) last = atomicAdd(b.ticket, 1u) == gridDim.x - 1;
+  if (tid == 0) last = atomicAdd(b.ticket, 1u) == gridDim.x - 1;
   __syncthreads();
   if (!last) return;
   __threadfence();
-  // last CTA: per-tensor exclusive scan of chunk bits -> offsets
-  __shared__ uint64_t wtot[8];
-  for (uint32_t it = 0; it < b.k; it++) {
-    const Item &I = b.item[it];
-    const uint32_t C = I.nchunks;
-    uint32_t *sw = (uint32_t *)I.stream;
-    uint64_t carry = 0;
-    for (uint32_t base = 0; base < C; base += 256) {
-      const uint32_t ci = base + threadIdx.x;
-      uint64_t v = ci < C ? __ldcg(I.cbits + ci) : 0ull;
-      uint64_t x = v;
+
+  // Last CTA: one exclusive scan over the chunks of all tensors in launch
+  // order; a tensor's offsets are that scan minus its value at the tensor's
+  // first chunk.
+  __shared__ uint64_t wtot[kOffThreads / 32];
+  __shared__ uint64_t base[EH_MAX_BATCH + 1];
+  __shared__ uint64_t carry_sh;
+  if (tid == 0) carry_sh = 0;
+  __syncthreads();
+  for (uint32_t t0 = 0; t0 < b.total_chunks; t0 += kOffTile) {
+    const uint32_t g0 = t0 + tid * kOffPerThread;
+    uint64_t v[kOffPerThread], local = 0;
+    #pragma unroll
+    for (int j = 0; j < kOffPerThread; j++) {
+      v[j] = 0;
+      const uint32_t gg = g0 + j;
+      if (gg < b.total_chunks) {
+        const Item &I = b.item[find_item(b, gg)];
+        v[j] = __ldcg(I.cbits + (gg - I.chunk0));
+      }
+      local += v[j];
+    }
+    uint64_t x = local;
+    #pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint64_t y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
+    }
+    if (lane == 31) wtot[warp] = x;
+    __syncthreads();
+    if (warp == 0) {
+      uint64_t t = wtot[lane];
       #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
-        uint64_t y = __shfl_up_sync(0xffffffffu, x, o);
-        if (lane >= o) x += y;
+        const uint64_t y = __shfl_up_sync(0xffffffffu, t, o);
+        if (lane >= o) t += y;
       }
-      if (lane == 31) wtot[warp] = x;
-      __syncthreads();
-      uint64_t pre = 0, tot = 0;
-      for (int w = 0; w < 8; w++) {
-        if (w < warp) pre += wtot[w];
-        tot += wtot[w];
-      }
-      if (ci < C) {
-        uint64_t off = carry + pre + x - v;
-        I.off[ci] = off;
-        sw[off >> 5] = 0u;  // word shared with the previous chunk: cleared for OR
-      }
-      carry += tot;
-      __syncthreads();
+      wtot[lane] = t;
     }
-    if (threadIdx.x == 0) {
-      I.off[C] = carry;
-      if (carry & 31) sw[carry >> 5] = 0u;
-      I.bits_out[0] = carry;
-      if (I.bits_dev) I.bits_dev[0] = carry;
+    __syncthreads();
+    const uint64_t carry = carry_sh;
+    uint64_t run = carry + (warp ? wtot[warp - 1] : 0ull) + x - local;  // exclusive at g0
+    uint64_t ex[kOffPerThread];
+    #pragma unroll
+    for (int j = 0; j < kOffPerThread; j++) {
+      ex[j] = run;
+      const uint32_t gg = g0 + j;
+      if (gg < b.total_chunks) {
+        const int it = find_item(b, gg);
+        if (gg == b.item[it].chunk0) base[it] = run;
+      }
+      run += v[j];
     }
+    __syncthreads();
+    #pragma unroll
+    for (int j = 0; j < kOffPerThread; j++) {
+      const uint32_t gg = g0 + j;
+      if (gg < b.total_chunks) {
+        const int it = find_item(b, gg);
+        const Item &I = b.item[it];
+        const uint64_t off = ex[j] - base[it];
+        I.off[gg - I.chunk0] = off;
+        ((uint32_t *)I.stream)[off >> 5] = 0u;  // word shared with the previous chunk: cleared for OR
+      }
+    }
+    __syncthreads();
+    if (tid == kOffThreads - 1) carry_sh = run;
+    __syncthreads();
   }
-  if (threadIdx.x == 0) *b.ticket = 0u;  // ready for the next call
+  // totals: the scan value after each tensor's last chunk
+  if (tid < (int)b.k) {
+    const Item &I = b.item[tid];
+    uint64_t end;
+    if (I.nchunks == 0) {
+      end = 0;
+    } else {
+      // exclusive value at the next tensor's first chunk, or the grand total
+      uint64_t after = carry_sh;
+      for (uint32_t j = tid + 1; j < b.k; j++)
+        if (b.item[j].nchunks) { after = base[j]; break; }
+      end = after - base[tid];
+    }
+    I.off[I.nchunks] = end;
+    if (end & 31) ((uint32_t *)I.stream)[end >> 5] = 0u;
+    I.bits_out[0] = end;
+    if (I.bits_dev) I.bits_dev[0] = end;
+  }
+  if (tid == 0) *b.ticket = 0u;  // ready for the next call
 }
 
 // ---------------------------------------------------------------- encode
@@ -515,9 +586,9 @@ cudaError_t launch_book(const Batch &b, cudaStream_t s) {
 }
 
 cudaError_t launch_offsets(const Batch &b, cudaStream_t s) {
-  uint32_t grid = (b.total_chunks + 7) / 8;
+  uint32_t grid = (b.total_chunks + kOffThreads / 32 - 1) / (kOffThreads / 32);
   if (grid == 0) grid = 1;  // the last CTA still writes off[0] = 0 and the bit totals
-  offsets_kernel<<<grid, 256, 0, s>>>(b);
+  offsets_kernel<<<grid, kOffThreads, 0, s>>>(b);
   return cudaGetLastError();
 }
 

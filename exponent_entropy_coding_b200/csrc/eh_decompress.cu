@@ -33,31 +33,48 @@ constexpr uint32_t kMaskBits = 64;            // code starts recorded per thread
 constexpr uint32_t kSpinLimit = 1u << 26;     // bounded mbarrier wait
 
 // ---------------------------------------------------------------- tables
-// One CTA of 256 threads per codebook.
+// kTabParts CTAs of 256 threads per codebook; each builds 1/kTabParts of the
+// first level, part 0 also writes the second levels and the limits.
+constexpr uint32_t kTabParts = 8;
+
+// Smallest L in [1, 32] with x < lim[L], 33 if there is none (lim is
+// nondecreasing for a valid code).
+__device__ __forceinline__ uint32_t code_length_of(uint32_t x, const uint64_t *limL) {
+  uint32_t lo = 1, hi = 33;
+  while (lo < hi) {
+    const uint32_t mid = (lo + hi) >> 1;
+    if ((uint64_t)x < limL[mid]) hi = mid;
+    else lo = mid + 1;
+  }
+  return lo;
+}
+
 __global__ void __launch_bounds__(256) tables_kernel(const __grid_constant__ Batch b) {
-  const Item &I = b.item[blockIdx.x];
+  const uint32_t part = blockIdx.x % kTabParts;
+  const Item &I = b.item[blockIdx.x / kTabParts];
   DecodeTables *T = (DecodeTables *)I.lut;
   const int A = alphabet_of(b.dtype);
   const int tid = threadIdx.x;
   __shared__ uint32_t cntL[33], firstL[33], baseL[33];
   __shared__ uint64_t limL[33];
-  __shared__ uint8_t lens[256];
   __shared__ uint8_t srt[256];
   __shared__ unsigned long long kraft;
   __shared__ uint32_t err;
+  __shared__ uint32_t wlen[8][33];  // per warp: symbols of each length
 
   if (blockIdx.x == 0 && tid == 0) {
     *b.status = 0u;  // this call's status starts clean
     *b.ticket = 0u;
   }
   if (tid <= 32) cntL[tid] = 0;
+  for (int i = tid; i < 8 * 33; i += 256) (&wlen[0][0])[i] = 0;
   if (tid == 0) { kraft = 0; err = 0; }
   const uint32_t l = tid < A ? I.code_len[tid] : 0u;
-  lens[tid] = (uint8_t)l;
   __syncthreads();
   if (l > 32) atomicOr(&err, 1u);
   else if (l) {
     atomicAdd(&cntL[l], 1u);
+    atomicAdd(&wlen[tid >> 5][l], 1u);
     atomicAdd(&kraft, 1ull << (32 - l));
   }
   const uint32_t nsym = __syncthreads_count(l > 0 && l <= 32);
@@ -81,41 +98,46 @@ __global__ void __launch_bounds__(256) tables_kernel(const __grid_constant__ Bat
     firstL[0] = baseL[0] = cntL[0] = 0;
     if (kraft > (1ull << 32)) err = 1;
     if (I.n > 0 && nsym == 0) err = 1;
-    T->gcd = g ? g : 1;
-    T->maxlen = maxlen;
-    T->nsym = nsym;
+    if (part == 0) {
+      T->gcd = g ? g : 1;
+      T->maxlen = maxlen;
+      T->nsym = nsym;
+    }
   }
   __syncthreads();
   // symbol order (length, symbol); the stored codes must be the canonical ones
+  // rank among the symbols of equal length below this one: earlier warps'
+  // counts plus the matching lower lanes of this warp
+  const uint32_t same = __match_any_sync(0xffffffffu, l);
   if (tid < A && l && l <= 32) {
-    uint32_t k = 0;
-    for (int s2 = 0; s2 < tid; s2++) k += lens[s2] == l;
+    uint32_t k = __popc(same & ((1u << (tid & 31)) - 1u));
+    for (int w = 0; w < (tid >> 5); w++) k += wlen[w][l];
     srt[baseL[l] + k] = (uint8_t)tid;
     if (I.code[tid] != firstL[l] + k) atomicOr(&err, 1u);
   }
-  if (tid <= 32) {
+  if (tid <= 32 && part == 0) {
     T->first[tid] = firstL[tid];
     T->base[tid] = baseL[tid];
     T->lim[tid] = limL[tid];
   }
   __syncthreads();
   if (err) {  // invalid codebook: nothing below may index with its values
-    if (tid == 0) T->err = err;
+    if (tid == 0 && part == 0) T->err = err;
     return;
   }
-  T->sorted[tid] = tid < (int)nsym ? srt[tid] : (uint8_t)0;
+  if (part == 0) T->sorted[tid] = tid < (int)nsym ? srt[tid] : (uint8_t)0;
 
   // first level.  Codes longer than kLutBits fill the left-justified range
   // [lim[kLutBits], lim[32]), so their prefixes are consecutive: the first
   // kNumSub of them get a second-level table.
   constexpr uint32_t kShift = 32 - kLutBits;
   const uint32_t sub0 = (uint32_t)(limL[kLutBits] >> kShift);
-  for (uint32_t p = tid; p < (1u << kLutBits); p += 256) {
+  constexpr uint32_t kPerPart = (1u << kLutBits) / kTabParts;
+  for (uint32_t p = part * kPerPart + tid; p < (part + 1) * kPerPart; p += 256) {
     uint32_t syms = 0, pos = 0, nc = 0, bnd = 0;
     while (nc < 4 && pos < (uint32_t)kLutBits) {
       const uint32_t x = (p << kShift) << pos;  // next bits, left-justified, zero-filled
-      uint32_t L = 1;
-      while (L <= 32 && (uint64_t)x >= limL[L]) L++;
+      const uint32_t L = code_length_of(x, limL);
       if (L > (uint32_t)kLutBits - pos) break;  // not complete inside the index bits
       const uint32_t v = x >> (32 - L);
       syms |= (uint32_t)srt[baseL[L] + v - firstL[L]] << (8 * nc);
@@ -128,6 +150,7 @@ __global__ void __launch_bounds__(256) tables_kernel(const __grid_constant__ Bat
     T->l1sym[p] = syms;
     T->l1meta[p] = pos | (nc << 4) | (bnd << 7) | (sub << 19);
   }
+  if (part != 0) return;
   // second level: codes of kLutBits+1 .. kLutBits+8 bits
   for (uint32_t j = 0; j < (uint32_t)kNumSub; j++) {
     uint32_t e = 0;
@@ -798,7 +821,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
 }  // namespace
 
 cudaError_t launch_tables(const Batch &b, cudaStream_t s) {
-  tables_kernel<<<b.k, 256, 0, s>>>(b);
+  tables_kernel<<<b.k * kTabParts, 256, 0, s>>>(b);
   return cudaGetLastError();
 }
 

@@ -29,7 +29,8 @@ EH_OK, EH_ERR_INVALID_ARG, EH_ERR_UNSUPPORTED, EH_ERR_INFEASIBLE = 0, 1, 2, 3
 EH_ERR_CUDA, EH_ERR_CORRUPT, EH_ERR_TIMEOUT, EH_ERR_NOMEM = 4, 5, 6, 7
 
 EXPORTED = ["eh_plan", "eh_compress_bound", "eh_compress_batch_workspace", "eh_compress",
-            "eh_compress_batch", "eh_decompress_workspace", "eh_decompress", "eh_decompress_batch",
+            "eh_compress_batch", "eh_compress_shard_begin", "eh_compress_shard_finish",
+            "eh_decompress_workspace", "eh_decompress", "eh_decompress_batch",
             "eh_decompress_chunks", "eh_decompress_batch_noalloc", "eh_get_status", "eh_status_str",
             "eh_version"]
 
@@ -70,6 +71,8 @@ def lib():
             "eh_compress_batch_workspace": [P(eh_plan_t), C.c_int, P(u64), P(u64)],
             "eh_compress": [P(eh_plan_t), vp, u64, P(eh_compressed_t), vp, u64, vp],
             "eh_compress_batch": [P(eh_plan_t), C.c_int, P(vp), P(eh_compressed_t), vp, vp, u64, vp],
+            "eh_compress_shard_begin": [P(eh_plan_t), vp, P(eh_compressed_t), vp, vp, u64, vp],
+            "eh_compress_shard_finish": [P(eh_plan_t), vp, P(eh_compressed_t), vp, vp, vp, u64, vp],
             "eh_decompress_workspace": [P(eh_plan_t), C.c_int, P(u64)],
             "eh_decompress": [P(eh_plan_t), P(eh_compressed_t), vp, vp, u64, vp],
             "eh_decompress_batch": [P(eh_plan_t), C.c_int, P(eh_compressed_t), P(vp), vp, u64, vp],
@@ -228,6 +231,35 @@ def compress(x: torch.Tensor, p: Optional[eh_plan_t] = None, workspace: Optional
                            C.c_void_p(workspace.data_ptr()), workspace.numel(), _stream_ptr(stream))
     _check(rc, "eh_compress")
     out.exp_stream_bits = s.exp_stream_bits
+    return out
+
+
+def compress_shard_begin(x: torch.Tensor, out: Compressed, counts: torch.Tensor, p: eh_plan_t,
+                         workspace: torch.Tensor, stream=None):
+    """Step 1 of sharded compression: local exponent counts (int64[A] on the
+    device, uint64 values) and packed sign/mantissa of the shard."""
+    x = _raw(x)
+    s = out.struct()
+    rc = lib().eh_compress_shard_begin(C.byref(p), C.c_void_p(x.data_ptr()) if x.numel() else None,
+                                       C.byref(s), C.c_void_p(counts.data_ptr()),
+                                       C.c_void_p(workspace.data_ptr()), workspace.numel(),
+                                       _stream_ptr(stream))
+    _check(rc, "eh_compress_shard_begin")
+
+
+def compress_shard_finish(x: torch.Tensor, out: Compressed, counts: torch.Tensor, p: eh_plan_t,
+                          workspace: torch.Tensor, bits_dev: Optional[torch.Tensor] = None, stream=None):
+    """Step 2: codebook from the summed counts, shard offsets and stream."""
+    x = _raw(x)
+    s = out.struct()
+    rc = lib().eh_compress_shard_finish(C.byref(p), C.c_void_p(x.data_ptr()) if x.numel() else None,
+                                        C.byref(s), C.c_void_p(counts.data_ptr()),
+                                        C.c_void_p(bits_dev.data_ptr()) if bits_dev is not None else None,
+                                        C.c_void_p(workspace.data_ptr()), workspace.numel(),
+                                        _stream_ptr(stream))
+    _check(rc, "eh_compress_shard_finish")
+    if bits_dev is None:
+        out.exp_stream_bits = s.exp_stream_bits
     return out
 
 

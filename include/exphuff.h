@@ -146,6 +146,29 @@ EH_API eh_status eh_compress_batch(const eh_plan_t *plan, int k,
                             uint64_t *bits_dev, void *workspace,
                             uint64_t workspace_bytes, void *stream);
 
+/* Compression of one tensor split across GPUs, each rank holding a shard of
+ * whole chunks (the codebook is built from the histogram of the whole tensor, as in
+ * the DFloat11 article, "方法介绍").
+ * Step 1, on every rank: eh_compress_shard_begin histograms the local shard
+ * into counts (device, u64[A], overwritten) and writes its packed
+ * sign/mantissa.  Between the steps the caller sums counts over the ranks
+ * (one all-reduce of A u64 values).  Step 2: eh_compress_shard_finish builds
+ * the codebook from the summed counts (every rank gets the same one), the
+ * shard's chunk offsets (starting at bit 0 of the shard) and its stream.  The
+ * global offset of a shard is the sum of the bit counts of the ranks before
+ * it (one all-gather).  `out`, `workspace` (eh_compress_bound for the shard's
+ * n) and `in` must be the same for both steps.  bits_dev as in
+ * eh_compress_batch.  Decompression of a shard needs no communication. */
+EH_API eh_status eh_compress_shard_begin(const eh_plan_t *plan, const void *in,
+                                         eh_compressed_t *out, uint64_t *counts,
+                                         void *workspace, uint64_t workspace_bytes,
+                                         void *stream);
+EH_API eh_status eh_compress_shard_finish(const eh_plan_t *plan, const void *in,
+                                          eh_compressed_t *out,
+                                          const uint64_t *counts, uint64_t *bits_dev,
+                                          void *workspace, uint64_t workspace_bytes,
+                                          void *stream);
+
 /* Workspace for decompressing up to k tensors in one call. */
 EH_API eh_status eh_decompress_workspace(const eh_plan_t *plan, int k,
                                   uint64_t *workspace_bytes);

@@ -244,3 +244,39 @@ def test_side_stream(eh, oracle):
     s.synchronize()
     assert_same(c, oracle.compress(0, x))
     assert torch.equal(y, t)
+
+
+def test_sharded_compress_on_one_gpu(eh, oracle):
+    # the two shard entry points for three shards of one tensor, with the
+    # counts summed on the device in place of the all-reduce; the stitched
+    # shards equal the single-rank stream and every shard decodes alone
+    from exponent_entropy_coding_b200 import parallel
+    n, world = 5 * 65536 + 123, 3
+    x = synth.normal_bf16(n, seed=31)
+    p = eh.plan(0)
+    counts = torch.zeros(256, dtype=torch.int64, device="cuda")
+    backends, xs = [], []
+    for r in range(world):
+        a, b = parallel.shard_value_range(n, CHUNK, world, r)
+        xr = dev(x[a:b])
+        be = parallel.GpuShardBackend(0)
+        counts += be.begin(xr)
+        backends.append(be)
+        xs.append(xr)
+    outs = []
+    for be, xr in zip(backends, xs):
+        out, bits = be.finish(xr, counts)
+        out.exp_stream_bits = int(bits.item())
+        outs.append(out)
+    ref = oracle.compress(0, x)
+    stream, nbits = parallel.stitch_streams(
+        [(o.exp_stream[:o.stream_bytes()].cpu().numpy(), o.exp_stream_bits) for o in outs])
+    assert nbits == ref.bits and np.array_equal(stream, ref.stream)
+    offs = parallel.stitch_offsets([o.chunk_bit_off.cpu().numpy().view(np.uint64) for o in outs],
+                                   [o.exp_stream_bits for o in outs])
+    assert np.array_equal(offs, ref.chunk_bit_off)
+    assert np.array_equal(np.concatenate([o.sign_mant.cpu().numpy() for o in outs]), ref.sign_mant)
+    for o in outs:
+        assert np.array_equal(o.code_len.cpu().numpy(), ref.code_len)
+    for o, xr in zip(outs, xs):
+        assert torch.equal(eh.decompress(o, p), xr)
