@@ -442,6 +442,33 @@ __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t *wsum, 
 // Loads the exponent fields of this thread's 16 values of a tile (fewer at
 // the end of the chunk; missing values get exponent 0 and are masked by the
 // caller).
+// Exclusive scan over the CTA with a single barrier: every warp publishes
+// its total, then each thread adds up the totals of the warps before its own.
+// The caller must separate two uses of `wsum` by a barrier.
+__device__ __forceinline__ uint32_t block_excl_scan1(uint32_t v, uint32_t *wsum, uint32_t *total) {
+  constexpr int kWarps = kThreads / 32;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  uint32_t x = v;
+  #pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) wsum[warp] = x;
+  __syncthreads();
+  // lane i < kWarps holds warp i's total; prefix over lanes below `warp`
+  const uint32_t t = lane < kWarps ? wsum[lane] : 0u;
+  const uint32_t before = lane < warp ? t : 0u;
+  uint32_t pre = before, all = t;
+  #pragma unroll
+  for (int o = 16; o; o >>= 1) {
+    pre += __shfl_xor_sync(0xffffffffu, pre, o);
+    all += __shfl_xor_sync(0xffffffffu, all, o);
+  }
+  *total = all;
+  return pre + x - v;
+}
+
 template <int DT>
 __device__ __forceinline__ void load_exps(const void *in, uint32_t idx, uint32_t cnt, uint4 &p, uint4 &q) {
   if (DT == EH_BF16) {
@@ -529,15 +556,24 @@ __global__ void __launch_bounds__(kThreads, 2) encode_kernel(const __grid_consta
     // two groups of 8 codes, each concatenated in a 32-bit accumulator when
     // it fits (the usual case); longer groups take the per-code path
     uint32_t acc[2] = {0u, 0u}, tot[2] = {0u, 0u};
-    #pragma unroll
-    for (int j = 0; j < kEncPerThread; j++) {
-      uint2 cl = tab[exp_of<DT>(p, q, j)];
-      if (idx + j >= cnt) cl = make_uint2(0u, 0u);
-      acc[j >> 3] = __funnelshift_lc(cl.x, acc[j >> 3], cl.y);
-      tot[j >> 3] += cl.y;
+    if (idx + kEncPerThread <= cnt) {
+      #pragma unroll
+      for (int j = 0; j < kEncPerThread; j++) {
+        const uint2 cl = tab[exp_of<DT>(p, q, j)];
+        acc[j >> 3] = __funnelshift_lc(cl.x, acc[j >> 3], cl.y);
+        tot[j >> 3] += cl.y;
+      }
+    } else {
+      #pragma unroll
+      for (int j = 0; j < kEncPerThread; j++) {
+        uint2 cl = tab[exp_of<DT>(p, q, j)];
+        if (idx + j >= cnt) cl = make_uint2(0u, 0u);
+        acc[j >> 3] = __funnelshift_lc(cl.x, acc[j >> 3], cl.y);
+        tot[j >> 3] += cl.y;
+      }
     }
     uint32_t total;
-    const uint32_t excl = block_excl_scan(tot[0] + tot[1], wsum, &total);
+    const uint32_t excl = block_excl_scan1(tot[0] + tot[1], wsum, &total);
     uint64_t pos = tile_base + excl;
     #pragma unroll
     for (int h = 0; h < 2; h++) {

@@ -179,39 +179,26 @@ __global__ void __launch_bounds__(256) tables_kernel(const __grid_constant__ Bat
 constexpr uint32_t kExpBytes = kMaxChunk + 4 * (kMaxChunk / 128);
 __device__ __forceinline__ uint32_t exp_slot(uint32_t j) { return j + ((j >> 7) << 2); }
 
-// Bit reader over the chunk's stream words (stored big-endian): a 64-bit
-// buffer holding the next bits MSB-first, refilled 32 bits at a time.
+// 32 stream bits starting at bit p.  Shared-memory stages are byte-swapped
+// once after the copy, so their words are already MSB-first; global words are
+// swapped on load.
 template <bool kSmem>
-struct Reader {
+struct Peek {
   const uint32_t *w;
-  uint64_t buf;    // next bits, MSB first; bits below the valid ones are zero
-  uint32_t avail;  // valid bits in buf, >= 32 between steps
-  uint32_t widx;   // next word to load
-  __device__ __forceinline__ uint32_t word(uint32_t i) const { return bswap32(kSmem ? w[i] : __ldg(w + i)); }
-  __device__ __forceinline__ void seek(uint32_t p) {
-    const uint32_t i = p >> 5, s = p & 31;
-    buf = (((uint64_t)word(i) << 32) | word(i + 1)) << s;
-    avail = 64 - s;
-    widx = i + 2;
-  }
-  __device__ __forceinline__ void skip(uint32_t nb) {
-    buf <<= nb;
-    avail -= nb;
-    if (avail < 32) {
-      buf |= (uint64_t)word(widx++) << (32 - avail);
-      avail += 32;
-    }
+  __device__ __forceinline__ uint32_t word(uint32_t i) const { return kSmem ? w[i] : bswap32(__ldg(w + i)); }
+  __device__ __forceinline__ uint32_t operator()(uint32_t p) const {
+    const uint32_t i = p >> 5;
+    return __funnelshift_l(word(i + 1), word(i), p & 31);
   }
 };
 
-__device__ __forceinline__ uint32_t lut_index(uint64_t buf) { return (uint32_t)(buf >> (64 - kLutBits)); }
+__device__ __forceinline__ uint32_t lut_index(uint32_t x) { return x >> (32 - kLutBits); }
 
 // Code longer than the first-level index: second-level table, else search of
 // the canonical limits.  Returns 1 and the symbol and length, or 0 for an
 // invalid code.
-__device__ __forceinline__ uint32_t decode_long(const DecodeTables &T, uint64_t buf, uint32_t meta,
+__device__ __forceinline__ uint32_t decode_long(const DecodeTables &T, uint32_t peek, uint32_t meta,
                                                 uint32_t &syms, uint32_t &nbits) {
-  const uint32_t peek = (uint32_t)(buf >> 32);
   const uint32_t si = (meta >> 19) & 63u;
   if (si != kNoSub) {
     const uint32_t e2 = T.sub[si][(peek >> (24 - kLutBits)) & 0xFFu];
@@ -232,14 +219,14 @@ __device__ __forceinline__ uint32_t decode_long(const DecodeTables &T, uint64_t 
   return 1;
 }
 
-// One decode step on the next bits `buf`, taking only codes that start in
+// One decode step on the next 32 bits `x`, taking only codes that start in
 // the next `lim` (>= 1) bits.  Returns the number of codes taken (0: invalid
 // code); their symbols (8 bits each, first in the low byte) when kSyms, the
 // bits up to the end of the last code taken, and the code starts as a bitmap.
 template <bool kSyms>
-__device__ __forceinline__ uint32_t decode_step(const DecodeTables &T, uint64_t buf, uint32_t lim,
+__device__ __forceinline__ uint32_t decode_step(const DecodeTables &T, uint32_t x, uint32_t lim,
                                                 uint32_t &syms, uint32_t &nbits, uint32_t &bnd) {
-  const uint32_t idx = lut_index(buf);
+  const uint32_t idx = lut_index(x);
   const uint32_t meta = T.l1meta[idx];
   uint32_t k = (meta >> 4) & 7u;
   if (k) {
@@ -260,7 +247,7 @@ __device__ __forceinline__ uint32_t decode_step(const DecodeTables &T, uint64_t 
     return k;
   }
   bnd = 1u;
-  return decode_long(T, buf, meta, syms, nbits);
+  return decode_long(T, x, meta, syms, nbits);
 }
 
 // The decoding CTA holds two independent groups of kGroupThreads threads.
@@ -329,6 +316,15 @@ __device__ __forceinline__ uint2 ld_nc8(const void *p) {
   uint2 v;
   asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "l"(p));
   return v;
+}
+
+// Named barrier shared by both groups (ids 1 and 2 are the groups' own).
+constexpr uint32_t kStaggerBarrier = 3;
+__device__ __forceinline__ void named_sync(uint32_t id, uint32_t n) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+__device__ __forceinline__ void named_arrive(uint32_t id, uint32_t n) {
+  asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(n) : "memory");
 }
 
 // Barriers of one group: named barrier `id` over kGroupThreads threads.
@@ -413,10 +409,9 @@ __device__ bool decode_chunk(GroupSmem &G, const DecodeTables &T, const uint32_t
   uint32_t W = (nbits + kGroupThreads - 1) / kGroupThreads;
   W = (W + gq - 1) / gq * gq;
   const uint32_t ws = min(gtid * W, nbits), we = min(ws + W, nbits);
-  Reader<kSmem> r;
-  r.w = words;
+  Peek<kSmem> peek{words};
   // Bulk decoding runs while 2 * kLutBits bits of the window remain: two
-  // first-level lookups per refill, no window-end handling.
+  // first-level lookups per 32-bit peek, no window-end handling.
   constexpr uint32_t kBulk = 2 * kLutBits;
 
   // 2. speculative decode of the own window; record where codes start in
@@ -424,68 +419,41 @@ __device__ bool decode_chunk(GroupSmem &G, const DecodeTables &T, const uint32_t
   uint32_t pos = ws, n = 0;
   uint64_t mask = 0;
   bool bad = false;
-  if (pos < we) {
-    r.seek(rel0 + pos);
-    while (pos + kBulk <= we && pos - ws < kMaskBits) {
-      const uint32_t off = pos - ws;
-      const uint32_t m1 = T.l1meta[lut_index(r.buf)];
-      const uint32_t k1 = (m1 >> 4) & 7u, nb1 = m1 & 15u;
-      if (!k1) {
-        uint32_t syms, nb;
-        if (!decode_long(T, r.buf, m1, syms, nb)) { bad = true; break; }
-        mask |= 1ull << off;
-        r.skip(nb);
-        pos += nb;
-        n += 1;
-        continue;
-      }
-      mask |= (uint64_t)((m1 >> 7) & 0xFFFu) << off;
-      const uint32_t m2 = T.l1meta[lut_index(r.buf << nb1)];
-      const uint32_t k2 = (m2 >> 4) & 7u, nb2 = m2 & 15u;
-      if (!k2) {
-        r.skip(nb1);
-        pos += nb1;
-        n += k1;
-        continue;
-      }
-      if (off + nb1 < kMaskBits) mask |= (uint64_t)((m2 >> 7) & 0xFFFu) << (off + nb1);
-      r.skip(nb1 + nb2);
-      pos += nb1 + nb2;
-      n += k1 + k2;
-    }
-    while (!bad && pos + kBulk <= we) {
-      const uint32_t m1 = T.l1meta[lut_index(r.buf)];
-      const uint32_t k1 = (m1 >> 4) & 7u, nb1 = m1 & 15u;
-      if (!k1) {
-        uint32_t syms, nb;
-        if (!decode_long(T, r.buf, m1, syms, nb)) { bad = true; break; }
-        r.skip(nb);
-        pos += nb;
-        n += 1;
-        continue;
-      }
-      const uint32_t m2 = T.l1meta[lut_index(r.buf << nb1)];
-      const uint32_t k2 = (m2 >> 4) & 7u, nb2 = m2 & 15u;
-      if (!k2) {
-        r.skip(nb1);
-        pos += nb1;
-        n += k1;
-        continue;
-      }
-      r.skip(nb1 + nb2);
-      pos += nb1 + nb2;
-      n += k1 + k2;
-    }
-    while (!bad && pos < we) {
-      uint32_t syms, nb, bnd;
-      const uint32_t k = decode_step<false>(T, r.buf, we - pos, syms, nb, bnd);
-      if (!k) { bad = true; break; }
-      const uint32_t off = pos - ws;
-      if (off < kMaskBits) mask |= (uint64_t)bnd << off;
-      r.skip(nb);
+  while (pos + kBulk <= we) {
+    const uint32_t x = peek(rel0 + pos);
+    const uint32_t off = pos - ws;
+    const uint32_t m1 = T.l1meta[lut_index(x)];
+    const uint32_t k1 = (m1 >> 4) & 7u, nb1 = m1 & 15u;
+    if (!k1) {
+      uint32_t syms, nb;
+      if (!decode_long(T, x, m1, syms, nb)) { bad = true; break; }
+      if (off < kMaskBits) mask |= 1ull << off;
       pos += nb;
-      n += k;
+      n += 1;
+      continue;
     }
+    const uint32_t m2 = T.l1meta[lut_index(x << nb1)];
+    const uint32_t k2 = (m2 >> 4) & 7u, nb2 = m2 & 15u;
+    if (off < kMaskBits) {
+      mask |= (uint64_t)((m1 >> 7) & 0xFFFu) << off;
+      if (k2 && off + nb1 < kMaskBits) mask |= (uint64_t)((m2 >> 7) & 0xFFFu) << (off + nb1);
+    }
+    if (!k2) {
+      pos += nb1;
+      n += k1;
+      continue;
+    }
+    pos += nb1 + nb2;
+    n += k1 + k2;
+  }
+  while (!bad && pos < we) {
+    uint32_t syms, nb, bnd;
+    const uint32_t k = decode_step<false>(T, peek(rel0 + pos), we - pos, syms, nb, bnd);
+    if (!k) { bad = true; break; }
+    const uint32_t off = pos - ws;
+    if (off < kMaskBits) mask |= (uint64_t)bnd << off;
+    pos += nb;
+    n += k;
   }
   const uint32_t spec_end = bad ? we : pos, spec_n = n;
   const uint64_t spec_mask = bad ? 0ull : mask;
@@ -503,10 +471,9 @@ __device__ bool decode_chunk(GroupSmem &G, const DecodeTables &T, const uint32_t
       my_start = pred;
       uint32_t p = pred, k = 0;
       bool synced = false, bad2 = false;
-      if (p < we) r.seek(rel0 + p);
       while (p < we) {
         uint32_t syms, nb, bnd;
-        const uint32_t kk = decode_step<false>(T, r.buf, we - p, syms, nb, bnd);
+        const uint32_t kk = decode_step<false>(T, peek(rel0 + p), we - p, syms, nb, bnd);
         if (!kk) { bad2 = true; break; }
         const uint32_t off = p - ws;
         if (off < kMaskBits) {
@@ -519,7 +486,6 @@ __device__ bool decode_chunk(GroupSmem &G, const DecodeTables &T, const uint32_t
             break;
           }
         }
-        r.skip(nb);
         p += nb;
         k += kk;
       }
@@ -556,43 +522,37 @@ __device__ bool decode_chunk(GroupSmem &G, const DecodeTables &T, const uint32_t
   ExpWriter out;
   out.init(G.exps, o);
   pos = gtid == 0 ? 0u : G.ends[gtid - 1];
-  if (pos < we) {
-    r.seek(rel0 + pos);
-    while (pos + kBulk <= we) {
-      const uint32_t i1 = lut_index(r.buf);
-      const uint32_t m1 = T.l1meta[i1];
-      const uint32_t k1 = (m1 >> 4) & 7u, nb1 = m1 & 15u;
-      if (!k1) {
-        uint32_t syms, nb;
-        if (!decode_long(T, r.buf, m1, syms, nb)) break;
-        r.skip(nb);
-        pos += nb;
-        out.put(syms, 1);
-        continue;
-      }
-      const uint32_t s1 = T.l1sym[i1];
-      const uint32_t i2 = lut_index(r.buf << nb1);
-      const uint32_t m2 = T.l1meta[i2];
-      const uint32_t k2 = (m2 >> 4) & 7u, nb2 = m2 & 15u;
-      out.put(s1, k1);
-      if (!k2) {
-        r.skip(nb1);
-        pos += nb1;
-        continue;
-      }
-      const uint32_t s2 = T.l1sym[i2];
-      r.skip(nb1 + nb2);
-      pos += nb1 + nb2;
-      out.put(s2, k2);
-    }
-    while (pos < we) {
-      uint32_t syms, nb, bnd;
-      const uint32_t k = decode_step<true>(T, r.buf, we - pos, syms, nb, bnd);
-      if (!k) break;
-      r.skip(nb);
+  while (pos + kBulk <= we) {
+    const uint32_t x = peek(rel0 + pos);
+    const uint32_t i1 = lut_index(x);
+    const uint32_t m1 = T.l1meta[i1];
+    const uint32_t k1 = (m1 >> 4) & 7u, nb1 = m1 & 15u;
+    if (!k1) {
+      uint32_t syms, nb;
+      if (!decode_long(T, x, m1, syms, nb)) break;
       pos += nb;
-      out.put(syms, k);
+      out.put(syms, 1);
+      continue;
     }
+    const uint32_t s1 = T.l1sym[i1];
+    const uint32_t i2 = lut_index(x << nb1);
+    const uint32_t m2 = T.l1meta[i2];
+    const uint32_t k2 = (m2 >> 4) & 7u, nb2 = m2 & 15u;
+    out.put(s1, k1);
+    if (!k2) {
+      pos += nb1;
+      continue;
+    }
+    const uint32_t s2 = T.l1sym[i2];
+    pos += nb1 + nb2;
+    out.put(s2, k2);
+  }
+  while (pos < we) {
+    uint32_t syms, nb, bnd;
+    const uint32_t k = decode_step<true>(T, peek(rel0 + pos), we - pos, syms, nb, bnd);
+    if (!k) break;
+    pos += nb;
+    out.put(syms, k);
   }
   out.finish();
   gsync(id);
@@ -690,6 +650,11 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
       if (ci.fits && gtid == 0) issue_stage(G, b, ci);
       pending = ci.fits;
     }
+    // Stagger the groups by one decode: group 1 starts its first chunk when
+    // group 0 has decoded its own and turns to the memory-bound output, so
+    // one group's output overlaps the other's decode instead of coinciding.
+    const bool stagger = seg_end - seg >= 2;
+    if (stagger && grp == 1) named_sync(kStaggerBarrier, kDecThreads);
     for (; g < seg_end; g += kNumGroups) {
       const uint64_t i0 = (uint64_t)ci.c * b.chunk_elems;
       const uint32_t cnt = ci.cnt;
@@ -710,6 +675,9 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
         } else {
           parity ^= 1u;
           pending = false;
+          // stream words to MSB-first order, once, for the peeks
+          for (uint32_t i = gtid; i < ci.bytes / 4; i += kGroupThreads) G.stage[i] = bswap32(G.stage[i]);
+          gsync(id);
         }
       } else {
         gsync(id);  // the cleared exponent buffer is visible to the group
@@ -724,6 +692,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
         set_status(b.status, kFlagCorrupt);
       }
 
+      if (stagger && grp == 0 && g == seg) named_arrive(kStaggerBarrier, kDecThreads);
       // the stage is free: start copying the group's next chunk
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       gsync(id);
