@@ -183,6 +183,39 @@ def run_ncu_case():
     return 0
 
 
+def measure_fp4_scales(eh, synth, items, dev, stream, reps=50):
+    """Compress + decompress of the seven matrices' E4M3 block scales (byte
+    alphabet) with CUDA events; returns GB/s of scale bytes and the ratio."""
+    import torch
+    scales = [synth.nvfp4_block_scales(synth.bf16_bits_to_f32(x)) for _, x in items]
+    xs = [torch.from_numpy(s).to(dev) for s in scales]
+    p = eh.plan(eh.EH_BYTES)
+    outs = [eh.alloc_compressed(p, x.numel(), dev) for x in xs]
+    ys = [torch.empty_like(x) for x in xs]
+    wsc = torch.empty(eh.compress_batch_workspace(p, [x.numel() for x in xs]), dtype=torch.uint8, device=dev)
+    wsd = torch.empty(eh.decompress_workspace(p, len(xs)), dtype=torch.uint8, device=dev)
+    bits = torch.zeros(len(xs), dtype=torch.int64, device=dev)
+    eh.compress_batch(p, xs, outs, wsc)
+    eh.decompress_batch(p, outs, ys, wsd)
+    assert eh.get_status(wsd) == eh.EH_OK and all(torch.equal(x, y) for x, y in zip(xs, ys))
+    nbytes = sum(x.numel() for x in xs)
+    comp = sum(o.compressed_bytes() for o in outs)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+    ev[0].record(stream)
+    for _ in range(reps):
+        eh.compress_batch(p, xs, outs, wsc, bits_dev=bits)
+    ev[1].record(stream)
+    for _ in range(reps):
+        eh.decompress_batch(p, outs, ys, wsd)
+    ev[2].record(stream)
+    torch.cuda.synchronize()
+    enc = ev[0].elapsed_time(ev[1]) / reps
+    dec = ev[1].elapsed_time(ev[2]) / reps
+    return {"kind": "E4M3 block scales, one per 16 BF16 values of the block", "bytes": nbytes,
+            "encode_gbs": nbytes / (enc * 1e-3) / 1e9, "decode_gbs": nbytes / (dec * 1e-3) / 1e9,
+            "size_ratio": comp / nbytes, "bits_per_scale": 8.0 * sum(o.stream_bytes() for o in outs) / nbytes}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -305,6 +338,10 @@ def main():
         e2e_ms = t.item()
         dist.barrier()
 
+    # side measurement (outside the timed region): the codec on the block's
+    # FP4 block scale factors (NVFP4-style E4M3 scales, one per 16 values)
+    fp4 = measure_fp4_scales(eh, synth, items, dev, stream)
+
     if rank == 0:
         peak, peak_kind = hbm_peak()
         value = world * 2 * in_bytes / (ms * 1e-3) / 1e9
@@ -341,6 +378,7 @@ def main():
                     "h2d_bytes_per_step": in_bytes, "d2h_bytes_per_step": 8 + 8 * len(ns) + 4,
                     "ms_per_step": e2e_ms},
             "gpu_launches": 6 * args.steps,
+            "fp4_scales": fp4,
             "clocks": clk.summary(),
         }
         if world == 1 and not args.no_cpu_baseline:

@@ -40,7 +40,7 @@ inline bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
 inline uint64_t ceil_div(uint64_t a, uint64_t b) { return (a + b - 1) / b; }
 
 bool plan_ok(const eh_plan_t *p) {
-  return p && (p->dtype == EH_BF16 || p->dtype == EH_FP8_E4M3) && p->chunk_elems >= 1024 &&
+  return p && (p->dtype == EH_BF16 || p->dtype == EH_FP8_E4M3 || p->dtype == EH_BYTES) && p->chunk_elems >= 1024 &&
          p->chunk_elems <= (uint32_t)kMaxChunk && p->chunk_elems % 1024 == 0 && p->max_code_len >= 1 &&
          p->max_code_len <= EH_MAX_CODE_LEN;
 }
@@ -49,7 +49,10 @@ uint64_t stream_cap_for(const eh_plan_t *p, uint64_t n) {
   return ((ceil_div(n * p->max_code_len, 8) + 15) & ~uint64_t(15)) + 16;
 }
 
-uint64_t sm_bytes_for(int dtype, uint64_t n) { return dtype == EH_BF16 ? n : ceil_div(n, 2); }
+uint64_t sm_bytes_for(int dtype, uint64_t n) {
+  if (dtype == EH_BYTES) return 0;
+  return dtype == EH_BF16 ? n : ceil_div(n, 2);
+}
 
 // ---- compress workspace layout
 //   [0, 256)                 status (u32), ticket (u32), bit totals u64[k]
@@ -137,8 +140,9 @@ eh_status prepare_compress(const eh_plan_t *plan, int k, const void *const *ins,
     if (o.dtype != plan->dtype || n > (1ull << 40)) return EH_ERR_INVALID_ARG;
     if (!o.code_len || !o.code || !o.chunk_bit_off) return EH_ERR_INVALID_ARG;
     if (((uintptr_t)o.code & 3u) || ((uintptr_t)o.chunk_bit_off & 7u)) return EH_ERR_INVALID_ARG;
-    if (n > 0 && (!ins[i] || !o.exp_stream || !o.sign_mant)) return EH_ERR_INVALID_ARG;
-    if (n > 0 && (!aligned16(ins[i]) || !aligned16(o.exp_stream) || !aligned16(o.sign_mant)))
+    const bool has_sm = plan->dtype != EH_BYTES;
+    if (n > 0 && (!ins[i] || !o.exp_stream || (has_sm && !o.sign_mant))) return EH_ERR_INVALID_ARG;
+    if (n > 0 && (!aligned16(ins[i]) || !aligned16(o.exp_stream) || (has_sm && !aligned16(o.sign_mant))))
       return EH_ERR_INVALID_ARG;
     if (o.exp_stream_cap < stream_cap_for(plan, n) && n > 0) return EH_ERR_INVALID_ARG;
     ns[i] = n;
@@ -304,8 +308,10 @@ eh_status decompress_impl(const eh_plan_t *plan, int k, const eh_compressed_t *c
     if ((uint64_t)first + count > C) return EH_ERR_INVALID_ARG;
     if (!c.code_len || !c.code || !c.chunk_bit_off || ((uintptr_t)c.chunk_bit_off & 7u)) return EH_ERR_INVALID_ARG;
     if (count > 0) {
-      if (!outs[i] || !c.exp_stream || !c.sign_mant) return EH_ERR_INVALID_ARG;
-      if (!aligned16(outs[i]) || !aligned16(c.exp_stream) || !aligned16(c.sign_mant)) return EH_ERR_INVALID_ARG;
+      const bool has_sm = plan->dtype != EH_BYTES;
+      if (!outs[i] || !c.exp_stream || (has_sm && !c.sign_mant)) return EH_ERR_INVALID_ARG;
+      if (!aligned16(outs[i]) || !aligned16(c.exp_stream) || (has_sm && !aligned16(c.sign_mant)))
+        return EH_ERR_INVALID_ARG;
     }
     Item &it = b.item[i];
     it.out = outs[i];

@@ -47,7 +47,7 @@ __device__ __forceinline__ uint32_t fp8x4_sm(uint32_t x) {
 // never the same address, however skewed the exponents are.
 template <int DT>
 __global__ void __launch_bounds__(kThreads, 2) hist_kernel(const __grid_constant__ Batch b) {
-  constexpr int A = DT == EH_BF16 ? 256 : 16;
+  constexpr int A = DT == EH_FP8_E4M3 ? 16 : 256;
   __shared__ uint32_t h[A * 32];
   const uint32_t g = blockIdx.x;
   const Item &I = b.item[find_item(b, g)];
@@ -82,6 +82,22 @@ __global__ void __launch_bounds__(kThreads, 2) hist_kernel(const __grid_constant
       atomicAdd(hl + (((x >> 7) & 0xFFu) << 5), 1u);
       smo[i] = (uint8_t)bf16x2_sm(x);
     }
+  } else if (DT == EH_BYTES) {
+    // every byte is a symbol; there is no sign/mantissa to write
+    const uint8_t *in = (const uint8_t *)I.in + i0;
+    const uint32_t nvec = cnt / 32;
+    #pragma unroll 2
+    for (uint32_t v = tid; v < nvec; v += kThreads) {
+      uint4 p = ld_stream(in + 32 * (uint64_t)v);
+      uint4 q = ld_stream(in + 32 * (uint64_t)v + 16);
+      const uint32_t w[8] = {p.x, p.y, p.z, p.w, q.x, q.y, q.z, q.w};
+      #pragma unroll
+      for (int j = 0; j < 8; j++) {
+        #pragma unroll
+        for (int k = 0; k < 4; k++) atomicAdd(hl + (((w[j] >> (8 * k)) & 0xFFu) << 5), 1u);
+      }
+    }
+    for (uint32_t i = nvec * 32 + tid; i < cnt; i += kThreads) atomicAdd(hl + ((uint32_t)in[i] << 5), 1u);
   } else {
     const uint8_t *in = (const uint8_t *)I.in + i0;
     uint8_t *smo = I.sm + i0 / 2;
@@ -415,33 +431,6 @@ constexpr int kEncTile = kThreads * kEncPerThread;       // 8192 values
 constexpr int kRingWords = 16384;                        // > one tile of 32-bit codes + carry
 constexpr uint32_t kRingMask = kRingWords - 1;
 
-__device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t *wsum, uint32_t *total) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  uint32_t x = v;
-  #pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
-    if (lane >= o) x += y;
-  }
-  if (lane == 31) wsum[warp] = x;
-  __syncthreads();
-  if (warp == 0) {
-    uint32_t t = lane < kThreads / 32 ? wsum[lane] : 0u;
-    #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      uint32_t y = __shfl_up_sync(0xffffffffu, t, o);
-      if (lane >= o) t += y;
-    }
-    if (lane < kThreads / 32) wsum[lane] = t;
-  }
-  __syncthreads();
-  *total = wsum[kThreads / 32 - 1];
-  return (warp ? wsum[warp - 1] : 0u) + x - v;
-}
-
-// Loads the exponent fields of this thread's 16 values of a tile (fewer at
-// the end of the chunk; missing values get exponent 0 and are masked by the
-// caller).
 // Exclusive scan over the CTA with a single barrier: every warp publishes
 // its total, then each thread adds up the totals of the warps before its own.
 // The caller must separate two uses of `wsum` by a barrier.
@@ -507,6 +496,9 @@ __device__ __forceinline__ uint32_t exp_of(const uint4 &p, const uint4 &q, int j
   if (DT == EH_BF16) {
     const uint32_t w[8] = {p.x, p.y, p.z, p.w, q.x, q.y, q.z, q.w};
     return (w[j >> 1] >> ((j & 1) ? 23 : 7)) & 0xFFu;
+  } else if (DT == EH_BYTES) {
+    const uint32_t w[4] = {p.x, p.y, p.z, p.w};
+    return (w[j >> 2] >> (8 * (j & 3))) & 0xFFu;
   } else {
     const uint32_t w[4] = {p.x, p.y, p.z, p.w};
     return (w[j >> 2] >> (8 * (j & 3) + 3)) & 0xFu;
@@ -525,7 +517,7 @@ __device__ __forceinline__ void ring_or(uint32_t *ring, uint64_t pos, uint32_t a
 
 template <int DT>
 __global__ void __launch_bounds__(kThreads, 2) encode_kernel(const __grid_constant__ Batch b) {
-  constexpr int A = DT == EH_BF16 ? 256 : 16;
+  constexpr int A = DT == EH_FP8_E4M3 ? 16 : 256;
   extern __shared__ uint32_t ring[];  // kRingWords words, code bits in MSB-first order
   __shared__ uint2 tab[A];            // (code left-aligned in 32 bits, length)
   __shared__ uint32_t wsum[kThreads / 32];
@@ -612,6 +604,7 @@ __global__ void __launch_bounds__(kThreads, 2) encode_kernel(const __grid_consta
 cudaError_t launch_hist(const Batch &b, cudaStream_t s) {
   if (b.total_chunks == 0) return cudaSuccess;
   if (b.dtype == EH_BF16) hist_kernel<EH_BF16><<<b.total_chunks, kThreads, 0, s>>>(b);
+  else if (b.dtype == EH_BYTES) hist_kernel<EH_BYTES><<<b.total_chunks, kThreads, 0, s>>>(b);
   else hist_kernel<EH_FP8_E4M3><<<b.total_chunks, kThreads, 0, s>>>(b);
   return cudaGetLastError();
 }
@@ -632,6 +625,8 @@ cudaError_t configure_encode() {
   const int smem = kRingWords * (int)sizeof(uint32_t);
   cudaError_t e = cudaFuncSetAttribute(encode_kernel<EH_BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(encode_kernel<EH_BYTES>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
   return cudaFuncSetAttribute(encode_kernel<EH_FP8_E4M3>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
 }
 
@@ -639,6 +634,7 @@ cudaError_t launch_encode(const Batch &b, cudaStream_t s) {
   if (b.total_chunks == 0) return cudaSuccess;
   const size_t smem = kRingWords * sizeof(uint32_t);
   if (b.dtype == EH_BF16) encode_kernel<EH_BF16><<<b.total_chunks, kThreads, smem, s>>>(b);
+  else if (b.dtype == EH_BYTES) encode_kernel<EH_BYTES><<<b.total_chunks, kThreads, smem, s>>>(b);
   else encode_kernel<EH_FP8_E4M3><<<b.total_chunks, kThreads, smem, s>>>(b);
   return cudaGetLastError();
 }

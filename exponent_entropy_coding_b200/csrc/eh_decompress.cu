@@ -743,6 +743,14 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
             const uint32_t sm = smp[i], e = G.exps[exp_slot(i)];
             outp[i] = (uint16_t)(((sm & 0x80u) << 8) | (e << 7) | (sm & 0x7Fu));
           }
+        } else if (DT == EH_BYTES) {
+          // the decoded symbols are the output bytes
+          uint8_t *outp = (uint8_t *)I.out + (i0 - I.elem0);
+          for (uint32_t v = gtid; v < nvec; v += kGroupThreads) {
+            const uint32_t *ew = (const uint32_t *)(G.exps + exp_slot(16 * v));
+            *(uint4 *)(outp + 16 * (uint64_t)v) = make_uint4(ew[0], ew[1], ew[2], ew[3]);
+          }
+          for (uint32_t i = nvec * 16 + gtid; i < cnt; i += kGroupThreads) outp[i] = G.exps[exp_slot(i)];
         } else {
           const uint8_t *smp = I.sm + i0 / 2;
           uint8_t *outp = (uint8_t *)I.out + (i0 - I.elem0);
@@ -800,6 +808,7 @@ cudaError_t launch_decode(const Batch &b, cudaStream_t s, int num_sms) {
   uint32_t grid = (uint32_t)num_sms;
   if (grid > b.total_chunks) grid = b.total_chunks;
   if (b.dtype == EH_BF16) decode_kernel<EH_BF16><<<grid, kDecThreads, smem, s>>>(b);
+  else if (b.dtype == EH_BYTES) decode_kernel<EH_BYTES><<<grid, kDecThreads, smem, s>>>(b);
   else decode_kernel<EH_FP8_E4M3><<<grid, kDecThreads, smem, s>>>(b);
   return cudaGetLastError();
 }
@@ -807,6 +816,8 @@ cudaError_t launch_decode(const Batch &b, cudaStream_t s, int num_sms) {
 cudaError_t configure_decode() {
   const int smem = (int)(sizeof(DecodeSmem) + 128);
   cudaError_t e = cudaFuncSetAttribute(decode_kernel<EH_BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(decode_kernel<EH_BYTES>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   return cudaFuncSetAttribute(decode_kernel<EH_FP8_E4M3>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
 }

@@ -23,7 +23,7 @@ constexpr uint32_t kFlagCorrupt = 1u;
 constexpr uint32_t kFlagInfeasible = 2u;
 constexpr uint32_t kFlagTimeout = 4u;
 
-__host__ __device__ inline int alphabet_of(int dtype) { return dtype == EH_BF16 ? 256 : 16; }
+__host__ __device__ inline int alphabet_of(int dtype) { return dtype == EH_FP8_E4M3 ? 16 : 256; }
 
 // Per-tensor part of a launch.
 struct Item {

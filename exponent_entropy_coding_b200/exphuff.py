@@ -18,6 +18,7 @@ LIB_PATH = os.path.join(HERE, "libexphuff.so")
 
 EH_BF16 = 0
 EH_FP8_E4M3 = 1
+EH_BYTES = 2     # every byte a symbol, no sign/mantissa (FP4 block scale factors)
 EH_DEFAULT_CHUNK_ELEMS = 65536
 EH_MAX_CODE_LEN = 32
 EH_MAX_BATCH = 16
@@ -109,7 +110,7 @@ def dtype_code(torch_dtype) -> int:
 
 
 def alphabet(dtype: int) -> int:
-    return 256 if dtype == EH_BF16 else 16
+    return 16 if dtype == EH_FP8_E4M3 else 256
 
 
 def plan(dtype: int, chunk_elems: int = 0, max_code_len: int = 0) -> eh_plan_t:

@@ -21,6 +21,9 @@ available; these stand in for them):
   scale, with 4 outlier channels per head scaled by 20, seed 3.  A 64-token
   page of one tensor is 64*8*128 = 65,536 values.
 * ``lm_head``   one BF16 128256x4096 tensor, N(0, 0.02^2), seed 4.
+* ``nvfp4_scales`` / ``mxfp4_scales``  the block scale bytes of the
+  ``llama8b_block`` weights quantised to FP4: E4M3 scales per 16 values
+  (13,631,488 bytes) or E8M0 scales per 32 values (6,815,744 bytes).
 """
 import math
 
@@ -38,6 +41,7 @@ LLAMA8B_BLOCK_SHAPES = [
 ]
 
 WORKLOADS = ("bf16_1m", "fp8_16m", "llama8b_block", "kv_layer", "lm_head")
+SCALE_WORKLOADS = ("nvfp4_scales", "mxfp4_scales")
 
 
 def to_bf16_bits(a: np.ndarray) -> np.ndarray:
@@ -50,6 +54,11 @@ def to_fp8_e4m3_bits(a: np.ndarray) -> np.ndarray:
     """float32 -> FP8 E4M3 (fn variant) bit patterns (uint8), round-to-nearest-even."""
     t = torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32))
     return t.to(torch.float8_e4m3fn).view(torch.uint8).numpy().reshape(a.shape)
+
+
+def bf16_bits_to_f32(bits: np.ndarray) -> np.ndarray:
+    """BF16 bit patterns -> float32 values (exact)."""
+    return (np.ascontiguousarray(bits, dtype=np.uint16).astype(np.uint32) << 16).view(np.float32)
 
 
 def normal_bf16(n: int, seed: int, std: float = 0.02) -> np.ndarray:
@@ -67,12 +76,35 @@ def normal_fp8(n: int, seed: int, std: float = 0.02) -> np.ndarray:
     return to_fp8_e4m3_bits(w)
 
 
-def student_t_bf16(shape, rng: np.random.Generator, df: float = 5.0,
-                   std: float = 0.02) -> np.ndarray:
+def student_t_f32(shape, rng: np.random.Generator, df: float = 5.0,
+                  std: float = 0.02) -> np.ndarray:
     # a t(df) draw has variance df/(df-2); rescale to the requested std
     w = rng.standard_t(df, size=shape).astype(np.float32)
     w *= np.float32(std / math.sqrt(df / (df - 2.0)))
-    return to_bf16_bits(w)
+    return w
+
+
+def student_t_bf16(shape, rng: np.random.Generator, df: float = 5.0,
+                   std: float = 0.02) -> np.ndarray:
+    return to_bf16_bits(student_t_f32(shape, rng, df, std))
+
+
+def nvfp4_block_scales(w: np.ndarray, block: int = 16) -> np.ndarray:
+    """E4M3 scale bytes of NVFP4-style quantisation: one scale per block of
+    `block` values, amax/6 (6 = largest FP4 E2M1 value) divided by a
+    per-tensor factor that maps the largest block scale to 448."""
+    a = np.abs(w.reshape(-1, block)).max(axis=1).astype(np.float32) / np.float32(6.0)
+    g = a.max() / np.float32(448.0) if a.max() > 0 else np.float32(1.0)
+    return to_fp8_e4m3_bits(a / g)
+
+
+def mxfp4_block_scales(w: np.ndarray, block: int = 32) -> np.ndarray:
+    """E8M0 scale bytes of MXFP4-style quantisation: one power-of-two scale
+    per block of `block` values, 2^(floor(log2(amax)) - 2) (2 = largest FP4
+    E2M1 exponent), stored as the biased exponent (+127)."""
+    a = np.abs(w.reshape(-1, block)).max(axis=1).astype(np.float64)
+    e = np.floor(np.log2(np.maximum(a, 2.0 ** -126))) - 2
+    return np.clip(e + 127, 0, 254).astype(np.uint8)
 
 
 def llama8b_block(seed: int = 2, scale: int = 1, count: int = 7):
@@ -104,6 +136,18 @@ def kv_layer(seed: int = 3, batch: int = 8, tokens: int = 8192):
     return [("k", k), ("v", v)]
 
 
+def fp4_scales(kind: str = "nv", seed: int = 2, scale: int = 1):
+    """[(name, scale bytes)] of the Llama-8B block's seven matrices (the same
+    Student-t weights as `llama8b_block`) quantised block-wise to FP4:
+    kind "nv" = E4M3 scales per 16 values, "mx" = E8M0 scales per 32 values."""
+    rng = np.random.default_rng(seed)
+    out = []
+    for name, (r, c) in LLAMA8B_BLOCK_SHAPES:
+        w = student_t_f32((max(1, r // scale), c), rng).reshape(-1)
+        out.append((name, nvfp4_block_scales(w) if kind == "nv" else mxfp4_block_scales(w)))
+    return out
+
+
 def workload(name: str, scale: int = 1):
     """Returns (dtype_name, [(item_name, bits)]).  ``scale`` > 1 shrinks the
     workload (fewer rows / tokens) for quick parity runs."""
@@ -117,4 +161,8 @@ def workload(name: str, scale: int = 1):
         return "bf16", kv_layer(seed=3, tokens=max(64, 8192 // scale))
     if name == "lm_head":
         return "bf16", [("w", normal_bf16((128256 // scale) * 4096, seed=4))]
+    if name == "nvfp4_scales":
+        return "bytes", fp4_scales("nv", seed=2, scale=scale)
+    if name == "mxfp4_scales":
+        return "bytes", fp4_scales("mx", seed=2, scale=scale)
     raise KeyError(name)

@@ -35,7 +35,8 @@
  *    chunk_bit_off[C] = exp_stream_bits;
  *  - sign_mant: BF16 one byte (s<<7)|m7 per element; FP8 one nibble
  *    (s<<3)|m3 per element, element 2i in the low nibble of byte i, the unused
- *    high nibble of an odd-length tensor zero.
+ *    high nibble of an odd-length tensor zero; EH_BYTES none (the symbol is
+ *    the whole byte; sign_mant may be NULL).
  *
  * Memory: every pointer passed to a compress/decompress call is a DEVICE
  * pointer on the current CUDA device, allocated and owned by the CALLER.  The
@@ -72,7 +73,11 @@ extern "C" {
 #define EH_MAX_BATCH 16               /* tensors per batched launch         */
 #define EH_NOALLOC_MAX_BATCH 8        /* tensors per eh_decompress_batch_noalloc */
 
-typedef enum { EH_BF16 = 0, EH_FP8_E4M3 = 1 } eh_dtype;
+/* EH_BYTES: every byte is its own symbol (alphabet 256) and there is no
+ * sign/mantissa array -- for FP4 block scale factors (E4M3 or E8M0 bytes),
+ * which the paper summary ("结果分析") and the edgentiq blog ("Insights into
+ * FP4 Compression") report compressible with Huffman coding. */
+typedef enum { EH_BF16 = 0, EH_FP8_E4M3 = 1, EH_BYTES = 2 } eh_dtype;
 
 typedef enum {
   EH_OK = 0,
@@ -104,7 +109,7 @@ typedef struct {
   uint64_t *chunk_bit_off;  /* device, [n_chunks + 1]                        */
   uint8_t *exp_stream;      /* device, exp_stream_cap bytes                  */
   uint64_t exp_stream_cap;  /* bytes; >= eh_compress_bound's stream_cap      */
-  uint8_t *sign_mant;       /* device, n (BF16) or ceil(n/2) (FP8) bytes     */
+  uint8_t *sign_mant;       /* device, n (BF16), ceil(n/2) (FP8), 0 (BYTES)  */
   uint64_t exp_stream_bits; /* total code bits (host copy)                   */
 } eh_compressed_t;
 

@@ -33,7 +33,9 @@
  *     back to back with no padding, off[c] = first bit of chunk c, the last
  *     byte zero-padded;
  *   - sign+mantissa: BF16 byte (s<<7)|m7; FP8 nibble (s<<3)|m3, element 2i in
- *     the low nibble of byte i, unused high nibble zero.
+ *     the low nibble of byte i, unused high nibble zero;
+ *   - BYTES (FP4 block scale factors): the whole byte is the symbol, there is
+ *     no sign+mantissa array.
  */
 #include "ehref.h"
 
@@ -44,7 +46,7 @@
 namespace {
 
 int alphabet_of(int dtype) {
-  if (dtype == EHREF_BF16) return 256;
+  if (dtype == EHREF_BF16 || dtype == EHREF_BYTES) return 256;
   if (dtype == EHREF_FP8_E4M3) return 16;
   return 0;
 }
@@ -61,9 +63,13 @@ void store_elem(int dtype, void *out, uint64_t i, uint32_t x) {
     ((uint8_t *)out)[i] = (uint8_t)x;
 }
 
-/* S1 for one element.  BF16 = s | e8 | m7 ; E4M3 = s | e4 | m3. */
+/* S1 for one element.  BF16 = s | e8 | m7 ; E4M3 = s | e4 | m3 ; BYTES: the
+ * byte is the symbol. */
 void split_one(int dtype, uint32_t x, uint8_t *e, uint8_t *sm) {
-  if (dtype == EHREF_BF16) {
+  if (dtype == EHREF_BYTES) {
+    *e = (uint8_t)x;
+    *sm = 0;
+  } else if (dtype == EHREF_BF16) {
     uint32_t s = (x >> 15) & 1u, ex = (x >> 7) & 0xFFu, m = x & 0x7Fu;
     *e = (uint8_t)ex;
     *sm = (uint8_t)((s << 7) | m);
@@ -75,6 +81,7 @@ void split_one(int dtype, uint32_t x, uint8_t *e, uint8_t *sm) {
 }
 
 uint32_t merge_one(int dtype, uint32_t e, uint32_t sm) {
+  if (dtype == EHREF_BYTES) return e;
   if (dtype == EHREF_BF16) {
     uint32_t s = (sm >> 7) & 1u, m = sm & 0x7Fu;
     return (s << 15) | (e << 7) | m;
@@ -314,6 +321,7 @@ int ehref_canonical_codes(const uint8_t *len, int A, uint32_t *code) {
 }
 
 uint64_t ehref_sm_bytes(int dtype, uint64_t n) {
+  if (dtype == EHREF_BYTES) return 0;
   return dtype == EHREF_BF16 ? n : (n + 1) / 2;
 }
 
@@ -326,7 +334,7 @@ int ehref_pack_sm(int dtype, const void *in, uint64_t n, uint8_t *out) {
     split_one(dtype, load_elem(dtype, in, i), &e, &sm);
     if (dtype == EHREF_BF16)
       out[i] = sm;
-    else
+    else if (dtype == EHREF_FP8_E4M3)
       out[i / 2] |= (uint8_t)(sm << (4 * (i & 1)));
   }
   return EHREF_OK;
@@ -418,10 +426,10 @@ int ehref_decompress_chunks(int dtype, uint64_t n, uint32_t chunk,
         }
       }
       if (sym < 0) return EHREF_ECORRUPT;
-      uint32_t sm;
+      uint32_t sm = 0;
       if (dtype == EHREF_BF16)
         sm = sm_packed[i];
-      else
+      else if (dtype == EHREF_FP8_E4M3)
         sm = (sm_packed[i / 2] >> (4 * (i & 1))) & 0xFu;
       store_elem(dtype, out, i - (uint64_t)first * chunk, merge_one(dtype, (uint32_t)sym, sm));
     }

@@ -34,7 +34,11 @@
 extern "C" {
 #endif
 
-enum { EHREF_BF16 = 0, EHREF_FP8_E4M3 = 1 };
+/* EHREF_BYTES: every byte is its own symbol and there is no sign/mantissa
+ * part -- the codec applied to FP4 block scale factors (E4M3 or E8M0 bytes),
+ * which the paper summary ("结果分析") and the edgentiq blog ("Insights into
+ * FP4 Compression") report compressible with Huffman coding. */
+enum { EHREF_BF16 = 0, EHREF_FP8_E4M3 = 1, EHREF_BYTES = 2 };
 
 enum {
   EHREF_OK = 0,
@@ -44,7 +48,8 @@ enum {
   EHREF_ECORRUPT = -4     /* compressed data inconsistent                   */
 };
 
-/* 256 for BF16 (8-bit exponent field), 16 for FP8 E4M3 (4-bit field). */
+/* 256 for BF16 (8-bit exponent field) and BYTES, 16 for FP8 E4M3 (4-bit
+ * field). */
 int ehref_alphabet(int dtype);
 
 /* Step S1.  Per element: exponent field e[i] and the raw sign+mantissa
@@ -74,7 +79,7 @@ int ehref_code_lengths(const uint64_t *cnt, int A, int Lmax, uint8_t *len);
 int ehref_canonical_codes(const uint8_t *len, int A, uint32_t *code);
 
 /* Sign/mantissa array in its stored layout: BF16 one byte per element; FP8
- * one nibble per element, element 2i in the low nibble of byte i. */
+ * one nibble per element, element 2i in the low nibble of byte i; BYTES none. */
 uint64_t ehref_sm_bytes(int dtype, uint64_t n);
 int ehref_pack_sm(int dtype, const void *in, uint64_t n, uint8_t *sm_packed);
 

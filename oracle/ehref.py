@@ -13,6 +13,7 @@ from . import build as _build
 
 BF16 = 0
 FP8_E4M3 = 1
+BYTES = 2
 
 OK, EINVAL, EINFEASIBLE, ECAPACITY, ECORRUPT = 0, -1, -2, -3, -4
 _NAMES = {EINVAL: "EINVAL", EINFEASIBLE: "EINFEASIBLE", ECAPACITY: "ECAPACITY",

@@ -44,7 +44,7 @@ def _same(c, ref):
 
 def _run(eh, oracle, name, page_ranges=False):
     dt, items = synth.workload(name)
-    dtype = 0 if dt == "bf16" else 1
+    dtype = {"bf16": 0, "fp8_e4m3": 1, "bytes": 2}[dt]
     p = eh.plan(dtype)
     xs = [_dev(x) for _, x in items]
     outs = [eh.alloc_compressed(p, x.numel(), "cuda") for x in xs]
@@ -93,3 +93,9 @@ def test_kv_layer(eh, oracle):
 def test_lm_head(eh, oracle):
     (c,) = _run(eh, oracle, "lm_head")
     assert c.n_chunks == 8016
+
+
+@pytest.mark.parametrize("name", list(synth.SCALE_WORKLOADS))
+def test_fp4_block_scales(eh, oracle, name):
+    outs = _run(eh, oracle, name)
+    assert len(outs) == 7

@@ -280,3 +280,18 @@ def test_sharded_compress_on_one_gpu(eh, oracle):
         assert np.array_equal(o.code_len.cpu().numpy(), ref.code_len)
     for o, xr in zip(outs, xs):
         assert torch.equal(eh.decompress(o, p), xr)
+
+
+@pytest.mark.parametrize("n,chunk", [(1, 65536), (3 * 65536 + 17, 65536), (10 * 1024 + 5, 1024)])
+def test_bytes_alphabet(eh, oracle, n, chunk):
+    # FP4 block scale bytes: every byte is a symbol, no sign/mantissa array
+    _, items = synth.workload("nvfp4_scales", scale=16)
+    x = np.concatenate([v for _, v in items])[:n]
+    c = roundtrip(eh, oracle, 2, x, chunk=chunk)
+    assert c.sign_mant.numel() == 0
+
+
+def test_bytes_every_value(eh, oracle):
+    rng = np.random.default_rng(8)
+    x = np.tile(np.arange(256, dtype=np.uint8), 1000)[rng.permutation(256 * 1000)]
+    roundtrip(eh, oracle, 2, x)

@@ -395,3 +395,60 @@ def test_decoder_rejects_corruption(oracle):
     cd = c.code.copy()
     cd[np.nonzero(c.code_len)[0][0]] ^= 1        # not the canonical code
     bad(code=cd)
+
+
+# ------------------------------------------------------- byte alphabet (FP4 scales)
+
+def test_bytes_handworked(oracle):
+    g = dict(r.split(":", 1) for r in read_golden("bytes_handworked.txt"))
+    x = np.array([int(h, 16) for h in g["input_hex"].split()], np.uint8)
+    c = oracle.compress(oracle.BYTES, x)
+    for item in g["lengths"].split():
+        s, l = item.split(":")
+        assert c.code_len[int(s)] == int(l)
+    for item in g["codes"].split():
+        s, bits = item.split(":")
+        assert format(int(c.code[int(s)]), f"0{len(bits)}b") == bits
+    assert c.bits == int(g["bits"])
+    assert bytes(c.stream) == bytes(int(h, 16) for h in g["stream_hex"].split())
+    assert c.sign_mant.size == 0
+    assert np.array_equal(oracle.decompress(c), x)
+
+
+def test_bytes_every_value_roundtrip(oracle):
+    rng = np.random.default_rng(3)
+    x = np.tile(np.arange(256, dtype=np.uint8), 300)[rng.permutation(256 * 300)]
+    e, sm = oracle.split(oracle.BYTES, x)
+    assert np.array_equal(e, x) and not sm.any()
+    for chunk in (1024, 65536):
+        c = oracle.compress(oracle.BYTES, x, chunk=chunk)
+        assert np.array_equal(oracle.decompress(c), x)
+
+
+@pytest.mark.parametrize("name", list(synth.SCALE_WORKLOADS))
+def test_entropy_bound_fp4_scales(oracle, name):
+    _, items = synth.workload(name, scale=64)
+    x = np.concatenate([v for _, v in items])
+    cnt = oracle.histogram(oracle.BYTES, x)
+    assert np.array_equal(cnt, np.bincount(x, minlength=256).astype(np.uint64))
+    lens = oracle.code_lengths(cnt, 32)
+    H = entropy_bits(cnt)
+    Lbar = float(np.dot(cnt.astype(np.float64), lens)) / cnt.sum()
+    assert H <= Lbar < H + 1
+    # the scales are compressible (well below 8 bits per byte)
+    assert Lbar < 6.0
+
+
+def test_fp4_scale_generators():
+    # E8M0: 2^(floor(log2 amax) - 2) stored as exponent + 127
+    w = np.zeros(64, np.float32)
+    w[5] = 3.0        # block 0: amax 3 -> floor(log2 3) = 1 -> 1 - 2 + 127
+    w[40] = -0.25     # block 1: amax 0.25 -> -2 -> -4 + 127
+    assert list(synth.mxfp4_block_scales(w)) == [126, 123]
+    # E4M3 (NVFP4): amax/6 rescaled so the largest block scale is 448
+    w = np.zeros(32, np.float32)
+    w[0] = 6.0
+    w[20] = 1.5
+    s = synth.nvfp4_block_scales(w)
+    vals = torch.from_numpy(s.copy()).view(torch.float8_e4m3fn).float().tolist()
+    assert vals == [448.0, 112.0]
