@@ -216,6 +216,51 @@ def measure_fp4_scales(eh, synth, items, dev, stream, reps=50):
             "size_ratio": comp / nbytes, "bits_per_scale": 8.0 * sum(o.stream_bytes() for o in outs) / nbytes}
 
 
+def measure_kv_pages(eh, synth, dev, stream, reps=20):
+    """Online K/V page store: a K cache of [2, 8192, 8, 128] (256 pages of 64
+    tokens); the codebook is frozen from the first 64 pages' exponent counts
+    plus one per symbol; the other 192 pages are appended into 28 KB slots in
+    one call and read back in one call (CUDA events, BF16 bytes per second)."""
+    import torch
+    rng = np.random.default_rng(3)
+    k = synth.kv_tensor(rng, 2, 8192)
+    page = 65536
+    p = eh.plan(eh.EH_BF16)
+    prefill = torch.from_numpy(k[: 64 * page].view(np.int16)).to(dev)
+    new = torch.from_numpy(k[64 * page:].view(np.int16)).to(dev)
+    n_new = new.numel() // page
+    scratch = eh.alloc_compressed(p, prefill.numel(), dev)
+    ws = torch.empty(eh.compress_bound(p, prefill.numel())[2], dtype=torch.uint8, device=dev)
+    counts = torch.zeros(256, dtype=torch.int64, device=dev)
+    eh.compress_shard_begin(prefill, scratch, counts, p, ws)
+    code_len, code = eh.codebook_from_counts(p, counts + 1)
+    store = eh.PageStore(p, code_len, code, n_slots=n_new, slot_bytes=28 * 1024, raw_cap=n_new, device=dev)
+    ids = torch.arange(n_new, dtype=torch.int32, device=dev)
+    store.append(new, ids)
+    assert store.status() == eh.EH_OK
+    y = store.read(ids)
+    assert torch.equal(y, new)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+    ev[0].record(stream)
+    for _ in range(reps):
+        store.raw_used.zero_()
+        store.append(new, ids)
+    ev[1].record(stream)
+    for _ in range(reps):
+        store.read(ids, out=y, check=False)
+    ev[2].record(stream)
+    torch.cuda.synchronize()
+    nbytes = 2 * new.numel()
+    meta = store.page_meta.cpu().numpy().view(np.uint32)
+    coded = meta[(meta & 0x80000000) == 0]
+    return {"kind": "K cache [2, 8192, 8, 128] BF16, 192 pages appended after a 64-page prefill",
+            "append_gbs": nbytes / (ev[0].elapsed_time(ev[1]) / reps * 1e-3) / 1e9,
+            "read_gbs": nbytes / (ev[1].elapsed_time(ev[2]) / reps * 1e-3) / 1e9,
+            "raw_pages": int((meta & 0x80000000).astype(bool).sum()),
+            "bits_per_exponent": float(coded.mean()) / page if coded.size else None,
+            "slot_bytes": 28 * 1024}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -341,6 +386,7 @@ def main():
     # side measurement (outside the timed region): the codec on the block's
     # FP4 block scale factors (NVFP4-style E4M3 scales, one per 16 values)
     fp4 = measure_fp4_scales(eh, synth, items, dev, stream)
+    kv_pages = measure_kv_pages(eh, synth, dev, stream)
 
     if rank == 0:
         peak, peak_kind = hbm_peak()
@@ -379,6 +425,7 @@ def main():
                     "ms_per_step": e2e_ms},
             "gpu_launches": 6 * args.steps,
             "fp4_scales": fp4,
+            "kv_pages": kv_pages,
             "clocks": clk.summary(),
         }
         if world == 1 and not args.no_cpu_baseline:

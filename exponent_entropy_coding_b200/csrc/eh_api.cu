@@ -361,6 +361,120 @@ eh_status eh_decompress_chunks(const eh_plan_t *plan, const eh_compressed_t *c, 
   return decompress_impl(plan, 1, c, outs, &first, &count, workspace, workspace_bytes, stream);
 }
 
+eh_status eh_codebook_from_counts(const eh_plan_t *plan, const uint64_t *counts, uint8_t *code_len, uint32_t *code,
+                                  void *workspace, uint64_t workspace_bytes, void *stream) {
+  if (!plan_ok(plan) || !counts || !code_len || !code || !workspace) return EH_ERR_INVALID_ARG;
+  if (((uintptr_t)workspace & 255u) || ((uintptr_t)counts & 7u) || ((uintptr_t)code & 3u)) return EH_ERR_INVALID_ARG;
+  const uint64_t zero = 0;
+  if (workspace_bytes < compress_ws_bytes(plan, 1, &zero)) return EH_ERR_NOMEM;
+  int num_sms = 0;
+  if (device_setup(&num_sms) != cudaSuccess) return EH_ERR_CUDA;
+  uint8_t *ws = (uint8_t *)workspace;
+  Batch b;
+  std::memset(&b, 0, sizeof(b));
+  b.k = 1;
+  b.chunk_elems = plan->chunk_elems;
+  b.dtype = plan->dtype;
+  b.max_code_len = plan->max_code_len;
+  b.status = (uint32_t *)ws;
+  b.ticket = (uint32_t *)(ws + 4);
+  Item &it = b.item[0];
+  it.counts = const_cast<uint64_t *>(counts);
+  it.code_len = code_len;
+  it.code = code;
+  it.pm_scratch = (uint64_t *)(ws + align256(kHeader + kCountsBytes));
+  cudaStream_t s = (cudaStream_t)stream;
+  if (cudaMemsetAsync(ws, 0, kHeader, s) != cudaSuccess) return EH_ERR_CUDA;
+  if (launch_book(b, s) != cudaSuccess) return EH_ERR_CUDA;
+  return EH_OK;
+}
+
+eh_status eh_pages_append(const eh_plan_t *plan, const eh_page_store_t *store, const void *in, uint32_t n_pages,
+                          const uint32_t *slot_ids, void *workspace, uint64_t workspace_bytes, void *stream) {
+  if (!plan_ok(plan) || !store || !workspace || workspace_bytes < kHeader) return EH_ERR_INVALID_ARG;
+  if (n_pages == 0) return EH_OK;
+  const bool has_sm = plan->dtype != EH_BYTES;
+  if (!in || !slot_ids || !store->code_len || !store->code || !store->slots || !store->page_meta ||
+      !store->raw_used || (has_sm && !store->sign_mant) || (store->raw_cap && !store->raw_pool))
+    return EH_ERR_INVALID_ARG;
+  if (!aligned16(in) || !aligned16(store->slots) || (has_sm && !aligned16(store->sign_mant)) ||
+      (store->raw_pool && !aligned16(store->raw_pool)) || store->slot_bytes % 16 || store->slot_bytes == 0 ||
+      ((uintptr_t)workspace & 255u))
+    return EH_ERR_INVALID_ARG;
+  int num_sms = 0;
+  if (device_setup(&num_sms) != cudaSuccess) return EH_ERR_CUDA;
+  PageLaunch pl;
+  std::memset(&pl, 0, sizeof(pl));
+  pl.in = in;
+  pl.slot_ids = slot_ids;
+  pl.n_pages = n_pages;
+  pl.page_elems = plan->chunk_elems;
+  pl.code_len = store->code_len;
+  pl.code = store->code;
+  pl.slots = store->slots;
+  pl.slot_bytes = store->slot_bytes;
+  pl.n_slots = store->n_slots;
+  pl.raw_cap = store->raw_cap;
+  pl.sm = store->sign_mant;
+  pl.page_meta = store->page_meta;
+  pl.raw_pool = store->raw_pool;
+  pl.raw_used = store->raw_used;
+  pl.status = (uint32_t *)workspace;
+  pl.dtype = plan->dtype;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (cudaMemsetAsync(workspace, 0, 4, s) != cudaSuccess) return EH_ERR_CUDA;
+  if (launch_page_append(pl, s) != cudaSuccess) return EH_ERR_CUDA;
+  return EH_OK;
+}
+
+eh_status eh_pages_read(const eh_plan_t *plan, const eh_page_store_t *store, const uint32_t *slot_ids,
+                        uint32_t n_pages, void *out, void *workspace, uint64_t workspace_bytes, void *stream) {
+  if (!plan_ok(plan) || !store || !workspace) return EH_ERR_INVALID_ARG;
+  if (((uintptr_t)workspace & 255u) != 0) return EH_ERR_INVALID_ARG;
+  if (workspace_bytes < kHeader + kLutBytes) return EH_ERR_NOMEM;
+  if (n_pages == 0) return EH_OK;
+  const bool has_sm = plan->dtype != EH_BYTES;
+  if (!out || !slot_ids || !store->code_len || !store->code || !store->slots || !store->page_meta ||
+      (has_sm && !store->sign_mant) || !aligned16(out) || !aligned16(store->slots) ||
+      (has_sm && !aligned16(store->sign_mant)) || (store->raw_pool && !aligned16(store->raw_pool)) ||
+      store->slot_bytes % 16 || store->slot_bytes == 0)
+    return EH_ERR_INVALID_ARG;
+  uint8_t *ws = (uint8_t *)workspace;
+  Batch b;
+  std::memset(&b, 0, sizeof(b));
+  b.k = 1;
+  b.chunk_elems = plan->chunk_elems;
+  b.dtype = plan->dtype;
+  b.max_code_len = plan->max_code_len;
+  b.status = (uint32_t *)ws;
+  b.ticket = (uint32_t *)(ws + 4);
+  b.total_chunks = n_pages;
+  Item &it = b.item[0];
+  it.out = out;
+  it.n = (uint64_t)n_pages * plan->chunk_elems;
+  it.chunk0 = 0;
+  it.nchunks = n_pages;
+  it.total_chunks = n_pages;
+  it.code_len = const_cast<uint8_t *>(store->code_len);
+  it.code = const_cast<uint32_t *>(store->code);
+  it.stream = store->slots;
+  it.stream_cap = (uint64_t)store->n_slots * store->slot_bytes;
+  it.sm = store->sign_mant;
+  it.lut = ws + kHeader;
+  it.slot_ids = slot_ids;
+  it.page_meta = store->page_meta;
+  it.raw_pool = store->raw_pool;
+  it.slot_bytes = store->slot_bytes;
+  it.n_slots = store->n_slots;
+  it.raw_cap = store->raw_cap;
+  int num_sms = 0;
+  if (device_setup(&num_sms) != cudaSuccess) return EH_ERR_CUDA;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (launch_tables(b, s) != cudaSuccess) return EH_ERR_CUDA;
+  if (launch_decode(b, s, num_sms) != cudaSuccess) return EH_ERR_CUDA;
+  return EH_OK;
+}
+
 eh_status eh_get_status(void *workspace, void *stream) {
   if (!workspace) return EH_ERR_INVALID_ARG;
   uint32_t st = 0;
@@ -369,6 +483,7 @@ eh_status eh_get_status(void *workspace, void *stream) {
   if (cudaStreamSynchronize(s) != cudaSuccess) return EH_ERR_CUDA;
   if (st & kFlagInfeasible) return EH_ERR_INFEASIBLE;
   if (st & kFlagTimeout) return EH_ERR_TIMEOUT;
+  if (st & kFlagNoRoom) return EH_ERR_NOMEM;
   if (st & kFlagCorrupt) return EH_ERR_CORRUPT;
   return EH_OK;
 }

@@ -515,28 +515,14 @@ __device__ __forceinline__ void ring_or(uint32_t *ring, uint64_t pos, uint32_t a
   if (s + nbits > 32) atomicOr(&ring[(w + 1) & kRingMask], (uint32_t)y);
 }
 
+// Packs the codes of values [0, cnt) of `in` into stream bits [bit0, bit1)
+// of gs.  The ring must be zero on entry and is zero on return.  Words that
+// the range shares with its neighbours are OR-ed into (pre-cleared) stream
+// words unless `exclusive`, when the range owns every word it touches.
 template <int DT>
-__global__ void __launch_bounds__(kThreads, 2) encode_kernel(const __grid_constant__ Batch b) {
-  constexpr int A = DT == EH_FP8_E4M3 ? 16 : 256;
-  extern __shared__ uint32_t ring[];  // kRingWords words, code bits in MSB-first order
-  __shared__ uint2 tab[A];            // (code left-aligned in 32 bits, length)
-  __shared__ uint32_t wsum[kThreads / 32];
-  const uint32_t g = blockIdx.x;
-  const Item &I = b.item[find_item(b, g)];
-  const uint32_t c = g - I.chunk0;
-  const uint64_t i0 = (uint64_t)c * b.chunk_elems;
-  const uint32_t cnt = (uint32_t)min((uint64_t)b.chunk_elems, I.n - i0);
+__device__ void encode_range(const uint2 *tab, const uint8_t *in, uint32_t cnt, uint64_t bit0, uint64_t bit1,
+                             uint32_t *gs, uint32_t *ring, uint32_t *wsum, bool exclusive) {
   const int tid = threadIdx.x;
-  for (int s2 = tid; s2 < A; s2 += kThreads) {
-    const uint32_t l = I.code_len[s2];
-    tab[s2] = make_uint2(l ? I.code[s2] << (32 - l) : 0u, l);
-  }
-  for (int i = tid; i < kRingWords; i += kThreads) ring[i] = 0u;
-  const uint64_t bit0 = I.off[c], bit1 = I.off[c + 1];
-  uint32_t *gs = (uint32_t *)I.stream;
-  const uint8_t *in = (const uint8_t *)I.in + i0 * (DT == EH_BF16 ? 2 : 1);
-  __syncthreads();
-
   uint64_t tile_base = bit0;           // stream bit where the current tile starts
   uint64_t wdone = bit0 >> 5;          // first stream word not yet written out
   uint4 np, nq;
@@ -591,11 +577,122 @@ __global__ void __launch_bounds__(kThreads, 2) encode_kernel(const __grid_consta
       const uint32_t slot = (uint32_t)(wi & kRingMask);
       const uint32_t val = bswap32(ring[slot]);
       ring[slot] = 0u;
-      const bool edge = (wi << 5) < bit0 || ((wi + 1) << 5) > bit1;
+      const bool edge = !exclusive && ((wi << 5) < bit0 || ((wi + 1) << 5) > bit1);
       if (edge) atomicOr(gs + wi, val);
       else gs[wi] = val;
     }
     wdone = wend;
+  }
+}
+
+template <int DT>
+__device__ __forceinline__ void load_code_table(uint2 *tab, const uint8_t *code_len, const uint32_t *code) {
+  constexpr int A = DT == EH_FP8_E4M3 ? 16 : 256;
+  for (int s2 = threadIdx.x; s2 < A; s2 += kThreads) {
+    const uint32_t l = code_len[s2];
+    tab[s2] = make_uint2(l ? code[s2] << (32 - l) : 0u, l);
+  }
+}
+
+template <int DT>
+__global__ void __launch_bounds__(kThreads, 2) encode_kernel(const __grid_constant__ Batch b) {
+  constexpr int A = DT == EH_FP8_E4M3 ? 16 : 256;
+  extern __shared__ uint32_t ring[];  // kRingWords words, code bits in MSB-first order
+  __shared__ uint2 tab[A];            // (code left-aligned in 32 bits, length)
+  __shared__ uint32_t wsum[kThreads / 32];
+  const uint32_t g = blockIdx.x;
+  const Item &I = b.item[find_item(b, g)];
+  const uint32_t c = g - I.chunk0;
+  const uint64_t i0 = (uint64_t)c * b.chunk_elems;
+  const uint32_t cnt = (uint32_t)min((uint64_t)b.chunk_elems, I.n - i0);
+  load_code_table<DT>(tab, I.code_len, I.code);
+  for (int i = threadIdx.x; i < kRingWords; i += kThreads) ring[i] = 0u;
+  const uint8_t *in = (const uint8_t *)I.in + i0 * (DT == EH_BF16 ? 2 : 1);
+  __syncthreads();
+  encode_range<DT>(tab, in, cnt, I.off[c], I.off[c + 1], (uint32_t *)I.stream, ring, wsum, false);
+}
+
+// ---------------------------------------------------------------- pages
+// One CTA per appended K/V page: code bits of the page with the frozen
+// codebook (and its sign/mantissa array), then either the codes into the
+// page's own slot (every word of the slot belongs to the page) or, when they
+// do not fit or an exponent has no code, the exponent bytes into the next
+// free page of the raw pool.
+template <int DT>
+__global__ void __launch_bounds__(kThreads, 2) page_append_kernel(const __grid_constant__ PageLaunch pl) {
+  constexpr int A = DT == EH_FP8_E4M3 ? 16 : 256;
+  extern __shared__ uint32_t ring[];
+  __shared__ uint2 tab[A];
+  __shared__ uint32_t wsum[kThreads / 32];
+  __shared__ uint32_t raw_idx;
+  const int tid = threadIdx.x;
+  const uint32_t pg = blockIdx.x;
+  const uint32_t slot = pl.slot_ids[pg];
+  if (slot >= pl.n_slots) {
+    if (tid == 0) set_status(pl.status, kFlagCorrupt);
+    return;
+  }
+  const uint32_t n = pl.page_elems;
+  const uint8_t *in = (const uint8_t *)pl.in + (uint64_t)pg * n * (DT == EH_BF16 ? 2 : 1);
+  const uint64_t sm_page = DT == EH_BF16 ? n : (DT == EH_FP8_E4M3 ? n / 2 : 0);
+  uint8_t *smo = pl.sm + (uint64_t)slot * sm_page;
+  load_code_table<DT>(tab, pl.code_len, pl.code);
+  for (int i = tid; i < kRingWords; i += kThreads) ring[i] = 0u;
+  __syncthreads();
+
+  // pass 1: code bits, missing codes, sign/mantissa
+  uint32_t bits = 0, missing = 0;
+  for (uint32_t idx = tid * kEncPerThread; idx < n; idx += kEncTile) {
+    uint4 p, q;
+    load_exps<DT>(in, idx, n, p, q);
+    #pragma unroll
+    for (int j = 0; j < kEncPerThread; j++) {
+      const uint32_t l = tab[exp_of<DT>(p, q, j)].y;
+      bits += l;
+      missing |= l == 0;
+    }
+    if (DT == EH_BF16) {
+      const uint32_t w[8] = {p.x, p.y, p.z, p.w, q.x, q.y, q.z, q.w};
+      uint32_t o[4];
+      #pragma unroll
+      for (int j = 0; j < 4; j++) o[j] = bf16x2_sm(w[2 * j]) | (bf16x2_sm(w[2 * j + 1]) << 16);
+      *(uint4 *)(smo + idx) = make_uint4(o[0], o[1], o[2], o[3]);
+    } else if (DT == EH_FP8_E4M3) {
+      const uint32_t w[4] = {p.x, p.y, p.z, p.w};
+      const uint32_t lo = fp8x4_sm(w[0]) | (fp8x4_sm(w[1]) << 16);
+      const uint32_t hi = fp8x4_sm(w[2]) | (fp8x4_sm(w[3]) << 16);
+      *(uint2 *)(smo + idx / 2) = make_uint2(lo, hi);
+    }
+  }
+  uint32_t total;
+  (void)block_excl_scan1(bits, wsum, &total);
+  const bool any_missing = __syncthreads_or(missing != 0);
+  const bool coded = !any_missing && (total + 7) / 8 + 16 <= pl.slot_bytes;
+  if (coded) {
+    const uint64_t b0 = (uint64_t)slot * pl.slot_bytes * 8;
+    encode_range<DT>(tab, in, n, b0, b0 + total, (uint32_t *)pl.slots, ring, wsum, true);
+    if (tid == 0) pl.page_meta[slot] = total;
+    return;
+  }
+  if (tid == 0) {
+    raw_idx = atomicAdd(pl.raw_used, 1u);
+    if (raw_idx >= pl.raw_cap) set_status(pl.status, kFlagNoRoom);
+    pl.page_meta[slot] = EH_PAGE_RAW | (raw_idx < pl.raw_cap ? raw_idx : 0x7FFFFFFFu);
+  }
+  __syncthreads();
+  if (raw_idx >= pl.raw_cap) return;
+  uint8_t *dst = pl.raw_pool + (uint64_t)raw_idx * n;
+  for (uint32_t idx = tid * kEncPerThread; idx < n; idx += kEncTile) {
+    uint4 p, q;
+    load_exps<DT>(in, idx, n, p, q);
+    uint32_t o[4];
+    #pragma unroll
+    for (int w = 0; w < 4; w++) {
+      o[w] = 0;
+      #pragma unroll
+      for (int k = 0; k < 4; k++) o[w] |= exp_of<DT>(p, q, 4 * w + k) << (8 * k);
+    }
+    *(uint4 *)(dst + idx) = make_uint4(o[0], o[1], o[2], o[3]);
   }
 }
 
@@ -627,7 +724,22 @@ cudaError_t configure_encode() {
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(encode_kernel<EH_BYTES>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  return cudaFuncSetAttribute(encode_kernel<EH_FP8_E4M3>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  e = cudaFuncSetAttribute(encode_kernel<EH_FP8_E4M3>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(page_append_kernel<EH_BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(page_append_kernel<EH_BYTES>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  return cudaFuncSetAttribute(page_append_kernel<EH_FP8_E4M3>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+}
+
+cudaError_t launch_page_append(const PageLaunch &pl, cudaStream_t s) {
+  if (pl.n_pages == 0) return cudaSuccess;
+  const size_t smem = kRingWords * sizeof(uint32_t);
+  if (pl.dtype == EH_BF16) page_append_kernel<EH_BF16><<<pl.n_pages, kThreads, smem, s>>>(pl);
+  else if (pl.dtype == EH_BYTES) page_append_kernel<EH_BYTES><<<pl.n_pages, kThreads, smem, s>>>(pl);
+  else page_append_kernel<EH_FP8_E4M3><<<pl.n_pages, kThreads, smem, s>>>(pl);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_encode(const Batch &b, cudaStream_t s) {

@@ -573,27 +573,63 @@ __device__ __forceinline__ uint32_t fp8_merge4(uint32_t nib16, uint32_t e4) {
 // Where one chunk's bits are and whether they fit a shared-memory stage.
 struct ChunkInfo {
   int item;
-  uint32_t c;       // tensor-local chunk index
+  uint32_t c;       // tensor-local chunk index (page index of the call in page mode)
   uint32_t cnt;     // values in the chunk
   uint32_t nbits;   // code bits of the chunk
   uint32_t rel0;    // first bit of the chunk relative to byte `lo`
   uint32_t bytes;   // stream bytes staged (multiple of 16)
   uint64_t lo;      // first staged stream byte (multiple of 16)
+  uint64_t sm_off;  // byte offset of the chunk's sign/mantissa array
+  uint64_t out_off; // index in `out` of the chunk's first value
+  uint32_t raw;     // page mode: raw page index + 1 (0: coded)
   bool ok;          // offsets consistent with the buffer
   bool fits;        // bits staged in shared memory
 };
 
+template <int DT>
 __device__ __forceinline__ ChunkInfo chunk_info(const Batch &b, uint32_t g) {
   ChunkInfo ci;
   ci.item = find_item(b, g);
   const Item &I = b.item[ci.item];
   ci.c = I.first_chunk + (g - I.chunk0);
-  const uint64_t i0 = (uint64_t)ci.c * b.chunk_elems;
-  ci.cnt = (uint32_t)min((uint64_t)b.chunk_elems, I.n - i0);
-  const uint64_t B0 = I.off[ci.c], B1 = I.off[ci.c + 1], Bt = I.off[I.total_chunks];
-  // the stream must hold every chunk's bits plus 16 readable bytes
-  ci.ok = I.off[0] == 0 && B0 <= B1 && B1 <= Bt && (Bt + 7) / 8 + 16 <= I.stream_cap && B1 - B0 >= ci.cnt &&
-          B1 - B0 <= (uint64_t)ci.cnt * 32u;
+  ci.raw = 0;
+  uint64_t B0, B1, Bt, i0;
+  if (I.page_meta) {
+    // page store: the page's codes start at bit 0 of its own slot
+    const uint32_t slot = I.slot_ids[ci.c];
+    ci.cnt = b.chunk_elems;
+    const uint32_t meta = slot < I.n_slots ? I.page_meta[slot] : 0u;
+    const uint64_t sm_page = DT == EH_BF16 ? b.chunk_elems : (DT == EH_FP8_E4M3 ? b.chunk_elems / 2 : 0);
+    ci.sm_off = (uint64_t)slot * sm_page;
+    ci.out_off = (uint64_t)ci.c * b.chunk_elems;
+    if (slot < I.n_slots && (meta & EH_PAGE_RAW)) {
+      const uint32_t idx = meta & ~EH_PAGE_RAW;
+      ci.raw = idx + 1;
+      ci.ok = idx < I.raw_cap;
+      ci.nbits = 0;
+      ci.lo = 0;
+      ci.rel0 = 0;
+      ci.fits = false;
+      ci.bytes = 0;
+      return ci;
+    }
+    B0 = (uint64_t)slot * I.slot_bytes * 8;
+    B1 = B0 + meta;
+    Bt = (uint64_t)I.n_slots * I.slot_bytes * 8;
+    ci.ok = slot < I.n_slots && B1 - B0 >= ci.cnt && B1 - B0 <= (uint64_t)ci.cnt * 32u &&
+            (B1 - B0 + 7) / 8 + 16 <= I.slot_bytes;
+  } else {
+    i0 = (uint64_t)ci.c * b.chunk_elems;
+    ci.cnt = (uint32_t)min((uint64_t)b.chunk_elems, I.n - i0);
+    ci.sm_off = DT == EH_BF16 ? i0 : (DT == EH_FP8_E4M3 ? i0 / 2 : 0);
+    ci.out_off = i0 - I.elem0;
+    B0 = I.off[ci.c];
+    B1 = I.off[ci.c + 1];
+    Bt = I.off[I.total_chunks];
+    // the stream must hold every chunk's bits plus 16 readable bytes
+    ci.ok = I.off[0] == 0 && B0 <= B1 && B1 <= Bt && (Bt + 7) / 8 + 16 <= I.stream_cap &&
+            B1 - B0 >= ci.cnt && B1 - B0 <= (uint64_t)ci.cnt * 32u;
+  }
   ci.nbits = (uint32_t)(B1 - B0);
   ci.lo = (B0 >> 3) & ~uint64_t(15);
   const uint64_t hi = (((B1 + 7) >> 3) + 16 + 15) & ~uint64_t(15);
@@ -646,7 +682,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
     ChunkInfo ci;
     ci.fits = false;
     if (g < seg_end) {
-      ci = chunk_info(b, g);
+      ci = chunk_info<DT>(b, g);
       if (ci.fits && gtid == 0) issue_stage(G, b, ci);
       pending = ci.fits;
     }
@@ -656,7 +692,6 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
     const bool stagger = seg_end - seg >= 2;
     if (stagger && grp == 1) named_sync(kStaggerBarrier, kDecThreads);
     for (; g < seg_end; g += kNumGroups) {
-      const uint64_t i0 = (uint64_t)ci.c * b.chunk_elems;
       const uint32_t cnt = ci.cnt;
       bool ok = ci.ok && !terr && !S.abort_flag;
 
@@ -682,7 +717,19 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
       } else {
         gsync(id);  // the cleared exponent buffer is visible to the group
       }
-      if (ok) {
+      if (ok && ci.raw) {
+        // page stored raw: its exponent bytes go straight to the buffer
+        const uint8_t *src = I.raw_pool + (uint64_t)(ci.raw - 1) * b.chunk_elems;
+        for (uint32_t v = gtid; v < cnt / 16; v += kGroupThreads) {
+          const uint4 x = __ldg((const uint4 *)src + v);
+          uint32_t *d = (uint32_t *)(G.exps + exp_slot(16 * v));  // 4-byte aligned
+          d[0] = x.x;
+          d[1] = x.y;
+          d[2] = x.z;
+          d[3] = x.w;
+        }
+        gsync(id);
+      } else if (ok) {
         if (ci.fits) ok = decode_chunk<true>(G, S.tabs, G.stage, ci.rel0, ci.nbits, cnt, id, gtid, &timeout);
         else
           ok = decode_chunk<false>(G, S.tabs, (const uint32_t *)(I.stream + ci.lo), ci.rel0, ci.nbits, cnt, id,
@@ -699,11 +746,11 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
       ChunkInfo cn;
       cn.fits = false;
       if (g + kNumGroups < seg_end && !pending && !S.abort_flag) {
-        cn = chunk_info(b, g + kNumGroups);
+        cn = chunk_info<DT>(b, g + kNumGroups);
         if (cn.fits && gtid == 0) issue_stage(G, b, cn);
         pending = cn.fits;
       } else if (g + kNumGroups < seg_end) {
-        cn = chunk_info(b, g + kNumGroups);
+        cn = chunk_info<DT>(b, g + kNumGroups);
         cn.fits = false;
       }
 
@@ -711,8 +758,8 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
       if (ok) {
         const uint32_t nvec = cnt / 16;
         if (DT == EH_BF16) {
-          const uint8_t *smp = I.sm + i0;
-          uint16_t *outp = (uint16_t *)I.out + (i0 - I.elem0);
+          const uint8_t *smp = I.sm + ci.sm_off;
+          uint16_t *outp = (uint16_t *)I.out + ci.out_off;
           for (uint32_t v0 = gtid; v0 < nvec; v0 += 4 * kGroupThreads) {
             uint4 m[4];
             #pragma unroll
@@ -745,15 +792,15 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
           }
         } else if (DT == EH_BYTES) {
           // the decoded symbols are the output bytes
-          uint8_t *outp = (uint8_t *)I.out + (i0 - I.elem0);
+          uint8_t *outp = (uint8_t *)I.out + ci.out_off;
           for (uint32_t v = gtid; v < nvec; v += kGroupThreads) {
             const uint32_t *ew = (const uint32_t *)(G.exps + exp_slot(16 * v));
             *(uint4 *)(outp + 16 * (uint64_t)v) = make_uint4(ew[0], ew[1], ew[2], ew[3]);
           }
           for (uint32_t i = nvec * 16 + gtid; i < cnt; i += kGroupThreads) outp[i] = G.exps[exp_slot(i)];
         } else {
-          const uint8_t *smp = I.sm + i0 / 2;
-          uint8_t *outp = (uint8_t *)I.out + (i0 - I.elem0);
+          const uint8_t *smp = I.sm + ci.sm_off;
+          uint8_t *outp = (uint8_t *)I.out + ci.out_off;
           for (uint32_t v0 = gtid; v0 < nvec; v0 += 4 * kGroupThreads) {
             uint2 m[4];
             #pragma unroll

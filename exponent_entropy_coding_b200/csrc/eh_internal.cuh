@@ -22,6 +22,7 @@ constexpr int kStageBytes = 32 * 1024;  // shared-memory window for one chunk's 
 constexpr uint32_t kFlagCorrupt = 1u;
 constexpr uint32_t kFlagInfeasible = 2u;
 constexpr uint32_t kFlagTimeout = 4u;
+constexpr uint32_t kFlagNoRoom = 8u;   // raw page pool exhausted
 
 __host__ __device__ inline int alphabet_of(int dtype) { return dtype == EH_FP8_E4M3 ? 16 : 256; }
 
@@ -49,6 +50,33 @@ struct Item {
   uint64_t *bits_out;      // compress: total bits (workspace copy)
   uint64_t *bits_dev;      // compress: optional caller copy (may be null)
   void *lut;               // decompress: DecodeTables
+  // page store mode (chunks live in fixed slots; null page_meta = tensor mode)
+  const uint32_t *slot_ids;  // [nchunks] slot of each page of the call
+  const uint32_t *page_meta; // [n_slots] code bits, or EH_PAGE_RAW | raw index
+  const uint8_t *raw_pool;   // [raw_cap][chunk_elems] exponent bytes
+  uint64_t slot_bytes;
+  uint32_t n_slots;
+  uint32_t raw_cap;
+};
+
+// Launch descriptor of the page append kernel.
+struct PageLaunch {
+  const void *in;
+  const uint32_t *slot_ids;
+  uint32_t n_pages;
+  uint32_t page_elems;
+  const uint8_t *code_len;
+  const uint32_t *code;
+  uint8_t *slots;
+  uint64_t slot_bytes;
+  uint32_t n_slots;
+  uint32_t raw_cap;
+  uint8_t *sm;
+  uint32_t *page_meta;
+  uint8_t *raw_pool;
+  uint32_t *raw_used;
+  uint32_t *status;
+  int32_t dtype;
 };
 
 struct Batch {
@@ -113,6 +141,7 @@ cudaError_t launch_hist(const Batch &b, cudaStream_t s);
 cudaError_t launch_book(const Batch &b, cudaStream_t s);
 cudaError_t launch_offsets(const Batch &b, cudaStream_t s);
 cudaError_t launch_encode(const Batch &b, cudaStream_t s);
+cudaError_t launch_page_append(const PageLaunch &pl, cudaStream_t s);
 cudaError_t launch_tables(const Batch &b, cudaStream_t s);
 cudaError_t launch_decode(const Batch &b, cudaStream_t s, int num_sms);
 cudaError_t configure_decode();  // once per device, before the first decode launch

@@ -32,8 +32,10 @@ EH_ERR_CUDA, EH_ERR_CORRUPT, EH_ERR_TIMEOUT, EH_ERR_NOMEM = 4, 5, 6, 7
 EXPORTED = ["eh_plan", "eh_compress_bound", "eh_compress_batch_workspace", "eh_compress",
             "eh_compress_batch", "eh_compress_shard_begin", "eh_compress_shard_finish",
             "eh_decompress_workspace", "eh_decompress", "eh_decompress_batch",
-            "eh_decompress_chunks", "eh_decompress_batch_noalloc", "eh_get_status", "eh_status_str",
-            "eh_version"]
+            "eh_decompress_chunks", "eh_decompress_batch_noalloc", "eh_codebook_from_counts",
+            "eh_pages_append", "eh_pages_read",
+            "eh_get_status", "eh_status_str", "eh_version"]
+EH_PAGE_RAW = 0x80000000
 
 
 class EhError(RuntimeError):
@@ -52,6 +54,13 @@ class eh_compressed_t(C.Structure):
                 ("code_len", C.c_void_p), ("code", C.c_void_p), ("chunk_bit_off", C.c_void_p),
                 ("exp_stream", C.c_void_p), ("exp_stream_cap", C.c_uint64),
                 ("sign_mant", C.c_void_p), ("exp_stream_bits", C.c_uint64)]
+
+
+class eh_page_store_t(C.Structure):
+    _fields_ = [("code_len", C.c_void_p), ("code", C.c_void_p), ("slots", C.c_void_p),
+                ("slot_bytes", C.c_uint64), ("n_slots", C.c_uint32), ("raw_cap", C.c_uint32),
+                ("sign_mant", C.c_void_p), ("page_meta", C.c_void_p), ("raw_pool", C.c_void_p),
+                ("raw_used", C.c_void_p)]
 
 
 _lib = None
@@ -79,6 +88,9 @@ def lib():
             "eh_decompress_batch": [P(eh_plan_t), C.c_int, P(eh_compressed_t), P(vp), vp, u64, vp],
             "eh_decompress_chunks": [P(eh_plan_t), P(eh_compressed_t), u32, u32, vp, vp, u64, vp],
             "eh_decompress_batch_noalloc": [P(eh_plan_t), C.c_int, P(eh_compressed_t), P(vp), vp],
+            "eh_codebook_from_counts": [P(eh_plan_t), vp, vp, vp, vp, u64, vp],
+            "eh_pages_append": [P(eh_plan_t), P(eh_page_store_t), vp, u32, vp, vp, u64, vp],
+            "eh_pages_read": [P(eh_plan_t), P(eh_page_store_t), vp, u32, vp, vp, u64, vp],
             "eh_get_status": [vp, vp],
             "eh_status_str": [C.c_int],
             "eh_version": [],
@@ -336,3 +348,82 @@ def get_status(workspace: torch.Tensor, stream=None) -> int:
 
 def version() -> str:
     return lib().eh_version().decode()
+
+
+def codebook_from_counts(p: eh_plan_t, counts: torch.Tensor, stream=None):
+    """(code_len uint8[A], code int32[A]) on the counts' device from
+    exponent counts (int64[A], uint64 values)."""
+    counts = counts.contiguous()
+    A = alphabet(p.dtype)
+    code_len = torch.zeros(A, dtype=torch.uint8, device=counts.device)
+    code = torch.zeros(A, dtype=torch.int32, device=counts.device)
+    ws = torch.empty(compress_bound(p, 0)[2], dtype=torch.uint8, device=counts.device)
+    rc = lib().eh_codebook_from_counts(C.byref(p), C.c_void_p(counts.data_ptr()),
+                                       C.c_void_p(code_len.data_ptr()), C.c_void_p(code.data_ptr()),
+                                       C.c_void_p(ws.data_ptr()), ws.numel(), _stream_ptr(stream))
+    _check(rc, "eh_codebook_from_counts")
+    _check(get_status(ws, stream), "eh_codebook_from_counts (device status)")
+    return code_len, code
+
+
+class PageStore:
+    """Fixed-slot page store (device arrays owned by torch) for online K/V
+    compression with a frozen codebook."""
+
+    def __init__(self, p: eh_plan_t, code_len: torch.Tensor, code: torch.Tensor, n_slots: int,
+                 slot_bytes: int, raw_cap: int, device):
+        dev = torch.device(device)
+        n = p.chunk_elems
+        sm_page = n if p.dtype == EH_BF16 else (n // 2 if p.dtype == EH_FP8_E4M3 else 0)
+        self.plan = p
+        self.code_len, self.code = code_len, code
+        self.n_slots, self.slot_bytes, self.raw_cap = n_slots, slot_bytes, raw_cap
+        self.slots = torch.zeros(n_slots * slot_bytes, dtype=torch.uint8, device=dev)
+        self.sign_mant = torch.empty(n_slots * sm_page, dtype=torch.uint8, device=dev)
+        self.page_meta = torch.zeros(n_slots, dtype=torch.int32, device=dev)
+        self.raw_pool = torch.empty(max(raw_cap, 1) * n, dtype=torch.uint8, device=dev)
+        self.raw_used = torch.zeros(1, dtype=torch.int32, device=dev)
+        self.workspace = torch.empty(max(256, decompress_workspace(p, 1)), dtype=torch.uint8, device=dev)
+
+    def struct(self) -> eh_page_store_t:
+        s = eh_page_store_t()
+        s.code_len = self.code_len.data_ptr()
+        s.code = self.code.data_ptr()
+        s.slots = self.slots.data_ptr()
+        s.slot_bytes = self.slot_bytes
+        s.n_slots = self.n_slots
+        s.raw_cap = self.raw_cap
+        s.sign_mant = self.sign_mant.data_ptr() if self.sign_mant.numel() else None
+        s.page_meta = self.page_meta.data_ptr()
+        s.raw_pool = self.raw_pool.data_ptr()
+        s.raw_used = self.raw_used.data_ptr()
+        return s
+
+    def append(self, x: torch.Tensor, slot_ids: torch.Tensor, stream=None):
+        """Codes len(slot_ids) full pages of x into the given slots."""
+        x = _raw(x)
+        ids = slot_ids.to(device=x.device, dtype=torch.int32).contiguous()
+        st = self.struct()
+        rc = lib().eh_pages_append(C.byref(self.plan), C.byref(st), C.c_void_p(x.data_ptr()), ids.numel(),
+                                   C.c_void_p(ids.data_ptr()), C.c_void_p(self.workspace.data_ptr()),
+                                   self.workspace.numel(), _stream_ptr(stream))
+        _check(rc, "eh_pages_append")
+        return ids
+
+    def read(self, slot_ids: torch.Tensor, out: Optional[torch.Tensor] = None, stream=None,
+             check: bool = True) -> torch.Tensor:
+        ids = slot_ids.to(device=self.slots.device, dtype=torch.int32).contiguous()
+        n = ids.numel() * self.plan.chunk_elems
+        if out is None:
+            out = torch.empty(n, dtype=_elem_dtype(self.plan.dtype), device=self.slots.device)
+        st = self.struct()
+        rc = lib().eh_pages_read(C.byref(self.plan), C.byref(st), C.c_void_p(ids.data_ptr()), ids.numel(),
+                                 C.c_void_p(out.data_ptr()), C.c_void_p(self.workspace.data_ptr()),
+                                 self.workspace.numel(), _stream_ptr(stream))
+        _check(rc, "eh_pages_read")
+        if check:
+            _check(get_status(self.workspace, stream), "eh_pages_read (device status)")
+        return out
+
+    def status(self, stream=None) -> int:
+        return get_status(self.workspace, stream)

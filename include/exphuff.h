@@ -216,8 +216,58 @@ EH_API eh_status eh_decompress_batch_noalloc(const eh_plan_t *plan, int k,
                                              const eh_compressed_t *cs,
                                              void *const *outs, void *stream);
 
+/* ---- Fixed-slot page store: online K/V cache compression.
+ * New K/V pages (one page = one chunk of chunk_elems values, e.g. 64 tokens x
+ * 8 heads x 128 dims = 65,536) are coded with a FROZEN codebook (code_len /
+ * code of an earlier eh_compress, e.g. of the prefill) into fixed-capacity
+ * slots, and decoded on reuse (ZipFloat §3.3 and §4.2: KV entries go to
+ * preallocated slots and are decompressed on demand; the paper summary,
+ * "局限性": real-time K/V compression needs a high-throughput
+ * implementation).  A page whose code does not fit its slot (ceil(bits/8) +
+ * 16 > slot_bytes) or that holds an exponent without a code is stored raw:
+ * its exponent fields (one byte each) go to the next free page of raw_pool.
+ * All arrays are device arrays owned by the caller. */
+#define EH_PAGE_RAW 0x80000000u /* page_meta: raw page; low 31 bits = raw index */
+typedef struct {
+  const uint8_t *code_len; /* device [A]: the frozen codebook                   */
+  const uint32_t *code;    /* device [A]                                         */
+  uint8_t *slots;          /* device [n_slots][slot_bytes]: codes from bit 0;
+                              bytes past ceil(bits/8) are unspecified           */
+  uint64_t slot_bytes;     /* multiple of 16                                     */
+  uint32_t n_slots;
+  uint32_t raw_cap;        /* pages raw_pool can hold                            */
+  uint8_t *sign_mant;      /* device [n_slots][sm bytes of one page]             */
+  uint32_t *page_meta;     /* device [n_slots]: code bits, or EH_PAGE_RAW | idx  */
+  uint8_t *raw_pool;       /* device [raw_cap][chunk_elems] exponent bytes      */
+  uint32_t *raw_used;      /* device counter of raw pages taken (zero it once)   */
+} eh_page_store_t;
+
+/* Codebook (code_len[A], code[A], device) from exponent counts (device
+ * u64[A]), exactly as eh_compress builds it for a tensor with those counts.
+ * To freeze a codebook for the page store that codes every exponent, pass the
+ * counts of earlier data plus one for every symbol.  Stream-ordered;
+ * workspace: the workspace_bytes of eh_compress_bound(plan, 0, ...). */
+EH_API eh_status eh_codebook_from_counts(const eh_plan_t *plan, const uint64_t *counts,
+                                         uint8_t *code_len, uint32_t *code,
+                                         void *workspace, uint64_t workspace_bytes,
+                                         void *stream);
+
+/* Codes n_pages full pages (in: n_pages * chunk_elems values, page i first)
+ * into the slots slot_ids[i] (device array).  Stream-ordered; a full raw pool
+ * sets EH_ERR_NOMEM in the workspace status word (workspace: 256 bytes). */
+EH_API eh_status eh_pages_append(const eh_plan_t *plan, const eh_page_store_t *store,
+                                 const void *in, uint32_t n_pages,
+                                 const uint32_t *slot_ids, void *workspace,
+                                 uint64_t workspace_bytes, void *stream);
+
+/* Decodes the pages in slots slot_ids[i] (device array) into out (page i at
+ * out + i * chunk_elems values).  Workspace: eh_decompress_workspace(plan, 1). */
+EH_API eh_status eh_pages_read(const eh_plan_t *plan, const eh_page_store_t *store,
+                               const uint32_t *slot_ids, uint32_t n_pages, void *out,
+                               void *workspace, uint64_t workspace_bytes, void *stream);
+
 /* Waits for `stream` and returns the status word of `workspace`: EH_OK,
- * EH_ERR_CORRUPT, EH_ERR_INFEASIBLE or EH_ERR_TIMEOUT.  Every compress or
+ * EH_ERR_CORRUPT, EH_ERR_INFEASIBLE, EH_ERR_NOMEM or EH_ERR_TIMEOUT.  Every compress or
  * decompress call resets the word when it starts, so it describes the most
  * recent call that used this workspace. */
 EH_API eh_status eh_get_status(void *workspace, void *stream);

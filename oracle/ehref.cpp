@@ -447,4 +447,66 @@ int ehref_decompress(int dtype, uint64_t n, uint32_t chunk, const uint8_t *len,
                                  stream_bytes, sm_packed, 0, (uint32_t)C, out);
 }
 
+int ehref_page_encode(int dtype, const void *in, uint64_t n, const uint8_t *len,
+                      const uint32_t *code, uint8_t *slot, uint64_t slot_bytes,
+                      uint8_t *sm_packed, uint8_t *raw_exps, uint64_t *bits,
+                      int *raw) {
+  if (!alphabet_of(dtype)) return EHREF_EINVAL;
+  int rc = ehref_pack_sm(dtype, in, n, sm_packed);
+  if (rc) return rc;
+  /* code bits of the page; an exponent without a code forces raw storage */
+  uint64_t total = 0;
+  bool missing = false;
+  for (uint64_t i = 0; i < n; i++) {
+    uint8_t e, sm;
+    split_one(dtype, load_elem(dtype, in, i), &e, &sm);
+    if (len[e] == 0) missing = true;
+    total += len[e];
+  }
+  if (missing || (total + 7) / 8 + 16 > slot_bytes) {
+    for (uint64_t i = 0; i < n; i++) {
+      uint8_t e, sm;
+      split_one(dtype, load_elem(dtype, in, i), &e, &sm);
+      raw_exps[i] = e;
+    }
+    *raw = 1;
+    *bits = 0;
+    return EHREF_OK;
+  }
+  for (uint64_t b = 0; b < slot_bytes; b++) slot[b] = 0;
+  uint64_t pos = 0;
+  for (uint64_t i = 0; i < n; i++) {
+    uint8_t e, sm;
+    split_one(dtype, load_elem(dtype, in, i), &e, &sm);
+    for (int b = len[e] - 1; b >= 0; b--) put_bit(slot, pos++, (code[e] >> b) & 1u);
+  }
+  *raw = 0;
+  *bits = pos;
+  return EHREF_OK;
+}
+
+int ehref_page_decode(int dtype, uint64_t n, const uint8_t *len,
+                      const uint32_t *code, const uint8_t *slot,
+                      uint64_t slot_bytes, uint64_t bits, int raw,
+                      const uint8_t *raw_exps, const uint8_t *sm_packed,
+                      void *out) {
+  if (!alphabet_of(dtype)) return EHREF_EINVAL;
+  if (raw) {
+    for (uint64_t i = 0; i < n; i++) {
+      uint32_t sm = 0;
+      if (dtype == EHREF_BF16)
+        sm = sm_packed[i];
+      else if (dtype == EHREF_FP8_E4M3)
+        sm = (sm_packed[i / 2] >> (4 * (i & 1))) & 0xFu;
+      store_elem(dtype, out, i, merge_one(dtype, raw_exps[i], sm));
+    }
+    return EHREF_OK;
+  }
+  /* one coded chunk: offsets [0, bits] */
+  uint64_t off[2] = {0, bits};
+  if ((bits + 7) / 8 > slot_bytes) return EHREF_ECORRUPT;
+  return ehref_decompress_chunks(dtype, n, n ? (uint32_t)n : 1u, len, code, off, slot,
+                                 slot_bytes, sm_packed, 0, n ? 1u : 0u, out);
+}
+
 }  // extern "C"

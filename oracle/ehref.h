@@ -111,6 +111,29 @@ int ehref_decompress(int dtype, uint64_t n, uint32_t chunk, const uint8_t *len,
                      const uint8_t *stream, uint64_t stream_bytes,
                      const uint8_t *sm_packed, void *out);
 
+/* Fixed-slot page store (online K/V cache compression).  A page of n values
+ * (one chunk; 64 tokens x 8 heads x 128 dims = 65,536 for Llama-3.1-8B K/V) is
+ * coded with a FROZEN codebook (len/code from earlier data) into a slot of
+ * slot_bytes bytes: the codes MSB-first from bit 0 of the slot, the rest of
+ * the slot zero.  The page is stored raw instead -- *raw = 1, slot untouched,
+ * exponent fields copied to raw_exps (one byte each) -- when one of its
+ * exponents has no code or when ceil(bits/8) + 16 > slot_bytes (the decoder
+ * reads up to 16 bytes past the last code).  sm_packed receives the page's
+ * sign/mantissa array in every case.  Sources: ZipFloat §3.3 and §4.2 (new KV
+ * entries are compressed into preallocated slots and decompressed on reuse);
+ * the paper summary "局限性" and "开放问题" (real-time K/V compression). */
+int ehref_page_encode(int dtype, const void *in, uint64_t n, const uint8_t *len,
+                      const uint32_t *code, uint8_t *slot, uint64_t slot_bytes,
+                      uint8_t *sm_packed, uint8_t *raw_exps, uint64_t *bits,
+                      int *raw);
+
+/* Inverse: rebuilds the page's n values from its slot (or raw exponents). */
+int ehref_page_decode(int dtype, uint64_t n, const uint8_t *len,
+                      const uint32_t *code, const uint8_t *slot,
+                      uint64_t slot_bytes, uint64_t bits, int raw,
+                      const uint8_t *raw_exps, const uint8_t *sm_packed,
+                      void *out);
+
 #ifdef __cplusplus
 }
 #endif

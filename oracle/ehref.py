@@ -50,6 +50,8 @@ def lib():
             "ehref_compress": (i32, [i32, vp, u64, u32, i32, vp, vp, vp, vp, u64, vp, vp]),
             "ehref_decompress_chunks": (i32, [i32, u64, u32, vp, vp, vp, vp, u64, vp, u32, u32, vp]),
             "ehref_decompress": (i32, [i32, u64, u32, vp, vp, vp, vp, u64, vp, vp]),
+            "ehref_page_encode": (i32, [i32, vp, u64, vp, vp, vp, u64, vp, vp, vp, vp]),
+            "ehref_page_decode": (i32, [i32, u64, vp, vp, vp, u64, u64, i32, vp, vp, vp]),
         }
         for name, (res, args) in sig.items():
             f = getattr(_lib, name)
@@ -205,3 +207,36 @@ def decompress(c: Compressed, first=None, count=None):
         _p(np.ascontiguousarray(c.chunk_bit_off, np.uint64)), _p(stream), stream.size,
         _p(np.ascontiguousarray(c.sign_mant, np.uint8)), first, count, _p(out)))
     return out
+
+
+@dataclass
+class Page:
+    slot: np.ndarray       # uint8[slot_bytes] (zero beyond the codes)
+    bits: int
+    raw: bool
+    raw_exps: np.ndarray   # uint8[n] when raw
+    sign_mant: np.ndarray
+
+
+def page_encode(dtype, x, lengths, codes, slot_bytes):
+    x = np.ascontiguousarray(x, dtype=elem_dtype(dtype))
+    n = x.size
+    slot = np.zeros(slot_bytes, np.uint8)
+    sm = np.zeros(max(sm_bytes(dtype, n), 1), np.uint8)
+    raw_exps = np.zeros(max(n, 1), np.uint8)
+    bits = C.c_uint64(0)
+    raw = C.c_int(0)
+    _check(lib().ehref_page_encode(dtype, _p(x), n, _p(np.ascontiguousarray(lengths, np.uint8)),
+                                   _p(np.ascontiguousarray(codes, np.uint32)), _p(slot), slot_bytes,
+                                   _p(sm), _p(raw_exps), C.byref(bits), C.byref(raw)))
+    return Page(slot, bits.value, bool(raw.value), raw_exps[:n], sm[:sm_bytes(dtype, n)])
+
+
+def page_decode(dtype, n, lengths, codes, page: Page):
+    out = np.zeros(max(n, 1), elem_dtype(dtype))
+    _check(lib().ehref_page_decode(dtype, n, _p(np.ascontiguousarray(lengths, np.uint8)),
+                                   _p(np.ascontiguousarray(codes, np.uint32)), _p(page.slot),
+                                   page.slot.size, page.bits, int(page.raw),
+                                   _p(np.ascontiguousarray(page.raw_exps, np.uint8)),
+                                   _p(np.ascontiguousarray(page.sign_mant, np.uint8)), _p(out)))
+    return out[:n]

@@ -452,3 +452,55 @@ def test_fp4_scale_generators():
     s = synth.nvfp4_block_scales(w)
     vals = torch.from_numpy(s.copy()).view(torch.float8_e4m3fn).float().tolist()
     assert vals == [448.0, 112.0]
+
+
+# ------------------------------------------------ fixed-slot K/V page store
+
+def _kv_pages(n_pages=6):
+    _, items = synth.workload("kv_layer", scale=64)
+    return items[0][1][: n_pages * 65536]
+
+
+def _smoothed_book(oracle, prefill):
+    """Codebook of the prefill's counts plus one for every symbol."""
+    cnt = oracle.histogram(0, prefill) + np.uint64(1)
+    lens = oracle.code_lengths(cnt, 32)
+    return lens, oracle.canonical_codes(lens)
+
+
+def test_page_slot_equals_chunk_stream(oracle):
+    k = _kv_pages()
+    lens, codes = _smoothed_book(oracle, k[: 3 * 65536])
+    assert lens.min() > 0 and lens.max() <= 32          # every exponent has a code
+    page = k[4 * 65536: 5 * 65536]
+    pg = oracle.page_encode(0, page, lens, codes, 32 * 1024)
+    assert not pg.raw
+    off, stream, bits = oracle.encode(0, page, 65536, lens, codes)
+    assert pg.bits == bits and list(off) == [0, bits]
+    assert np.array_equal(pg.slot[: stream.size], stream) and not pg.slot[stream.size:].any()
+    assert np.array_equal(pg.sign_mant, oracle.pack_sm(0, page))
+    assert np.array_equal(oracle.page_decode(0, 65536, lens, codes, pg), page)
+
+
+def test_page_capacity_boundary(oracle):
+    k = _kv_pages()
+    lens, codes = _smoothed_book(oracle, k[: 3 * 65536])
+    page = k[3 * 65536: 4 * 65536]
+    bits = oracle.page_encode(0, page, lens, codes, 1 << 20).bits
+    need = (bits + 7) // 8 + 16
+    assert not oracle.page_encode(0, page, lens, codes, need).raw
+    pg = oracle.page_encode(0, page, lens, codes, need - 1)
+    assert pg.raw and pg.bits == 0
+    assert np.array_equal(pg.raw_exps, oracle.split(0, page)[0])
+    assert np.array_equal(oracle.page_decode(0, 65536, lens, codes, pg), page)
+
+
+def test_page_missing_symbol_is_raw(oracle):
+    k = _kv_pages()
+    book = oracle.compress(0, k[: 2 * 65536])
+    page = k[2 * 65536: 3 * 65536].copy()
+    page[100] = 0x7F00                      # exponent 254: not in the codebook
+    assert book.code_len[254] == 0
+    pg = oracle.page_encode(0, page, book.code_len, book.code, 64 * 1024)
+    assert pg.raw
+    assert np.array_equal(oracle.page_decode(0, 65536, book.code_len, book.code, pg), page)
