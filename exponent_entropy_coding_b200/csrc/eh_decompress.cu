@@ -134,13 +134,19 @@ __global__ void __launch_bounds__(256) tables_kernel(const __grid_constant__ Bat
   const uint32_t sub0 = (uint32_t)(limL[kLutBits] >> kShift);
   constexpr uint32_t kPerPart = (1u << kLutBits) / kTabParts;
   for (uint32_t p = part * kPerPart + tid; p < (part + 1) * kPerPart; p += 256) {
-    uint32_t syms = 0, pos = 0, nc = 0, bnd = 0;
-    while (nc < 4 && pos < (uint32_t)kLutBits) {
+    // every complete code inside the index bits: all of them for counting,
+    // the first four (their symbols fill 32 bits) for writing
+    uint32_t syms = 0, pos = 0, nc = 0, bnd = 0, pos4 = 0, nc4 = 0;
+    while (pos < (uint32_t)kLutBits) {
       const uint32_t x = (p << kShift) << pos;  // next bits, left-justified, zero-filled
       const uint32_t L = code_length_of(x, limL);
       if (L > (uint32_t)kLutBits - pos) break;  // not complete inside the index bits
-      const uint32_t v = x >> (32 - L);
-      syms |= (uint32_t)srt[baseL[L] + v - firstL[L]] << (8 * nc);
+      if (nc < 4) {
+        const uint32_t v = x >> (32 - L);
+        syms |= (uint32_t)srt[baseL[L] + v - firstL[L]] << (8 * nc);
+        pos4 = pos + L;
+        nc4 = nc + 1;
+      }
       bnd |= 1u << pos;
       pos += L;
       nc++;
@@ -148,7 +154,7 @@ __global__ void __launch_bounds__(256) tables_kernel(const __grid_constant__ Bat
     uint32_t sub = kNoSub;
     if (nc == 0 && ((uint64_t)p << kShift) < limL[32] && p - sub0 < (uint32_t)kNumSub) sub = p - sub0;
     T->l1sym[p] = syms;
-    T->l1meta[p] = pos | (nc << 4) | (bnd << 7) | (sub << 19);
+    T->l1meta[p] = pos4 | (nc4 << 4) | (bnd << 7) | (sub << 19) | (pos << 24) | (nc << 28);
   }
   if (part != 0) return;
   // second level: codes of kLutBits+1 .. kLutBits+8 bits
@@ -199,7 +205,7 @@ __device__ __forceinline__ uint32_t lut_index(uint32_t x) { return x >> (32 - kL
 // invalid code.
 __device__ __forceinline__ uint32_t decode_long(const DecodeTables &T, uint32_t peek, uint32_t meta,
                                                 uint32_t &syms, uint32_t &nbits) {
-  const uint32_t si = (meta >> 19) & 63u;
+  const uint32_t si = (meta >> 19) & 31u;
   if (si != kNoSub) {
     const uint32_t e2 = T.sub[si][(peek >> (24 - kLutBits)) & 0xFFu];
     const uint32_t l = (e2 >> 8) & 63u;
@@ -228,9 +234,12 @@ __device__ __forceinline__ uint32_t decode_step(const DecodeTables &T, uint32_t 
                                                 uint32_t &syms, uint32_t &nbits, uint32_t &bnd) {
   const uint32_t idx = lut_index(x);
   const uint32_t meta = T.l1meta[idx];
-  uint32_t k = (meta >> 4) & 7u;
+  // writing takes the first four codes (their symbols), counting all of them
+  uint32_t k = kSyms ? (meta >> 4) & 7u : meta >> 28;
   if (k) {
-    uint32_t nb = meta & 15u, bm = (meta >> 7) & 0xFFFu;
+    uint32_t nb = kSyms ? meta & 15u : (meta >> 24) & 15u;
+    uint32_t bm = (meta >> 7) & 0xFFFu;
+    if (kSyms) bm &= (1u << nb) - 1u;
     uint32_t sy = kSyms ? T.l1sym[idx] : 0u;
     if (nb > lim) {
       // codes starting at or after the limit belong to the next window
@@ -423,7 +432,7 @@ __device__ bool decode_chunk(GroupSmem &G, const DecodeTables &T, const uint32_t
     const uint32_t x = peek(rel0 + pos);
     const uint32_t off = pos - ws;
     const uint32_t m1 = T.l1meta[lut_index(x)];
-    const uint32_t k1 = (m1 >> 4) & 7u, nb1 = m1 & 15u;
+    const uint32_t k1 = m1 >> 28, nb1 = (m1 >> 24) & 15u;
     if (!k1) {
       uint32_t syms, nb;
       if (!decode_long(T, x, m1, syms, nb)) { bad = true; break; }
@@ -433,7 +442,7 @@ __device__ bool decode_chunk(GroupSmem &G, const DecodeTables &T, const uint32_t
       continue;
     }
     const uint32_t m2 = T.l1meta[lut_index(x << nb1)];
-    const uint32_t k2 = (m2 >> 4) & 7u, nb2 = m2 & 15u;
+    const uint32_t k2 = m2 >> 28, nb2 = (m2 >> 24) & 15u;
     if (off < kMaskBits) {
       mask |= (uint64_t)((m1 >> 7) & 0xFFFu) << off;
       if (k2 && off + nb1 < kMaskBits) mask |= (uint64_t)((m2 >> 7) & 0xFFFu) << (off + nb1);

@@ -108,16 +108,18 @@ __device__ __forceinline__ void set_status(uint32_t *status, uint32_t flag) {
 // workspace and copied to shared memory by each decoding CTA.
 //
 // First level, indexed by the next kLutBits stream bits, as two u32 arrays:
-//   l1sym:  up to four decoded symbols, 8 bits each (first in bits 0..7)
-//   l1meta: bits  0..3  bits consumed by the `cnt` complete codes in the index
-//           bits  4..6  cnt: complete codes inside the index bits (0..4)
-//           bits  7..18 bit i set when one of those codes starts at offset i
-//           bits 19..24 second-level table of this prefix (kNoSub: none)
+//   l1sym:  the symbols of the first four complete codes, 8 bits each
+//   l1meta: bits  0..3  bits consumed by those (up to four) codes
+//           bits  4..6  their number (0..4)
+//           bits  7..18 bit i set when a complete code starts at offset i
+//           bits 19..23 second-level table of this prefix (kNoSub: none)
+//           bits 24..27 bits consumed by all complete codes in the index
+//           bits 28..31 their number (0..12); counting uses these
 // Second level, indexed by the 8 bits after the prefix.  u32 entry:
 //   bits 0..7 symbol, bits 8..13 code length (0: longer -> search).
 // The search path handles any length up to 32 with the canonical limits.
 constexpr int kLutBits = 12;
-constexpr uint32_t kNoSub = 63;
+constexpr uint32_t kNoSub = 31;
 struct DecodeTables {
   uint32_t l1meta[1 << kLutBits];
   uint32_t l1sym[1 << kLutBits];
