@@ -382,27 +382,31 @@ __device__ __forceinline__ uint32_t group_excl_scan(uint32_t v, uint32_t *wsum, 
 // shares with its neighbours need no special case.
 struct ExpWriter {
   uint32_t *words;  // exponent buffer as words
-  uint32_t wj;      // output index of the word being filled (multiple of 4)
-  uint32_t na;      // bytes of that word filled so far (those below the run are zero)
-  uint64_t acc;
+  uint32_t wi;      // word being filled (exponents 4*wi .. 4*wi+3)
+  uint32_t s;       // bits of that word filled so far (those below the run are zero)
+  uint32_t acc;
   __device__ __forceinline__ void init(uint8_t *e, uint32_t j) {
     words = (uint32_t *)e;
-    wj = j & ~3u;
-    na = j & 3u;
+    wi = j >> 2;
+    s = 8 * (j & 3u);
     acc = 0;
   }
-  __device__ __forceinline__ void put(uint32_t syms, uint32_t k) {
-    acc |= (uint64_t)syms << (8 * na);
-    na += k;
-    if (na >= 4) {
-      atomicOr(words + (exp_slot(wj) >> 2), (uint32_t)acc);
-      acc >>= 32;
-      na -= 4;
-      wj += 4;
+  // up to four symbols, first in the low byte, zero above; k8 = 8 * count
+  __device__ __forceinline__ void put(uint32_t syms, uint32_t k8) {
+    const uint32_t lo = acc | (syms << s);
+    const uint32_t hi = __funnelshift_l(syms, 0u, s);  // the bytes past the word; none for s = 0
+    s += k8;
+    if (s >= 32) {
+      atomicOr(words + wi + (wi >> 5), lo);  // word wi of the padded rows
+      wi++;
+      acc = hi;
+      s -= 32;
+    } else {
+      acc = lo;
     }
   }
   __device__ __forceinline__ void finish() {
-    if (na) atomicOr(words + (exp_slot(wj) >> 2), (uint32_t)acc);
+    if (s) atomicOr(words + wi + (wi >> 5), acc);
   }
 };
 
@@ -428,7 +432,8 @@ __device__ bool decode_chunk(GroupSmem &G, const DecodeTables &T, const uint32_t
   uint32_t pos = ws, n = 0;
   uint64_t mask = 0;
   bool bad = false;
-  while (pos + kBulk <= we) {
+  // (a) while the recorded bits last
+  while (pos + kBulk <= we && pos - ws < kMaskBits) {
     const uint32_t x = peek(rel0 + pos);
     const uint32_t off = pos - ws;
     const uint32_t m1 = T.l1meta[lut_index(x)];
@@ -436,25 +441,35 @@ __device__ bool decode_chunk(GroupSmem &G, const DecodeTables &T, const uint32_t
     if (!k1) {
       uint32_t syms, nb;
       if (!decode_long(T, x, m1, syms, nb)) { bad = true; break; }
-      if (off < kMaskBits) mask |= 1ull << off;
+      mask |= 1ull << off;
+      pos += nb;
+      n += 1;
+      continue;
+    }
+    // a prefix with no complete code has count, bits and starts all zero
+    const uint32_t m2 = T.l1meta[lut_index(x << nb1)];
+    mask |= (uint64_t)((m1 >> 7) & 0xFFFu) << off;
+    if (off + nb1 < kMaskBits) mask |= (uint64_t)((m2 >> 7) & 0xFFFu) << (off + nb1);
+    pos += nb1 + ((m2 >> 24) & 15u);
+    n += k1 + (m2 >> 28);
+  }
+  // (b) the rest of the window, counting only
+  while (!bad && pos + kBulk <= we) {
+    const uint32_t x = peek(rel0 + pos);
+    const uint32_t m1 = T.l1meta[lut_index(x)];
+    const uint32_t k1 = m1 >> 28, nb1 = (m1 >> 24) & 15u;
+    if (!k1) {
+      uint32_t syms, nb;
+      if (!decode_long(T, x, m1, syms, nb)) { bad = true; break; }
       pos += nb;
       n += 1;
       continue;
     }
     const uint32_t m2 = T.l1meta[lut_index(x << nb1)];
-    const uint32_t k2 = m2 >> 28, nb2 = (m2 >> 24) & 15u;
-    if (off < kMaskBits) {
-      mask |= (uint64_t)((m1 >> 7) & 0xFFFu) << off;
-      if (k2 && off + nb1 < kMaskBits) mask |= (uint64_t)((m2 >> 7) & 0xFFFu) << (off + nb1);
-    }
-    if (!k2) {
-      pos += nb1;
-      n += k1;
-      continue;
-    }
-    pos += nb1 + nb2;
-    n += k1 + k2;
+    pos += nb1 + ((m2 >> 24) & 15u);
+    n += k1 + (m2 >> 28);
   }
+  // (c) the window's last bits, taking only codes that start inside it
   while (!bad && pos < we) {
     uint32_t syms, nb, bnd;
     const uint32_t k = decode_step<false>(T, peek(rel0 + pos), we - pos, syms, nb, bnd);
@@ -535,18 +550,18 @@ __device__ bool decode_chunk(GroupSmem &G, const DecodeTables &T, const uint32_t
     const uint32_t x = peek(rel0 + pos);
     const uint32_t i1 = lut_index(x);
     const uint32_t m1 = T.l1meta[i1];
-    const uint32_t k1 = (m1 >> 4) & 7u, nb1 = m1 & 15u;
+    const uint32_t k1 = (m1 >> 1) & 0x38u, nb1 = m1 & 15u;  // k1: 8 * codes
     if (!k1) {
       uint32_t syms, nb;
       if (!decode_long(T, x, m1, syms, nb)) break;
       pos += nb;
-      out.put(syms, 1);
+      out.put(syms, 8);
       continue;
     }
     const uint32_t s1 = T.l1sym[i1];
     const uint32_t i2 = lut_index(x << nb1);
     const uint32_t m2 = T.l1meta[i2];
-    const uint32_t k2 = (m2 >> 4) & 7u, nb2 = m2 & 15u;
+    const uint32_t k2 = (m2 >> 1) & 0x38u, nb2 = m2 & 15u;
     out.put(s1, k1);
     if (!k2) {
       pos += nb1;
@@ -561,7 +576,7 @@ __device__ bool decode_chunk(GroupSmem &G, const DecodeTables &T, const uint32_t
     const uint32_t k = decode_step<true>(T, peek(rel0 + pos), we - pos, syms, nb, bnd);
     if (!k) break;
     pos += nb;
-    out.put(syms, k);
+    out.put(syms, 8 * k);
   }
   out.finish();
   gsync(id);
