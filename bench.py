@@ -261,6 +261,78 @@ def measure_kv_pages(eh, synth, dev, stream, reps=20):
             "slot_bytes": 28 * 1024}
 
 
+def measure_prefetch(eh, xs, outs, p, dev, tokens, layers=8, depth=2, max_ctas=0, reps=3):
+    """Linear layers of `layers` Llama-3.1-8B blocks run on `tokens` rows of
+    activations (y = x @ W^T for q, k, v, o, gate, up, down; every layer reuses
+    the one compressed block).  Three ways, each timed with CUDA events on the
+    consumer stream (median of `reps`):
+      resident   the uncompressed weights stay in HBM;
+      serial     each block is decompressed, then its GEMMs run, one stream;
+      prefetch   the block for layer l+depth is decompressed on a decode
+                 stream into a ring slot while layers l..l+depth-1 compute.
+    The outputs of the last layer are checked equal across the three."""
+    import torch
+    cons = torch.cuda.current_stream()
+    torch.manual_seed(0)
+    shapes = [(x.numel() // (4096 if i < 6 else 14336), 4096 if i < 6 else 14336) for i, x in enumerate(xs)]
+    acts = [torch.randn(tokens, k, device=dev).to(torch.bfloat16) for _, k in shapes]
+    ws_res = [x.view(torch.bfloat16).view(r, k) for x, (r, k) in zip(xs, shapes)]
+    slot_bytes = sum((2 * x.numel() + 255) // 256 * 256 for x in xs)
+    pf = eh.Prefetcher(p, depth, slot_bytes, dev, max_ctas=max_ctas)
+    serial_buf = [torch.empty_like(x) for x in xs]
+    wsd = torch.empty(eh.decompress_workspace(p, len(xs)), dtype=torch.uint8, device=dev)
+
+    def gemms(ws):
+        return [a @ w.t() for a, w in zip(acts, ws)]
+
+    def run_resident():
+        for _ in range(layers):
+            ys = gemms(ws_res)
+        return ys
+
+    def run_serial():
+        for _ in range(layers):
+            eh.decompress_batch(p, outs, serial_buf, wsd)
+            ys = gemms([b.view(torch.bfloat16).view(r, k) for b, (r, k) in zip(serial_buf, shapes)])
+        return ys
+
+    def run_prefetch(start):
+        pf.stream.wait_event(start)
+        pending = [pf.submit(outs) for _ in range(min(depth, layers))]
+        for l in range(layers):
+            slot, views = pending.pop(0)
+            pf.acquire(slot, cons)
+            ys = gemms([v.view(torch.bfloat16).view(r, k) for v, (r, k) in zip(views, shapes)])
+            pf.release(slot, cons)
+            if l + depth < layers:
+                pending.append(pf.submit(outs))
+        return ys
+
+    times = {"resident": [], "serial": [], "prefetch": []}
+    results = {}
+    for rep in range(reps + 1):  # the first round warms up
+        for name in times:
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(cons)
+            ys = run_prefetch(e0) if name == "prefetch" else (run_serial() if name == "serial" else run_resident())
+            e1.record(cons)
+            torch.cuda.synchronize()
+            if rep:
+                times[name].append(e0.elapsed_time(e1))
+            results[name] = ys
+    for s in range(depth):
+        assert pf.status(s) == eh.EH_OK
+    same = all(torch.equal(a, b) and torch.equal(a, c)
+               for a, b, c in zip(results["resident"], results["serial"], results["prefetch"]))
+    pf.close()
+    med = {k: statistics.median(v) for k, v in times.items()}
+    return {"tokens": tokens, "layers": layers, "depth": depth, "decode_ctas": max_ctas or "all",
+            "resident_ms": med["resident"], "serial_ms": med["serial"], "prefetch_ms": med["prefetch"],
+            "prefetch_over_resident": med["prefetch"] / med["resident"],
+            "serial_over_resident": med["serial"] / med["resident"], "outputs_equal": same}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -387,6 +459,8 @@ def main():
     # FP4 block scale factors (NVFP4-style E4M3 scales, one per 16 values)
     fp4 = measure_fp4_scales(eh, synth, items, dev, stream)
     kv_pages = measure_kv_pages(eh, synth, dev, stream)
+    # decompression into the operand buffers of the next GEMMs (prefetch ring)
+    prefetch = [measure_prefetch(eh, xs, outs, p, dev, t) for t in (1, 8192)]
 
     if rank == 0:
         peak, peak_kind = hbm_peak()
@@ -426,6 +500,9 @@ def main():
             "gpu_launches": 6 * args.steps,
             "fp4_scales": fp4,
             "kv_pages": kv_pages,
+            "prefetch": {"workload": "8 layers of Llama-3.1-8B block linears (q,k,v,o,gate,up,down) "
+                                     "on `tokens` BF16 rows; weights decoded into a 2-slot ring",
+                         "runs": prefetch},
             "clocks": clk.summary(),
         }
         if world == 1 and not args.no_cpu_baseline:

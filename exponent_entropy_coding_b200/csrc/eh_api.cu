@@ -280,11 +280,10 @@ eh_status eh_decompress_workspace(const eh_plan_t *plan, int k, uint64_t *worksp
 
 }  // extern "C"
 
-namespace {
-
-eh_status decompress_impl(const eh_plan_t *plan, int k, const eh_compressed_t *cs, void *const *outs,
+// Shared by the decompression entry points and the prefetcher.
+eh_status eh::decompress_impl(const eh_plan_t *plan, int k, const eh_compressed_t *cs, void *const *outs,
                           const uint32_t *firsts, const uint32_t *counts, void *workspace,
-                          uint64_t workspace_bytes, void *stream) {
+                          uint64_t workspace_bytes, void *stream, uint32_t max_ctas) {
   if (!plan_ok(plan) || k < 1 || k > EH_MAX_BATCH || !cs || !outs || !workspace) return EH_ERR_INVALID_ARG;
   if (((uintptr_t)workspace & 255u) != 0) return EH_ERR_INVALID_ARG;
   if (workspace_bytes < kHeader + (uint64_t)k * kLutBytes) return EH_ERR_NOMEM;
@@ -335,30 +334,29 @@ eh_status decompress_impl(const eh_plan_t *plan, int k, const eh_compressed_t *c
   int num_sms = 0;
   if (device_setup(&num_sms) != cudaSuccess) return EH_ERR_CUDA;
   cudaStream_t s = (cudaStream_t)stream;
+  if (max_ctas && max_ctas < (uint32_t)num_sms) num_sms = (int)max_ctas;
   if (launch_tables(b, s) != cudaSuccess) return EH_ERR_CUDA;
   if (launch_decode(b, s, num_sms) != cudaSuccess) return EH_ERR_CUDA;
   return EH_OK;
 }
-
-}  // namespace
 
 extern "C" {
 
 eh_status eh_decompress(const eh_plan_t *plan, const eh_compressed_t *c, void *out, void *workspace,
                         uint64_t workspace_bytes, void *stream) {
   void *outs[1] = {out};
-  return decompress_impl(plan, 1, c, outs, nullptr, nullptr, workspace, workspace_bytes, stream);
+  return decompress_impl(plan, 1, c, outs, nullptr, nullptr, workspace, workspace_bytes, stream, 0);
 }
 
 eh_status eh_decompress_batch(const eh_plan_t *plan, int k, const eh_compressed_t *cs, void *const *outs,
                               void *workspace, uint64_t workspace_bytes, void *stream) {
-  return decompress_impl(plan, k, cs, outs, nullptr, nullptr, workspace, workspace_bytes, stream);
+  return decompress_impl(plan, k, cs, outs, nullptr, nullptr, workspace, workspace_bytes, stream, 0);
 }
 
 eh_status eh_decompress_chunks(const eh_plan_t *plan, const eh_compressed_t *c, uint32_t first, uint32_t count,
                                void *out, void *workspace, uint64_t workspace_bytes, void *stream) {
   void *outs[1] = {out};
-  return decompress_impl(plan, 1, c, outs, &first, &count, workspace, workspace_bytes, stream);
+  return decompress_impl(plan, 1, c, outs, &first, &count, workspace, workspace_bytes, stream, 0);
 }
 
 eh_status eh_codebook_from_counts(const eh_plan_t *plan, const uint64_t *counts, uint8_t *code_len, uint32_t *code,

@@ -149,4 +149,11 @@ cudaError_t launch_decode(const Batch &b, cudaStream_t s, int num_sms);
 cudaError_t configure_decode();  // once per device, before the first decode launch
 cudaError_t configure_encode();  // once per device, before the first encode launch
 
+// Validates a decompression call (k tensors, optional chunk ranges) and
+// launches the table and decode kernels on `stream`.  max_ctas caps the
+// decoder's grid (0: one CTA per SM), leaving SMs free for concurrent work.
+eh_status decompress_impl(const eh_plan_t *plan, int k, const eh_compressed_t *cs, void *const *outs,
+                          const uint32_t *firsts, const uint32_t *counts, void *workspace,
+                          uint64_t workspace_bytes, void *stream, uint32_t max_ctas);
+
 }  // namespace eh

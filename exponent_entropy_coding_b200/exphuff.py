@@ -34,7 +34,11 @@ EXPORTED = ["eh_plan", "eh_compress_bound", "eh_compress_batch_workspace", "eh_c
             "eh_decompress_workspace", "eh_decompress", "eh_decompress_batch",
             "eh_decompress_chunks", "eh_decompress_batch_noalloc", "eh_codebook_from_counts",
             "eh_pages_append", "eh_pages_read",
+            "eh_prefetch_workspace", "eh_prefetch_create", "eh_prefetch_submit",
+            "eh_prefetch_acquire", "eh_prefetch_release", "eh_prefetch_status",
+            "eh_prefetch_destroy",
             "eh_get_status", "eh_status_str", "eh_version"]
+EH_PREFETCH_MAX_DEPTH = 8
 EH_PAGE_RAW = 0x80000000
 
 
@@ -91,6 +95,13 @@ def lib():
             "eh_codebook_from_counts": [P(eh_plan_t), vp, vp, vp, vp, u64, vp],
             "eh_pages_append": [P(eh_plan_t), P(eh_page_store_t), vp, u32, vp, vp, u64, vp],
             "eh_pages_read": [P(eh_plan_t), P(eh_page_store_t), vp, u32, vp, vp, u64, vp],
+            "eh_prefetch_workspace": [P(eh_plan_t), C.c_int, P(u64)],
+            "eh_prefetch_create": [P(eh_plan_t), C.c_int, P(vp), u64, vp, u64, vp, u32, P(vp)],
+            "eh_prefetch_submit": [vp, C.c_int, P(eh_compressed_t), P(u64), P(C.c_int)],
+            "eh_prefetch_acquire": [vp, C.c_int, vp],
+            "eh_prefetch_release": [vp, C.c_int, vp],
+            "eh_prefetch_status": [vp, C.c_int],
+            "eh_prefetch_destroy": [vp],
             "eh_get_status": [vp, vp],
             "eh_status_str": [C.c_int],
             "eh_version": [],
@@ -427,3 +438,63 @@ class PageStore:
 
     def status(self, stream=None) -> int:
         return get_status(self.workspace, stream)
+
+
+class Prefetcher:
+    """Ring of `depth` decoded-operand slots (device memory owned by torch)
+    filled on a decode stream ahead of the consumer stream.  submit() enqueues
+    the decompression of a group of tensors (e.g. one transformer block) into
+    the next slot and returns (slot, views); acquire()/release() bracket the
+    consumer's use of a slot on the consumer stream."""
+
+    def __init__(self, p: eh_plan_t, depth: int, slot_bytes: int, device, decode_stream=None,
+                 max_ctas: int = 0):
+        dev = torch.device(device)
+        self.plan, self.depth = p, depth
+        self.slot_bytes = (slot_bytes + 255) // 256 * 256
+        self.slots = [torch.empty(self.slot_bytes, dtype=torch.uint8, device=dev) for _ in range(depth)]
+        wsb = C.c_uint64(0)
+        _check(lib().eh_prefetch_workspace(C.byref(p), depth, C.byref(wsb)), "eh_prefetch_workspace")
+        self.workspace = torch.empty(wsb.value, dtype=torch.uint8, device=dev)
+        self.stream = decode_stream if decode_stream is not None else torch.cuda.Stream(device=dev)
+        ptrs = (C.c_void_p * depth)(*[t.data_ptr() for t in self.slots])
+        h = C.c_void_p()
+        _check(lib().eh_prefetch_create(C.byref(p), depth, ptrs, self.slot_bytes,
+                                        C.c_void_p(self.workspace.data_ptr()), self.workspace.numel(),
+                                        C.c_void_p(self.stream.cuda_stream), max_ctas, C.byref(h)),
+               "eh_prefetch_create")
+        self._h = h
+        self._keep = [None] * depth  # the compressed inputs of each slot's decode, alive until reuse
+
+    def submit(self, cs: List[Compressed]):
+        k = len(cs)
+        structs = (eh_compressed_t * k)(*[c.struct() for c in cs])
+        offs = (C.c_uint64 * k)()
+        slot = C.c_int(-1)
+        _check(lib().eh_prefetch_submit(self._h, k, structs, offs, C.byref(slot)), "eh_prefetch_submit")
+        s = slot.value
+        self._keep[s] = list(cs)
+        et = _elem_dtype(self.plan.dtype)
+        size = 2 if self.plan.dtype == EH_BF16 else 1
+        views = [self.slots[s][offs[i]:offs[i] + c.n * size].view(et) for i, c in enumerate(cs)]
+        return s, views
+
+    def acquire(self, slot: int, stream=None):
+        _check(lib().eh_prefetch_acquire(self._h, slot, _stream_ptr(stream)), "eh_prefetch_acquire")
+
+    def release(self, slot: int, stream=None):
+        _check(lib().eh_prefetch_release(self._h, slot, _stream_ptr(stream)), "eh_prefetch_release")
+
+    def status(self, slot: int) -> int:
+        return lib().eh_prefetch_status(self._h, slot)
+
+    def close(self):
+        if self._h:
+            lib().eh_prefetch_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

@@ -266,6 +266,68 @@ EH_API eh_status eh_pages_read(const eh_plan_t *plan, const eh_page_store_t *sto
                                const uint32_t *slot_ids, uint32_t n_pages, void *out,
                                void *workspace, uint64_t workspace_bytes, void *stream);
 
+/* ---- Prefetcher: decompression straight into the operand buffers of the
+ * next consumer (a GEMM), on a decode stream that runs ahead of the consumer
+ * stream.  The DFloat11 article ("方法介绍") decompresses a whole transformer
+ * block just before the block runs; the tile-level ANS paper summary (the
+ * Lattice page, abstract) aligns decoding with the inference GEMMs.  Here a
+ * ring of `depth` caller-owned slots holds decoded blocks: the decode of
+ * block i+depth overlaps the consumer's work on blocks i..i+depth-1, and
+ * CUDA events order the two streams, so nothing waits on the host.
+ *
+ * Use (one host thread per prefetcher):
+ *   submit(b0) ... submit(b{depth-1})            fill the ring
+ *   for each block i: acquire(slot_i, s)          s waits for the decode
+ *                     <consumer work on s>        reads the slot
+ *                     release(slot_i, s)          slot reusable after that work
+ *                     submit(b{i+depth})          decode waits for the release
+ * Slots are used round-robin.  submit() fails with EH_ERR_INVALID_ARG (and
+ * does nothing) when its slot has not been released since its last submit;
+ * acquire() needs a submitted slot and release() an acquired one. */
+#define EH_PREFETCH_MAX_DEPTH 8
+typedef struct eh_prefetch eh_prefetch;
+
+/* Device workspace for a prefetcher of `depth` slots (1..EH_PREFETCH_MAX_DEPTH):
+ * one decompression workspace of EH_MAX_BATCH tensors per slot. */
+EH_API eh_status eh_prefetch_workspace(const eh_plan_t *plan, int depth,
+                                       uint64_t *workspace_bytes);
+
+/* Creates a prefetcher.  slots[depth]: device buffers of slot_bytes bytes
+ * each, 256-byte aligned, owned by the caller; workspace: device, 256-byte
+ * aligned, eh_prefetch_workspace() bytes, owned by the caller;
+ * decode_stream: the stream the decodes run on (not the consumer's).
+ * max_ctas caps the decoder's grid (0: one CTA per SM) so that a consumer
+ * running at the same time keeps the other SMs.  The handle (host memory and
+ * 2*depth CUDA events) is freed by eh_prefetch_destroy. */
+EH_API eh_status eh_prefetch_create(const eh_plan_t *plan, int depth,
+                                    void *const *slots, uint64_t slot_bytes,
+                                    void *workspace, uint64_t workspace_bytes,
+                                    void *decode_stream, uint32_t max_ctas,
+                                    eh_prefetch **out);
+
+/* Enqueues the decompression of k (1..EH_MAX_BATCH) tensors into the next
+ * slot, after the consumer work released from that slot.  Tensor i lands at
+ * byte offsets[i] of the slot (host array of k entries, filled here): each
+ * tensor starts on a 256-byte boundary after the previous one.  *slot
+ * receives the slot index.  EH_ERR_NOMEM when the tensors do not fit. */
+EH_API eh_status eh_prefetch_submit(eh_prefetch *pf, int k, const eh_compressed_t *cs,
+                                    uint64_t *offsets, int *slot);
+
+/* Makes consumer_stream wait (on the GPU) for the slot's decode. */
+EH_API eh_status eh_prefetch_acquire(eh_prefetch *pf, int slot, void *consumer_stream);
+
+/* Marks the slot reusable once the work enqueued so far on consumer_stream
+ * has run. */
+EH_API eh_status eh_prefetch_release(eh_prefetch *pf, int slot, void *consumer_stream);
+
+/* Waits for the slot's last decode and returns its status word (EH_OK or a
+ * data error, as eh_get_status). */
+EH_API eh_status eh_prefetch_status(eh_prefetch *pf, int slot);
+
+/* Waits for the decode stream, destroys the events and frees the handle.
+ * NULL is accepted. */
+EH_API eh_status eh_prefetch_destroy(eh_prefetch *pf);
+
 /* Waits for `stream` and returns the status word of `workspace`: EH_OK,
  * EH_ERR_CORRUPT, EH_ERR_INFEASIBLE, EH_ERR_NOMEM or EH_ERR_TIMEOUT.  Every compress or
  * decompress call resets the word when it starts, so it describes the most
