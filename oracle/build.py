@@ -11,14 +11,14 @@ LIB = os.path.join(HERE, "libehref.so")
 
 
 def build(force: bool = False) -> str:
-    src = os.path.join(HERE, "ehref.cpp")
-    hdr = os.path.join(HERE, "ehref.h")
+    srcs = [os.path.join(HERE, f) for f in ("ehref.cpp", "zfref.cpp")]
+    deps = srcs + [os.path.join(HERE, f) for f in ("ehref.h", "zfref.h")]
     if (not force and os.path.exists(LIB)
-            and os.path.getmtime(LIB) >= max(os.path.getmtime(src), os.path.getmtime(hdr))):
+            and os.path.getmtime(LIB) >= max(os.path.getmtime(f) for f in deps)):
         return LIB
     tmp = LIB + ".tmp"
     cmd = ["g++", "-std=c++17", "-O2", "-fPIC", "-shared", "-Wall", "-Wextra",
-           "-o", tmp, src]
+           "-o", tmp, *srcs]
     subprocess.run(cmd, check=True)
     os.replace(tmp, LIB)
     return LIB

@@ -52,6 +52,10 @@ def lib():
             "ehref_decompress": (i32, [i32, u64, u32, vp, vp, vp, vp, u64, vp, vp]),
             "ehref_page_encode": (i32, [i32, vp, u64, vp, vp, vp, u64, vp, vp, vp, vp]),
             "ehref_page_decode": (i32, [i32, u64, vp, vp, vp, u64, u64, i32, vp, vp, vp]),
+            "zfref_blocks": (u64, [u64]),
+            "zfref_block_base": (i32, [vp, u32, vp, vp]),
+            "zfref_compress": (i32, [vp, u64, vp, vp, vp, vp, vp, u64, vp]),
+            "zfref_decompress": (i32, [u64, vp, vp, vp, vp, vp, u64, vp]),
         }
         for name, (res, args) in sig.items():
             f = getattr(_lib, name)
@@ -240,3 +244,57 @@ def page_decode(dtype, n, lengths, codes, page: Page):
                                    _p(np.ascontiguousarray(page.raw_exps, np.uint8)),
                                    _p(np.ascontiguousarray(page.sign_mant, np.uint8)), _p(out)))
     return out[:n]
+
+
+# ---- ZipFloat comparison codec (BF16 only; format in zfref.h)
+ZF_BLOCK = 2048
+
+
+@dataclass
+class ZfCompressed:
+    n: int
+    sign_mant: np.ndarray   # uint8[n]
+    meta: np.ndarray        # uint32[B]: l_b | records << 8
+    dense: np.ndarray       # uint32[B*192]: 3 bit planes of 64 words per block
+    sparse_off: np.ndarray  # uint32[B]
+    sparse: np.ndarray      # uint16[records]
+
+    def nbytes(self):
+        return self.sign_mant.size + 4 * self.meta.size + 4 * self.dense.size + 4 * self.sparse_off.size + \
+            2 * self.sparse.size
+
+
+def zf_blocks(n):
+    return lib().zfref_blocks(n)
+
+
+def zf_block_base(x):
+    x = np.ascontiguousarray(x, np.uint16)
+    md, lb = C.c_uint32(0), C.c_uint32(0)
+    _check(lib().zfref_block_base(_p(x), x.size, C.byref(md), C.byref(lb)))
+    return md.value, lb.value
+
+
+def zf_compress(x):
+    x = np.ascontiguousarray(x, np.uint16)
+    n = x.size
+    B = zf_blocks(n)
+    sm = np.zeros(max(n, 1), np.uint8)
+    meta = np.zeros(max(B, 1), np.uint32)
+    dense = np.zeros(max(B * 192, 1), np.uint32)
+    off = np.zeros(max(B, 1), np.uint32)
+    sparse = np.zeros(max(n, 1), np.uint16)
+    nrec = C.c_uint64(0)
+    _check(lib().zfref_compress(_p(x), n, _p(sm), _p(meta), _p(dense), _p(off), _p(sparse), n, C.byref(nrec)))
+    return ZfCompressed(n, sm[:n], meta[:B], dense[:B * 192], off[:B], sparse[:nrec.value].copy())
+
+
+def zf_decompress(c: ZfCompressed):
+    out = np.zeros(max(c.n, 1), np.uint16)
+    sp = np.ascontiguousarray(c.sparse, np.uint16)
+    _check(lib().zfref_decompress(c.n, _p(np.ascontiguousarray(c.sign_mant, np.uint8)),
+                                  _p(np.ascontiguousarray(c.meta, np.uint32)),
+                                  _p(np.ascontiguousarray(c.dense, np.uint32)),
+                                  _p(np.ascontiguousarray(c.sparse_off, np.uint32)),
+                                  _p(sp) if sp.size else None, sp.size, _p(out)))
+    return out[:c.n]
