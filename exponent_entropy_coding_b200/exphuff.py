@@ -37,6 +37,7 @@ EXPORTED = ["eh_plan", "eh_compress_bound", "eh_compress_batch_workspace", "eh_c
             "eh_prefetch_workspace", "eh_prefetch_create", "eh_prefetch_submit",
             "eh_prefetch_acquire", "eh_prefetch_release", "eh_prefetch_status",
             "eh_prefetch_destroy",
+            "eh_zf_bound", "eh_zf_compress", "eh_zf_decompress",
             "eh_get_status", "eh_status_str", "eh_version"]
 EH_PREFETCH_MAX_DEPTH = 8
 EH_PAGE_RAW = 0x80000000
@@ -58,6 +59,12 @@ class eh_compressed_t(C.Structure):
                 ("code_len", C.c_void_p), ("code", C.c_void_p), ("chunk_bit_off", C.c_void_p),
                 ("exp_stream", C.c_void_p), ("exp_stream_cap", C.c_uint64),
                 ("sign_mant", C.c_void_p), ("exp_stream_bits", C.c_uint64)]
+
+
+class eh_zf_t(C.Structure):
+    _fields_ = [("n", C.c_uint64), ("sign_mant", C.c_void_p), ("meta", C.c_void_p), ("dense", C.c_void_p),
+                ("sparse_off", C.c_void_p), ("sparse", C.c_void_p), ("sparse_cap", C.c_uint64),
+                ("n_records", C.c_uint64)]
 
 
 class eh_page_store_t(C.Structure):
@@ -102,6 +109,9 @@ def lib():
             "eh_prefetch_release": [vp, C.c_int, vp],
             "eh_prefetch_status": [vp, C.c_int],
             "eh_prefetch_destroy": [vp],
+            "eh_zf_bound": [u64, P(u64), P(u64)],
+            "eh_zf_compress": [vp, P(eh_zf_t), vp, u64, C.c_int, vp],
+            "eh_zf_decompress": [P(eh_zf_t), vp, vp, u64, vp],
             "eh_get_status": [vp, vp],
             "eh_status_str": [C.c_int],
             "eh_version": [],
@@ -498,3 +508,64 @@ class Prefetcher:
             self.close()
         except Exception:
             pass
+
+
+class ZfCompressed:
+    """ZipFloat comparison codec buffers (device, owned by torch)."""
+
+    def __init__(self, n: int, device):
+        blocks, cap = C.c_uint64(0), C.c_uint64(0)
+        _check(lib().eh_zf_bound(n, C.byref(blocks), C.byref(cap)), "eh_zf_bound")
+        dev = torch.device(device)
+        B = blocks.value
+        self.n = n
+        self.sign_mant = torch.empty(max(n, 16), dtype=torch.uint8, device=dev)
+        self.meta = torch.empty(max(B, 1), dtype=torch.int32, device=dev)
+        self.dense = torch.empty(max(B * 192, 4), dtype=torch.int32, device=dev)
+        self.sparse_off = torch.empty(max(B, 1), dtype=torch.int32, device=dev)
+        self.sparse = torch.empty(max(cap.value, 1), dtype=torch.int16, device=dev)
+        self.workspace = torch.empty(256, dtype=torch.uint8, device=dev)
+        self.blocks = B
+        self.n_records = 0
+        self._s = eh_zf_t()
+
+    def struct(self) -> eh_zf_t:
+        s = self._s
+        s.n = self.n
+        s.sign_mant = self.sign_mant.data_ptr()
+        s.meta = self.meta.data_ptr()
+        s.dense = self.dense.data_ptr()
+        s.sparse_off = self.sparse_off.data_ptr()
+        s.sparse = self.sparse.data_ptr()
+        s.sparse_cap = self.sparse.numel()
+        s.n_records = self.n_records
+        return s
+
+    def compressed_bytes(self) -> int:
+        return self.n + 8 * self.blocks + 768 * self.blocks + 2 * self.n_records
+
+
+def zf_compress(x: torch.Tensor, out: Optional[ZfCompressed] = None, wait: bool = True, stream=None) -> ZfCompressed:
+    x = _raw(x)
+    if out is None:
+        out = ZfCompressed(x.numel(), x.device)
+    st = out.struct()
+    rc = lib().eh_zf_compress(C.c_void_p(x.data_ptr()), C.byref(st), C.c_void_p(out.workspace.data_ptr()),
+                              out.workspace.numel(), int(wait), _stream_ptr(stream))
+    _check(rc, "eh_zf_compress")
+    if wait:
+        out.n_records = st.n_records
+    return out
+
+
+def zf_decompress(c: ZfCompressed, out: Optional[torch.Tensor] = None, stream=None,
+                  check: bool = True) -> torch.Tensor:
+    if out is None:
+        out = torch.empty(c.n, dtype=torch.int16, device=c.sign_mant.device)
+    st = c.struct()
+    rc = lib().eh_zf_decompress(C.byref(st), C.c_void_p(out.data_ptr()), C.c_void_p(c.workspace.data_ptr()),
+                                c.workspace.numel(), _stream_ptr(stream))
+    _check(rc, "eh_zf_decompress")
+    if check:
+        _check(get_status(c.workspace, stream), "eh_zf_decompress (device status)")
+    return out

@@ -328,6 +328,48 @@ EH_API eh_status eh_prefetch_status(eh_prefetch *pf, int slot);
  * NULL is accepted. */
 EH_API eh_status eh_prefetch_destroy(eh_prefetch *pf);
 
+/* ---- ZipFloat comparison codec (BF16 only).  A different codec, kept beside
+ * the Huffman format as a point of comparison for ratio and speed on the same
+ * inputs.  "ZipFloat: An Ultra-fast and Lossless Floating-Point Compressor for
+ * LLM Inference Systems": blocks of 2048 values (§3.1); per block the most
+ * frequent exponent MD, l_b = (MD - 6) mod 256 and r = (e - l_b) mod 256
+ * (§3.2, Eq. 4; ties in MD go to the smaller field); the low three bits of r
+ * as three bit planes of 64 words per block (bit i of word w of plane p = bit
+ * p of r of element 32w+i), and for r >= 8 a record (i << 5) | (r >> 3) with
+ * i the index in the block (§3.3); sign/mantissa bytes (s << 7) | m7.
+ * Each block's records are contiguous, in element order, at sparse_off[b];
+ * the blocks' ranges are reserved with an atomic, so their order in `sparse`
+ * depends on scheduling.  All arrays are device memory owned by the caller;
+ * sign_mant and dense 16-byte aligned; n < 2^32. */
+typedef struct {
+  uint64_t n;            /* values                                          */
+  uint8_t *sign_mant;    /* n bytes                                         */
+  uint32_t *meta;        /* per block: l_b | (records of the block) << 8    */
+  uint32_t *dense;       /* per block 3 planes x 64 words                   */
+  uint32_t *sparse_off;  /* per block: index of its first record            */
+  uint16_t *sparse;      /* sparse_cap records                              */
+  uint64_t sparse_cap;   /* records the buffer holds (n always suffices)    */
+  uint64_t n_records;    /* out: records written (when compress waits)      */
+} eh_zf_t;
+
+/* blocks = ceil(n / 2048) (length of meta and sparse_off; dense holds
+ * 192 * blocks words); sparse_cap = n, which no input exceeds. */
+EH_API eh_status eh_zf_bound(uint64_t n, uint64_t *blocks, uint64_t *sparse_cap);
+
+/* Compresses n = out->n BF16 values from `in` (device, 16-byte aligned).
+ * workspace: device, >= 256 bytes, 256-byte aligned (status word and the
+ * record counter).  wait != 0: waits for the stream, fills out->n_records and
+ * returns EH_ERR_NOMEM if the records overflowed sparse_cap.  Otherwise
+ * fully stream-ordered (eh_get_status reports the overflow). */
+EH_API eh_status eh_zf_compress(const void *in, eh_zf_t *out, void *workspace,
+                                uint64_t workspace_bytes, int wait, void *stream);
+
+/* Rebuilds the n values into out (device, 16-byte aligned).  Stream-ordered;
+ * a block whose record range or indices are out of bounds is skipped and
+ * sets EH_ERR_CORRUPT in the workspace's status word. */
+EH_API eh_status eh_zf_decompress(const eh_zf_t *c, void *out, void *workspace,
+                                  uint64_t workspace_bytes, void *stream);
+
 /* Waits for `stream` and returns the status word of `workspace`: EH_OK,
  * EH_ERR_CORRUPT, EH_ERR_INFEASIBLE, EH_ERR_NOMEM or EH_ERR_TIMEOUT.  Every compress or
  * decompress call resets the word when it starts, so it describes the most

@@ -99,3 +99,11 @@ def test_lm_head(eh, oracle):
 def test_fp4_block_scales(eh, oracle, name):
     outs = _run(eh, oracle, name)
     assert len(outs) == 7
+
+
+def test_zipfloat_comparison_codec_on_the_block(eh, oracle):
+    """The ZipFloat comparison codec over the whole block, byte parity per
+    block against the oracle (record ranges compared through their offsets)."""
+    from test_gpu_zipfloat import check_parity
+    for _, x in synth.llama8b_block():
+        check_parity(eh, oracle, x)
