@@ -261,6 +261,36 @@ def measure_kv_pages(eh, synth, dev, stream, reps=20):
             "slot_bytes": 28 * 1024}
 
 
+def measure_zipfloat(eh, xs, dev, stream, reps=20):
+    """The ZipFloat comparison codec on the same block (seven calls each way
+    per repetition, CUDA events): GB/s of BF16 bytes and the size ratio."""
+    import torch
+    cs = [eh.zf_compress(x) for x in xs]
+    ys = [torch.empty_like(x) for x in xs]
+    for c, x, y in zip(cs, xs, ys):
+        eh.zf_decompress(c, out=y)
+        assert torch.equal(x, y)
+    nbytes = sum(2 * x.numel() for x in xs)
+    comp = sum(c.compressed_bytes() for c in cs)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+    ev[0].record(stream)
+    for _ in range(reps):
+        for c, x in zip(cs, xs):
+            eh.zf_compress(x, out=c, wait=False)
+    ev[1].record(stream)
+    for _ in range(reps):
+        for c, y in zip(cs, ys):
+            eh.zf_decompress(c, out=y, check=False)
+    ev[2].record(stream)
+    torch.cuda.synchronize()
+    enc = ev[0].elapsed_time(ev[1]) / reps
+    dec = ev[1].elapsed_time(ev[2]) / reps
+    return {"kind": "ZipFloat comparison codec (blocks of 2048, l_b = MD - 6, 3 bit planes, 16-bit records)",
+            "encode_gbs": nbytes / (enc * 1e-3) / 1e9, "decode_gbs": nbytes / (dec * 1e-3) / 1e9,
+            "size_ratio": comp / nbytes,
+            "records_per_value": sum(c.n_records for c in cs) / (nbytes / 2)}
+
+
 def measure_prefetch(eh, xs, outs, p, dev, tokens, layers=8, depth=2, max_ctas=0, reps=3):
     """Linear layers of `layers` Llama-3.1-8B blocks run on `tokens` rows of
     activations (y = x @ W^T for q, k, v, o, gate, up, down; every layer reuses
@@ -461,6 +491,7 @@ def main():
     kv_pages = measure_kv_pages(eh, synth, dev, stream)
     # decompression into the operand buffers of the next GEMMs (prefetch ring)
     prefetch = [measure_prefetch(eh, xs, outs, p, dev, t) for t in (1, 8192)]
+    zipfloat = measure_zipfloat(eh, xs, dev, stream)
 
     if rank == 0:
         peak, peak_kind = hbm_peak()
@@ -500,6 +531,7 @@ def main():
             "gpu_launches": 6 * args.steps,
             "fp4_scales": fp4,
             "kv_pages": kv_pages,
+            "zipfloat": zipfloat,
             "prefetch": {"workload": "8 layers of Llama-3.1-8B block linears (q,k,v,o,gate,up,down) "
                                      "on `tokens` BF16 rows; weights decoded into a 2-slot ring",
                          "runs": prefetch},

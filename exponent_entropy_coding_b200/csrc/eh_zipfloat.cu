@@ -11,10 +11,12 @@
 // blocks' record ranges depends on scheduling; everything else is
 // deterministic.
 //
-// One CTA of 256 threads per block, eight values per thread: the thread's
-// eight bits of each plane form one byte of that plane (bit j = element
-// 8*tid + j), so the planes are assembled in shared memory byte by byte and
-// written with 16-byte stores.
+// One warp per block (the page's §3.3: a warp works on 32 rows of the bit
+// matrix at a time), eight blocks per CTA of 256 threads.  The block is read
+// as eight 256-value slices; in slice c lane l holds values 256c + 8l .. +7,
+// so every load and store of a slice is a coalesced 16 bytes per lane, and
+// the lane's eight bits of a plane are byte 32c + l of that plane.  Nothing
+// but the records' reservation (one atomic per CTA) is shared between warps.
 #include <cstring>
 
 #include "eh_internal.cuh"
@@ -23,13 +25,16 @@ namespace eh {
 namespace {
 
 constexpr uint32_t kZfBlock = 2048;
-constexpr uint32_t kZfThreads = 256;
-constexpr uint32_t kZfPlaneWords = 64;  // 2048 bits
+constexpr uint32_t kZfWarps = 8;              // blocks per CTA
+constexpr uint32_t kZfThreads = 32 * kZfWarps;
+constexpr uint32_t kZfPlaneBytes = kZfBlock / 8;  // 256
+constexpr uint32_t kZfSlices = kZfBlock / 256;    // 8
 
 struct ZfArgs {
   const uint16_t *in;
   uint16_t *out;
   uint64_t n;
+  uint64_t blocks;
   uint8_t *sm;
   uint32_t *meta;
   uint32_t *dense;
@@ -40,193 +45,210 @@ struct ZfArgs {
   uint32_t *counter;  // workspace word 2: records reserved so far
 };
 
-__device__ __forceinline__ uint32_t block_excl_scan256(uint32_t v, uint32_t *wsum, uint32_t *total) {
-  const uint32_t lane = threadIdx.x & 31u, warp = threadIdx.x >> 5;
-  uint32_t x = v;
-  #pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
-    if (lane >= (uint32_t)o) x += y;
-  }
-  if (lane == 31) wsum[warp] = x;
-  __syncthreads();
-  if (warp == 0) {
-    uint32_t t = lane < kZfThreads / 32 ? wsum[lane] : 0u;
-    #pragma unroll
-    for (int o = 1; o < 8; o <<= 1) {
-      const uint32_t y = __shfl_up_sync(0xffffffffu, t, o);
-      if (lane >= (uint32_t)o) t += y;
-    }
-    if (lane < kZfThreads / 32) wsum[lane] = t;
-  }
-  __syncthreads();
-  *total = wsum[kZfThreads / 32 - 1];
-  return (warp ? wsum[warp - 1] : 0u) + x - v;
+// the eight values [i, i+8) of the tensor as four words (zero past n)
+__device__ __forceinline__ uint4 load8(const uint16_t *in, uint64_t i, uint64_t n) {
+  if (i + 8 <= n) return __ldg((const uint4 *)(in + i));
+  uint32_t w[4] = {0, 0, 0, 0};
+  for (int j = 0; j < 8; j++)
+    if (i + j < n) w[j / 2] |= (uint32_t)in[i + j] << (16 * (j & 1));
+  return make_uint4(w[0], w[1], w[2], w[3]);
 }
 
-__global__ void __launch_bounds__(kZfThreads) zf_compress_kernel(const __grid_constant__ ZfArgs a) {
-  __shared__ uint32_t hist[256];
-  __shared__ alignas(16) uint8_t planes[3 * kZfThreads];
-  __shared__ uint32_t wsum[kZfThreads / 32];
-  __shared__ uint32_t s_lb, s_base;
-  const uint32_t tid = threadIdx.x, lane = tid & 31u;
-  const uint64_t i0 = (uint64_t)blockIdx.x * kZfBlock;
-  const uint32_t count = (uint32_t)min((uint64_t)kZfBlock, a.n - i0);
-  const uint32_t j0 = 8 * tid;  // first element of this thread in the block
+__device__ __forceinline__ uint32_t half_of(const uint4 &q, int j) {
+  const uint32_t w = j < 2 ? q.x : j < 4 ? q.y : j < 6 ? q.z : q.w;
+  return (w >> (16 * (j & 1))) & 0xFFFFu;
+}
 
-  hist[tid] = 0;
-  uint16_t v[8];
-  if (j0 + 8 <= count) {
-    const uint4 q = __ldg((const uint4 *)(a.in + i0 + j0));
-    const uint32_t w[4] = {q.x, q.y, q.z, q.w};
-    #pragma unroll
-    for (int j = 0; j < 8; j++) v[j] = (uint16_t)(w[j / 2] >> (16 * (j & 1)));
-  } else {
-    #pragma unroll
-    for (int j = 0; j < 8; j++) v[j] = j0 + j < count ? a.in[i0 + j0 + j] : (uint16_t)0;
-  }
-  __syncthreads();
-
-  // §3.2: MD, the most frequent exponent field of the block.  Lanes holding
-  // the same field add once (warp-aggregated); lanes past the end get a key
-  // no field has.
+__global__ void __launch_bounds__(kZfThreads, 4) zf_compress_kernel(const __grid_constant__ ZfArgs a) {
+  __shared__ uint32_t hist[kZfWarps][256];
+  __shared__ __align__(16) uint8_t planes[kZfWarps][3 * kZfPlaneBytes];
+  __shared__ uint16_t recs[kZfWarps][kZfBlock];
+  __shared__ uint32_t s_nnz[kZfWarps], s_base[kZfWarps];
+  const uint32_t lane = threadIdx.x & 31u, warp = threadIdx.x >> 5;
+  const uint64_t blk = (uint64_t)blockIdx.x * kZfWarps + warp;
+  const bool live = blk < a.blocks;
+  const uint64_t i0 = blk * kZfBlock;
+  const uint32_t count = live ? (uint32_t)min((uint64_t)kZfBlock, a.n - i0) : 0u;
+  // the whole block in registers: all eight loads in flight at once
+  uint4 q[kZfSlices];
   #pragma unroll
-  for (int j = 0; j < 8; j++) {
-    const bool ok = j0 + j < count;
-    const uint32_t key = ok ? (v[j] >> 7) & 0xFFu : 256u + lane;
-    const uint32_t same = __match_any_sync(0xffffffffu, key);
-    if (ok && lane == (uint32_t)(__ffs(same) - 1)) atomicAdd(&hist[key], (uint32_t)__popc(same));
-  }
-  __syncthreads();
-  if (tid < 32) {
-    // (count << 8) | (255 - field): the maximum is the most frequent field,
-    // the smaller field on ties
-    uint32_t best = 0;
-    #pragma unroll
-    for (int k = 0; k < 8; k++) {
-      const uint32_t e = tid * 8 + k;
-      best = max(best, (hist[e] << 8) | (255u - e));
-    }
-    best = __reduce_max_sync(0xffffffffu, best);
-    if (tid == 0) s_lb = ((255u - (best & 0xFFu)) + 256u - 6u) & 0xFFu;  // l_b = MD - 6
-  }
-  __syncthreads();
-  const uint32_t lb = s_lb;
-
-  // Eq. 4 remap; the low three bits into the planes, high parts counted
-  uint32_t pb0 = 0, pb1 = 0, pb2 = 0, hi_mask = 0;
-  uint8_t r[8];
+  for (uint32_t c = 0; c < kZfSlices; c++) q[c] = load8(a.in, i0 + 256 * c + 8 * lane, i0 + count);
+  uint32_t *h = hist[warp];
   #pragma unroll
-  for (int j = 0; j < 8; j++) {
-    const uint32_t rj = j0 + j < count ? (((v[j] >> 7) & 0xFFu) + 256u - lb) & 0xFFu : 0u;
-    r[j] = (uint8_t)rj;
-    pb0 |= (rj & 1u) << j;
-    pb1 |= ((rj >> 1) & 1u) << j;
-    pb2 |= ((rj >> 2) & 1u) << j;
-    hi_mask |= (rj >= 8u ? 1u : 0u) << j;
-  }
-  planes[tid] = (uint8_t)pb0;
-  planes[kZfThreads + tid] = (uint8_t)pb1;
-  planes[2 * kZfThreads + tid] = (uint8_t)pb2;
+  for (int k = 0; k < 8; k++) h[lane + 32 * k] = 0;
+  __syncwarp();
 
-  uint32_t nnz;
-  const uint32_t pos = block_excl_scan256((uint32_t)__popc(hi_mask), wsum, &nnz);
-  if (tid == 0) {
-    const uint32_t base = nnz ? atomicAdd(a.counter, nnz) : 0u;
-    s_base = base;
-    a.meta[blockIdx.x] = lb | (nnz << 8);
-    a.sparse_off[blockIdx.x] = base;
-    if ((uint64_t)base + nnz > a.sparse_cap) set_status(a.status, kFlagNoRoom);
-  }
-  __syncthreads();  // planes complete, base known
-  if (tid < 3 * kZfThreads / 16) {
-    const uint32_t p = tid / (kZfThreads / 16), q = tid % (kZfThreads / 16);
-    *(uint4 *)(a.dense + (uint64_t)blockIdx.x * 3 * kZfPlaneWords + p * kZfPlaneWords + 4 * q) =
-        *(const uint4 *)(planes + p * kZfThreads + 16 * q);
-  }
-  const uint64_t base = s_base;
-  if (base + nnz <= a.sparse_cap) {
-    uint32_t k = pos;
+  // §3.2: MD, the most frequent exponent field of the block
+  #pragma unroll
+  for (uint32_t c = 0; c < kZfSlices; c++) {
+    const uint32_t j0 = 256 * c + 8 * lane;
     #pragma unroll
     for (int j = 0; j < 8; j++)
-      if ((hi_mask >> j) & 1u) a.sparse[base + k++] = (uint16_t)(((j0 + j) << 5) | (r[j] >> 3));
+      if (j0 + j < count) atomicAdd(&h[(half_of(q[c], j) >> 7) & 0xFFu], 1u);
   }
-  // raw sign and mantissa
-  if (j0 + 8 <= count) {
-    uint32_t lo = 0, hi = 0;
+  __syncwarp();
+  // (count << 8) | (255 - field): the maximum is the most frequent field, the
+  // smaller field on ties; l_b = MD - 6
+  uint32_t best = 0;
+  #pragma unroll
+  for (int k = 0; k < 8; k++) best = max(best, (h[8 * lane + k] << 8) | (255u - (8 * lane + k)));
+  best = __reduce_max_sync(0xffffffffu, best);
+  const uint32_t lb = ((255u - (best & 0xFFu)) + 256u - 6u) & 0xFFu;
+
+  // Eq. 4 remap: plane bytes, raw sign/mantissa bytes, and the records,
+  // staged in shared memory in element order until the block's place in
+  // `sparse` is known
+  uint16_t *rec = recs[warp];
+  uint32_t nnz = 0;
+  #pragma unroll
+  for (uint32_t c = 0; c < kZfSlices; c++) {
+    const uint32_t j0 = 256 * c + 8 * lane;
+    uint16_t v[8];
+    #pragma unroll
+    for (int j = 0; j < 8; j++) v[j] = (uint16_t)half_of(q[c], j);
+    uint32_t pb0 = 0, pb1 = 0, pb2 = 0, hm = 0, lo = 0, hi = 0;
     #pragma unroll
     for (int j = 0; j < 8; j++) {
-      const uint32_t s = ((v[j] >> 8) & 0x80u) | (v[j] & 0x7Fu);
-      if (j < 4) lo |= s << (8 * j);
-      else hi |= s << (8 * (j - 4));
+      const uint32_t rj = j0 + j < count ? (((v[j] >> 7) & 0xFFu) + 256u - lb) & 0xFFu : 0u;
+      pb0 |= (rj & 1u) << j;
+      pb1 |= ((rj >> 1) & 1u) << j;
+      pb2 |= ((rj >> 2) & 1u) << j;
+      hm |= (rj >= 8u ? 1u : 0u) << j;
+      const uint32_t sv = ((v[j] >> 8) & 0x80u) | (v[j] & 0x7Fu);
+      if (j < 4) lo |= sv << (8 * j);
+      else hi |= sv << (8 * (j - 4));
     }
-    *(uint2 *)(a.sm + i0 + j0) = make_uint2(lo, hi);
-  } else {
-    for (int j = 0; j < 8; j++)
-      if (j0 + j < count) a.sm[i0 + j0 + j] = (uint8_t)(((v[j] >> 8) & 0x80u) | (v[j] & 0x7Fu));
+    planes[warp][32 * c + lane] = (uint8_t)pb0;
+    planes[warp][kZfPlaneBytes + 32 * c + lane] = (uint8_t)pb1;
+    planes[warp][2 * kZfPlaneBytes + 32 * c + lane] = (uint8_t)pb2;
+    if (j0 + 8 <= count) {
+      *(uint2 *)(a.sm + i0 + j0) = make_uint2(lo, hi);
+    } else {
+      for (int j = 0; j < 8; j++)
+        if (j0 + j < count) a.sm[i0 + j0 + j] = (uint8_t)(((v[j] >> 8) & 0x80u) | (v[j] & 0x7Fu));
+    }
+    const uint32_t mine = (uint32_t)__popc(hm);
+    uint32_t x = mine;
+    #pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= (uint32_t)o) x += y;
+    }
+    if (hm) {
+      uint32_t k = nnz + x - mine;
+      #pragma unroll
+      for (int j = 0; j < 8; j++) {
+        if ((hm >> j) & 1u) {
+          const uint32_t rj = (((v[j] >> 7) & 0xFFu) + 256u - lb) & 0xFFu;
+          rec[k++] = (uint16_t)(((j0 + j) << 5) | (rj >> 3));
+        }
+      }
+    }
+    nnz += __shfl_sync(0xffffffffu, x, 31);
   }
+  __syncwarp();
+  // the planes: 768 bytes as 48 16-byte stores
+  if (live) {
+    for (uint32_t t = lane; t < 3 * kZfPlaneBytes / 16; t += 32)
+      *(uint4 *)(a.dense + blk * 192 + 4 * t) = *(const uint4 *)(&planes[warp][16 * t]);
+  }
+  // one reservation for the CTA's blocks, in block order
+  if (lane == 0) s_nnz[warp] = live ? nnz : 0u;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    uint32_t tot = 0;
+    for (uint32_t w = 0; w < kZfWarps; w++) tot += s_nnz[w];
+    uint32_t base = tot ? atomicAdd(a.counter, tot) : 0u;
+    if ((uint64_t)base + tot > a.sparse_cap) set_status(a.status, kFlagNoRoom);
+    for (uint32_t w = 0; w < kZfWarps; w++) {
+      s_base[w] = s_nnz[w] ? base : 0u;
+      base += s_nnz[w];
+    }
+  }
+  __syncthreads();
+  if (!live) return;
+  const uint64_t base = s_base[warp];
+  if (lane == 0) {
+    a.meta[blk] = lb | (nnz << 8);
+    a.sparse_off[blk] = (uint32_t)base;
+  }
+  if (base + nnz > a.sparse_cap) return;
+  for (uint32_t k = lane; k < nnz; k += 32) a.sparse[base + k] = rec[k];
 }
 
-__global__ void __launch_bounds__(kZfThreads) zf_decompress_kernel(const __grid_constant__ ZfArgs a) {
-  __shared__ alignas(16) uint8_t high[kZfBlock];
-  __shared__ alignas(16) uint8_t planes[3 * kZfThreads];
-  __shared__ uint32_t s_bad;
-  const uint32_t tid = threadIdx.x;
-  const uint64_t i0 = (uint64_t)blockIdx.x * kZfBlock;
+__global__ void __launch_bounds__(kZfThreads, 4) zf_decompress_kernel(const __grid_constant__ ZfArgs a) {
+  __shared__ __align__(16) uint8_t high[kZfWarps][kZfBlock];
+  __shared__ __align__(16) uint8_t planes[kZfWarps][3 * kZfPlaneBytes];
+  const uint32_t lane = threadIdx.x & 31u, warp = threadIdx.x >> 5;
+  const uint64_t blk = (uint64_t)blockIdx.x * kZfWarps + warp;
+  if (blk >= a.blocks) return;  // warp-uniform; no CTA barrier below
+  const uint64_t i0 = blk * kZfBlock;
   const uint32_t count = (uint32_t)min((uint64_t)kZfBlock, a.n - i0);
-  const uint32_t j0 = 8 * tid;
-  const uint32_t meta = a.meta[blockIdx.x];
+  const uint32_t meta = a.meta[blk];
   const uint32_t lb = meta & 0xFFu, nnz = meta >> 8;
-  const uint64_t off = a.sparse_off[blockIdx.x];
-  if (nnz > count || off + nnz > a.sparse_cap) {  // uniform over the CTA
-    if (tid == 0) set_status(a.status, kFlagCorrupt);
+  const uint64_t off = a.sparse_off[blk];
+  if (nnz > count || off + nnz > a.sparse_cap) {
+    if (lane == 0) set_status(a.status, kFlagCorrupt);
     return;
   }
-  if (tid == 0) s_bad = 0;
-  *(uint2 *)(high + j0) = make_uint2(0, 0);
-  if (tid < 3 * kZfThreads / 16) {
-    const uint32_t p = tid / (kZfThreads / 16), q = tid % (kZfThreads / 16);
-    *(uint4 *)(planes + p * kZfThreads + 16 * q) =
-        __ldg((const uint4 *)(a.dense + (uint64_t)blockIdx.x * 3 * kZfPlaneWords + p * kZfPlaneWords + 4 * q));
-  }
-  __syncthreads();
-  for (uint32_t k = tid; k < nnz; k += kZfThreads) {
-    const uint32_t rcd = a.sparse[off + k];
-    if ((rcd >> 5) < count) high[rcd >> 5] = (uint8_t)(rcd & 31u);
-    else s_bad = 1;
-  }
-  __syncthreads();
-  if (s_bad) {
-    if (tid == 0) set_status(a.status, kFlagCorrupt);
-    return;
-  }
-  const uint32_t p0 = planes[tid], p1 = planes[kZfThreads + tid], p2 = planes[2 * kZfThreads + tid];
-  const uint2 h = *(const uint2 *)(high + j0);
-  uint32_t e[8];
+  // the block's sign/mantissa bytes: all eight loads in flight at once
+  uint2 smv[kZfSlices];
   #pragma unroll
-  for (int j = 0; j < 8; j++) {
-    const uint32_t hj = ((j < 4 ? h.x : h.y) >> (8 * (j & 3))) & 0xFFu;
-    const uint32_t rj = ((p0 >> j) & 1u) | (((p1 >> j) & 1u) << 1) | (((p2 >> j) & 1u) << 2) | (hj << 3);
-    e[j] = (rj + lb) & 0xFFu;  // inverse of Eq. 4
+  for (uint32_t c = 0; c < kZfSlices; c++) {
+    const uint32_t j0 = 256 * c + 8 * lane;
+    smv[c] = j0 + 8 <= count ? __ldg((const uint2 *)(a.sm + i0 + j0)) : make_uint2(0, 0);
   }
-  if (j0 + 8 <= count) {
-    const uint2 s = __ldg((const uint2 *)(a.sm + i0 + j0));
-    uint32_t o[4];
+  uint8_t *hb = high[warp];
+  #pragma unroll
+  for (int k = 0; k < 4; k++) *(uint4 *)(hb + 16 * (lane + 32 * k)) = make_uint4(0, 0, 0, 0);
+  for (uint32_t t = lane; t < 3 * kZfPlaneBytes / 16; t += 32)
+    *(uint4 *)(&planes[warp][16 * t]) = __ldg((const uint4 *)(a.dense + blk * 192 + 4 * t));
+  __syncwarp();
+  bool bad = false;
+  for (uint32_t k = lane; k < nnz; k += 32) {
+    const uint32_t rcd = a.sparse[off + k];
+    if ((rcd >> 5) < count) hb[rcd >> 5] = (uint8_t)(rcd & 31u);
+    else bad = true;
+  }
+  if (__any_sync(0xffffffffu, bad)) {
+    if (lane == 0) set_status(a.status, kFlagCorrupt);
+    return;
+  }
+  __syncwarp();
+  #pragma unroll
+  for (uint32_t c = 0; c < kZfSlices; c++) {
+    const uint32_t j0 = 256 * c + 8 * lane;
+    if (j0 >= count) break;
+    const uint32_t p0 = planes[warp][32 * c + lane];
+    const uint32_t p1 = planes[warp][kZfPlaneBytes + 32 * c + lane];
+    const uint32_t p2 = planes[warp][2 * kZfPlaneBytes + 32 * c + lane];
+    const uint2 hh = *(const uint2 *)(hb + j0);
+    uint32_t e[8];
     #pragma unroll
-    for (int q = 0; q < 4; q++) {
-      const uint32_t sw = q < 2 ? s.x : s.y;
-      const uint32_t s0 = (sw >> (16 * (q & 1))) & 0xFFu, s1 = (sw >> (16 * (q & 1) + 8)) & 0xFFu;
-      const uint32_t x0 = ((s0 & 0x80u) << 8) | (e[2 * q] << 7) | (s0 & 0x7Fu);
-      const uint32_t x1 = ((s1 & 0x80u) << 8) | (e[2 * q + 1] << 7) | (s1 & 0x7Fu);
-      o[q] = x0 | (x1 << 16);
+    for (int j = 0; j < 8; j++) {
+      const uint32_t hj = ((j < 4 ? hh.x : hh.y) >> (8 * (j & 3))) & 0xFFu;
+      const uint32_t rj = ((p0 >> j) & 1u) | (((p1 >> j) & 1u) << 1) | (((p2 >> j) & 1u) << 2) | (hj << 3);
+      e[j] = (rj + lb) & 0xFFu;  // inverse of Eq. 4
     }
-    *(uint4 *)(a.out + i0 + j0) = make_uint4(o[0], o[1], o[2], o[3]);
-  } else {
-    for (int j = 0; j < 8; j++)
-      if (j0 + j < count) {
-        const uint32_t s = a.sm[i0 + j0 + j];
-        a.out[i0 + j0 + j] = (uint16_t)(((s & 0x80u) << 8) | (e[j] << 7) | (s & 0x7Fu));
+    if (j0 + 8 <= count) {
+      const uint2 s = smv[c];
+      uint32_t o[4];
+      #pragma unroll
+      for (int q = 0; q < 4; q++) {
+        const uint32_t sw = q < 2 ? s.x : s.y;
+        const uint32_t s0 = (sw >> (16 * (q & 1))) & 0xFFu, s1 = (sw >> (16 * (q & 1) + 8)) & 0xFFu;
+        const uint32_t x0 = ((s0 & 0x80u) << 8) | (e[2 * q] << 7) | (s0 & 0x7Fu);
+        const uint32_t x1 = ((s1 & 0x80u) << 8) | (e[2 * q + 1] << 7) | (s1 & 0x7Fu);
+        o[q] = x0 | (x1 << 16);
       }
+      *(uint4 *)(a.out + i0 + j0) = make_uint4(o[0], o[1], o[2], o[3]);
+    } else {
+      for (int j = 0; j < 8; j++)
+        if (j0 + j < count) {
+          const uint32_t sv = a.sm[i0 + j0 + j];
+          a.out[i0 + j0 + j] = (uint16_t)(((sv & 0x80u) << 8) | (e[j] << 7) | (sv & 0x7Fu));
+        }
+    }
   }
 }
 
@@ -244,6 +266,7 @@ bool zf_args(const eh_zf_t *c, ZfArgs *a, void *workspace, uint64_t workspace_by
   if (!al16(c->sign_mant) || !al16(c->dense) || !c->meta || !c->sparse_off || !c->sparse) return false;
   std::memset(a, 0, sizeof(*a));
   a->n = c->n;
+  a->blocks = (c->n + kZfBlock - 1) / kZfBlock;
   a->sm = c->sign_mant;
   a->meta = c->meta;
   a->dense = c->dense;
@@ -275,8 +298,8 @@ eh_status eh_zf_compress(const void *in, eh_zf_t *out, void *workspace, uint64_t
   if (out->n) {
     if (!in || ((uintptr_t)in & 15u)) return EH_ERR_INVALID_ARG;
     a.in = (const uint16_t *)in;
-    const uint32_t B = (uint32_t)((out->n + kZfBlock - 1) / kZfBlock);
-    zf_compress_kernel<<<B, kZfThreads, 0, s>>>(a);
+    const uint32_t grid = (uint32_t)((a.blocks + kZfWarps - 1) / kZfWarps);
+    zf_compress_kernel<<<grid, kZfThreads, 0, s>>>(a);
     if (cudaGetLastError() != cudaSuccess) return EH_ERR_CUDA;
   }
   if (wait) {
@@ -297,8 +320,8 @@ eh_status eh_zf_decompress(const eh_zf_t *c, void *out, void *workspace, uint64_
   if (c->n) {
     if (!out || ((uintptr_t)out & 15u)) return EH_ERR_INVALID_ARG;
     a.out = (uint16_t *)out;
-    const uint32_t B = (uint32_t)((c->n + kZfBlock - 1) / kZfBlock);
-    zf_decompress_kernel<<<B, kZfThreads, 0, s>>>(a);
+    const uint32_t grid = (uint32_t)((a.blocks + kZfWarps - 1) / kZfWarps);
+    zf_decompress_kernel<<<grid, kZfThreads, 0, s>>>(a);
     if (cudaGetLastError() != cudaSuccess) return EH_ERR_CUDA;
   }
   return EH_OK;
