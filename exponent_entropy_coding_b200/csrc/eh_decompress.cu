@@ -1,23 +1,27 @@
 // eh_decompress.cu -- decompression kernels of libexphuff (sm_100a).
 //
-//   tables  one CTA per codebook: validates the code lengths and codes and
-//           builds the decode tables (an 8-bit first level that decodes up to
-//           four short codes per lookup, 8-bit second-level tables for codes
-//           of 9..16 bits, canonical limits for anything longer);
-//   decode  persistent CTAs, one chunk at a time:
+//   tables  eight CTAs per codebook: validate the code lengths and codes and
+//           build the decode tables (a 12-bit first level giving, for the
+//           index bits, the symbols of up to four complete codes, their bits,
+//           and the number, bits and start offsets of all complete codes;
+//           8-bit second-level tables for codes of 13..20 bits; canonical
+//           limits for anything longer);
+//   decode  persistent CTAs of two independent groups, one chunk per group
+//           at a time:
 //             1. the chunk's bit range is copied into shared memory with one
 //                bulk asynchronous copy (cp.async.bulk + mbarrier) when it
 //                fits, else read from global memory;
-//             2. every thread decodes speculatively from the start of its own
-//                window of the chunk's bits, recording the code boundaries of
-//                its first 32 bits;
+//             2. every thread counts the codes of its own window of the
+//                chunk's bits, starting speculatively at the window start and
+//                recording the code boundaries of its first 64 bits;
 //             3. fix-up rounds: each thread restarts from the true end of its
 //                predecessor and stops as soon as it lands on one of its
 //                recorded boundaries (Huffman codes resynchronise after a few
 //                codes), until no end moves;
-//             4. CTA-wide exclusive scan of the per-thread code counts gives
-//                every thread its first output index;
-//             5. the threads decode again and write exponents to shared memory;
+//             4. group-wide exclusive scan of the per-thread code counts
+//                gives every thread its first output index;
+//             5. the threads decode again from their true starts and write
+//                their exponents to shared memory;
 //             6. coalesced pass: exponents merged with the sign/mantissa
 //                stream and stored with 16-byte stores.
 // The DFloat11 article ("方法介绍") describes compact LUTs sized for on-chip
@@ -410,6 +414,9 @@ struct ExpWriter {
   }
 };
 
+// the low r8 / 8 bytes of a word (r8 a multiple of 8, at most 32)
+__device__ __forceinline__ uint32_t low_bytes_mask(uint32_t r8) { return r8 >= 32 ? ~0u : (1u << r8) - 1u; }
+
 // Steps 2-5 for one chunk whose bits are [rel0, rel0 + nbits) of `words`,
 // decoded by one group.  Returns false (group-uniform) if the chunk is
 // corrupt.
@@ -542,11 +549,13 @@ __device__ bool decode_chunk(GroupSmem &G, const DecodeTables &T, const uint32_t
   const bool ok = !gsync_or(id, bad) && total == cnt && G.ends[kGroupThreads - 1] == nbits;
   if (!ok) return false;
 
-  // 5. decode again from the true start, writing exponents
+  // 5. decode again from the true start, writing exactly the thread's my_n
+  //    exponents (a count, not the window end, stops the loop)
   ExpWriter out;
   out.init(G.exps, o);
   pos = gtid == 0 ? 0u : G.ends[gtid - 1];
-  while (pos + kBulk <= we) {
+  uint32_t rem8 = 8 * my_n;  // exponent bits still to write
+  while (rem8) {
     const uint32_t x = peek(rel0 + pos);
     const uint32_t i1 = lut_index(x);
     const uint32_t m1 = T.l1meta[i1];
@@ -556,27 +565,31 @@ __device__ bool decode_chunk(GroupSmem &G, const DecodeTables &T, const uint32_t
       if (!decode_long(T, x, m1, syms, nb)) break;
       pos += nb;
       out.put(syms, 8);
+      rem8 -= 8;
       continue;
     }
     const uint32_t s1 = T.l1sym[i1];
+    if (k1 >= rem8) {  // the last codes of the thread
+      out.put(s1 & low_bytes_mask(rem8), rem8);
+      break;
+    }
+    out.put(s1, k1);
+    rem8 -= k1;
     const uint32_t i2 = lut_index(x << nb1);
     const uint32_t m2 = T.l1meta[i2];
     const uint32_t k2 = (m2 >> 1) & 0x38u, nb2 = m2 & 15u;
-    out.put(s1, k1);
     if (!k2) {
       pos += nb1;
       continue;
     }
     const uint32_t s2 = T.l1sym[i2];
-    pos += nb1 + nb2;
+    if (k2 >= rem8) {
+      out.put(s2 & low_bytes_mask(rem8), rem8);
+      break;
+    }
     out.put(s2, k2);
-  }
-  while (pos < we) {
-    uint32_t syms, nb, bnd;
-    const uint32_t k = decode_step<true>(T, peek(rel0 + pos), we - pos, syms, nb, bnd);
-    if (!k) break;
-    pos += nb;
-    out.put(syms, 8 * k);
+    rem8 -= k2;
+    pos += nb1 + nb2;
   }
   out.finish();
   gsync(id);
