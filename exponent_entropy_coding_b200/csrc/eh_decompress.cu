@@ -355,30 +355,29 @@ __device__ __forceinline__ bool gsync_or(uint32_t id, bool pred) {
   return r != 0;
 }
 
-__device__ __forceinline__ uint32_t group_excl_scan(uint32_t v, uint32_t *wsum, uint32_t *total, uint32_t id,
-                                                    uint32_t gtid) {
-  constexpr int kWarps = kGroupThreads / 32;
-  const int lane = gtid & 31, warp = gtid >> 5;
+// Exclusive scan of v over the group with one barrier, which also ORs `pred`
+// over the group (*any).  Every warp reduces the warp totals itself.
+__device__ __forceinline__ uint32_t group_excl_scan_or(uint32_t v, bool pred, uint32_t *wsum, uint32_t *total,
+                                                       bool *any, uint32_t id, uint32_t gtid) {
+  constexpr uint32_t kWarps = kGroupThreads / 32;
+  const uint32_t lane = gtid & 31u, warp = gtid >> 5;
   uint32_t x = v;
   #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
-    uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
-    if (lane >= o) x += y;
+    const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= (uint32_t)o) x += y;
   }
   if (lane == 31) wsum[warp] = x;
-  gsync(id);
-  if (warp == 0) {
-    uint32_t t = lane < kWarps ? wsum[lane] : 0u;
-    #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      uint32_t y = __shfl_up_sync(0xffffffffu, t, o);
-      if (lane >= o) t += y;
-    }
-    if (lane < kWarps) wsum[lane] = t;
+  *any = gsync_or(id, pred);
+  const uint32_t t = lane < kWarps ? wsum[lane] : 0u;
+  uint32_t pre = lane < warp ? t : 0u, all = t;
+  #pragma unroll
+  for (int o = 16; o; o >>= 1) {
+    pre += __shfl_xor_sync(0xffffffffu, pre, o);
+    all += __shfl_xor_sync(0xffffffffu, all, o);
   }
-  gsync(id);
-  *total = wsum[kWarps - 1];
-  return (warp ? wsum[warp - 1] : 0u) + x - v;
+  *total = all;
+  return pre + x - v;
 }
 
 // Packs decoded exponents four to a word into the exponent buffer, which
@@ -533,7 +532,9 @@ __device__ bool decode_chunk(GroupSmem &G, const DecodeTables &T, const uint32_t
       changed = new_end != my_end;
       my_end = new_end;
     }
-    gsync(id);
+    // A successor may read this end in the same round, before or after the
+    // store: an older end only costs it another round, and a round in which
+    // no end moved (seen by everyone after the barrier) ends the fix-up.
     if (changed) G.ends[gtid] = my_end;
     if (!gsync_or(id, changed)) break;
     if (round > kGroupThreads + 1) {  // cannot happen for consistent data
@@ -545,8 +546,9 @@ __device__ bool decode_chunk(GroupSmem &G, const DecodeTables &T, const uint32_t
 
   // 4. output index of every thread's first code
   uint32_t total;
-  const uint32_t o = group_excl_scan(my_n, G.wsum, &total, id, gtid);
-  const bool ok = !gsync_or(id, bad) && total == cnt && G.ends[kGroupThreads - 1] == nbits;
+  bool anybad;
+  const uint32_t o = group_excl_scan_or(my_n, bad, G.wsum, &total, &anybad, id, gtid);
+  const bool ok = !anybad && total == cnt && G.ends[kGroupThreads - 1] == nbits;
   if (!ok) return false;
 
   // 5. decode again from the true start, writing exactly the thread's my_n
@@ -732,13 +734,21 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
       const uint32_t cnt = ci.cnt;
       bool ok = ci.ok && !terr && !S.abort_flag;
 
-      // the exponent words are OR-ed in: clear them
-      for (uint32_t i = gtid; i < kExpBytes / 16; i += kGroupThreads) ((uint4 *)G.exps)[i] = make_uint4(0, 0, 0, 0);
+      // One barrier per chunk before the decode: after it the stage holds the
+      // chunk's stream words in MSB-first order and every thread of the group
+      // is done with the previous chunk's exponent buffer.
       if (ci.fits) {
         uint32_t spins = 0;
         while (!mbar_try_wait(&G.mbar, parity) && ++spins < kSpinLimit) {
         }
-        if (gsync_or(id, spins >= kSpinLimit)) {
+        const bool late = spins >= kSpinLimit;
+        if (!late) {
+          // stream words to MSB-first order, once, for the peeks
+          for (uint32_t i = gtid; i < ci.bytes / 4; i += kGroupThreads) G.stage[i] = bswap32(G.stage[i]);
+        }
+        // these generic writes come before the next bulk copy into the stage
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        if (gsync_or(id, late)) {
           if (gtid == 0) {
             set_status(b.status, kFlagTimeout);
             S.abort_flag = 1;
@@ -747,12 +757,9 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
         } else {
           parity ^= 1u;
           pending = false;
-          // stream words to MSB-first order, once, for the peeks
-          for (uint32_t i = gtid; i < ci.bytes / 4; i += kGroupThreads) G.stage[i] = bswap32(G.stage[i]);
-          gsync(id);
         }
       } else {
-        gsync(id);  // the cleared exponent buffer is visible to the group
+        gsync(id);
       }
       if (ok && ci.raw) {
         // page stored raw: its exponent bytes go straight to the buffer
@@ -765,8 +772,12 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
           d[2] = x.z;
           d[3] = x.w;
         }
+        for (uint32_t i = cnt / 16 * 16 + gtid; i < cnt; i += kGroupThreads) G.exps[exp_slot(i)] = src[i];
         gsync(id);
       } else if (ok) {
+        // the exponent words are OR-ed in: clear them (ordered before the
+        // writing pass by the decoder's barriers)
+        for (uint32_t i = gtid; i < kExpBytes / 16; i += kGroupThreads) ((uint4 *)G.exps)[i] = make_uint4(0, 0, 0, 0);
         if (ci.fits) ok = decode_chunk<true>(G, S.tabs, G.stage, ci.rel0, ci.nbits, cnt, id, gtid, &timeout);
         else
           ok = decode_chunk<false>(G, S.tabs, (const uint32_t *)(I.stream + ci.lo), ci.rel0, ci.nbits, cnt, id,
@@ -777,9 +788,9 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
       }
 
       if (stagger && grp == 0 && g == seg) named_arrive(kStaggerBarrier, kDecThreads);
-      // the stage is free: start copying the group's next chunk
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      gsync(id);
+      // The stage is free: every read of it came before the decoder's last
+      // barrier, and its generic writes were fenced before the chunk's first
+      // barrier.  Start copying the group's next chunk.
       ChunkInfo cn;
       cn.fits = false;
       if (g + kNumGroups < seg_end && !pending && !S.abort_flag) {
@@ -865,7 +876,8 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
           }
         }
       }
-      gsync(id);  // the exponent buffer may be cleared for the next chunk
+      // no barrier here: the next chunk's first barrier orders these reads of
+      // the exponent buffer before it is cleared or written again
       ci = cn;
     }
     seg = seg_end;
