@@ -515,6 +515,16 @@ __device__ __forceinline__ void ring_or(uint32_t *ring, uint64_t pos, uint32_t a
   if (s + nbits > 32) atomicOr(&ring[(w + 1) & kRingMask], (uint32_t)y);
 }
 
+// ORs the low nbits (1..64) of (hi:lo) into the ring at stream bit pos.
+__device__ __forceinline__ void ring_or64(uint32_t *ring, uint64_t pos, uint32_t hi, uint32_t lo, uint32_t nbits) {
+  const uint32_t s = (uint32_t)(pos & 31);
+  const uint64_t w = pos >> 5;
+  const uint64_t L = (((uint64_t)hi << 32) | lo) << (64 - nbits);  // left-aligned
+  atomicOr(&ring[w & kRingMask], (uint32_t)(L >> (32 + s)));
+  if (s + nbits > 32) atomicOr(&ring[(w + 1) & kRingMask], (uint32_t)(L >> s));
+  if (s + nbits > 64) atomicOr(&ring[(w + 2) & kRingMask], (uint32_t)(L << (32 - s)));
+}
+
 // Packs the codes of values [0, cnt) of `in` into stream bits [bit0, bit1)
 // of gs.  The ring must be zero on entry and is zero on return.  Words that
 // the range shares with its neighbours are OR-ed into (pre-cleared) stream
@@ -531,14 +541,16 @@ __device__ void encode_range(const uint2 *tab, const uint8_t *in, uint32_t cnt, 
     const uint32_t idx = t0 + tid * kEncPerThread;
     const uint4 p = np, q = nq;
     if (t0 + kEncTile < cnt) load_exps<DT>(in, idx + kEncTile, cnt, np, nq);
-    // two groups of 8 codes, each concatenated in a 32-bit accumulator when
-    // it fits (the usual case); longer groups take the per-code path
-    uint32_t acc[2] = {0u, 0u}, tot[2] = {0u, 0u};
+    // two groups of 8 codes, each concatenated in a 64-bit accumulator
+    // (hi:lo) when it fits (all but pathological codes); longer groups take
+    // the per-code path
+    uint32_t hi[2] = {0u, 0u}, lo[2] = {0u, 0u}, tot[2] = {0u, 0u};
     if (idx + kEncPerThread <= cnt) {
       #pragma unroll
       for (int j = 0; j < kEncPerThread; j++) {
         const uint2 cl = tab[exp_of<DT>(p, q, j)];
-        acc[j >> 3] = __funnelshift_lc(cl.x, acc[j >> 3], cl.y);
+        hi[j >> 3] = __funnelshift_lc(lo[j >> 3], hi[j >> 3], cl.y);
+        lo[j >> 3] = __funnelshift_lc(cl.x, lo[j >> 3], cl.y);
         tot[j >> 3] += cl.y;
       }
     } else {
@@ -546,7 +558,8 @@ __device__ void encode_range(const uint2 *tab, const uint8_t *in, uint32_t cnt, 
       for (int j = 0; j < kEncPerThread; j++) {
         uint2 cl = tab[exp_of<DT>(p, q, j)];
         if (idx + j >= cnt) cl = make_uint2(0u, 0u);
-        acc[j >> 3] = __funnelshift_lc(cl.x, acc[j >> 3], cl.y);
+        hi[j >> 3] = __funnelshift_lc(lo[j >> 3], hi[j >> 3], cl.y);
+        lo[j >> 3] = __funnelshift_lc(cl.x, lo[j >> 3], cl.y);
         tot[j >> 3] += cl.y;
       }
     }
@@ -556,8 +569,8 @@ __device__ void encode_range(const uint2 *tab, const uint8_t *in, uint32_t cnt, 
     #pragma unroll
     for (int h = 0; h < 2; h++) {
       if (tot[h] == 0) continue;
-      if (tot[h] <= 32) {
-        ring_or(ring, pos, acc[h], tot[h]);
+      if (tot[h] <= 64) {
+        ring_or64(ring, pos, hi[h], lo[h], tot[h]);
       } else {
         uint64_t pp = pos;
         for (int j = 8 * h; j < 8 * h + 8; j++) {
