@@ -49,6 +49,7 @@ template <int DT>
 __global__ void __launch_bounds__(kThreads, 2) hist_kernel(const __grid_constant__ Batch b) {
   constexpr int A = DT == EH_FP8_E4M3 ? 16 : 256;
   __shared__ uint32_t h[A * 32];
+  pdl_trigger();
   const uint32_t g = blockIdx.x;
   const Item &I = b.item[find_item(b, g)];
   const uint32_t c = g - I.chunk0;
@@ -141,11 +142,12 @@ __global__ void __launch_bounds__(kThreads, 2) hist_kernel(const __grid_constant
 // ---------------------------------------------------------------- book
 // One CTA of 256 threads per tensor.
 __global__ void __launch_bounds__(256) book_kernel(const __grid_constant__ Batch b) {
+  pdl_trigger();
+  pdl_wait();  // the histogram kernel's counts
   const Item &I = b.item[blockIdx.x];
   const int A = alphabet_of(b.dtype);
   const int Lmax = (int)b.max_code_len;
   const int tid = threadIdx.x;
-  __shared__ uint64_t cnt[256];
   __shared__ uint64_t lw[256];      // leaf weights in (count, symbol) order
   __shared__ uint64_t iw[256];      // internal node weights in creation order
   __shared__ uint16_t lpar[256], ipar[256];
@@ -153,12 +155,13 @@ __global__ void __launch_bounds__(256) book_kernel(const __grid_constant__ Batch
   __shared__ uint8_t len[256];
   __shared__ uint32_t nlen[33], firstc[33];
   __shared__ uint32_t xsel[33];     // package-merge: leaves selected per level
-  __shared__ uint32_t maxd;
+  __shared__ uint32_t maxd, nint_s;
   __shared__ uint8_t ps[256];       // present symbols, increasing
+  __shared__ uint64_t pcnt[256];    // their counts, in the same order
+  __shared__ uint8_t plen[256];     // their code lengths, in the same order
   __shared__ uint32_t wpres[8];
 
   const uint64_t c = tid < A ? I.counts[tid] : 0ull;
-  cnt[tid] = c;
   len[tid] = 0;
   if (tid <= 32) nlen[tid] = 0;
   if (tid == 0) maxd = 0;
@@ -172,16 +175,22 @@ __global__ void __launch_bounds__(256) book_kernel(const __grid_constant__ Batch
     if (w < (tid >> 5)) pidx += wpres[w];
     m += wpres[w];
   }
-  if (c > 0) ps[pidx] = (uint8_t)tid;
-  __syncthreads();
   if (c > 0) {
-    int r = 0;
+    ps[pidx] = (uint8_t)tid;
+    pcnt[pidx] = c;
+  }
+  __syncthreads();
+  // rank of each present symbol in (count, symbol) order (independent loads)
+  uint32_t r_asc = 0, r_desc = 0;
+  if (c > 0) {
+    #pragma unroll 4
     for (int j = 0; j < m; j++) {
-      const int s2 = ps[j];
-      const uint64_t c2 = cnt[s2];
-      r += c2 < c || (c2 == c && s2 < tid);
+      const uint64_t c2 = pcnt[j];
+      const bool below = ps[j] < tid;
+      r_asc += c2 < c || (c2 == c && below);
+      r_desc += c2 > c || (c2 == c && below);
     }
-    lw[r] = c;
+    lw[r_asc] = c;
   }
   bool feasible = m <= 1 || Lmax >= 32 || (uint64_t)m <= (1ull << Lmax);
   if (!feasible) {
@@ -193,26 +202,58 @@ __global__ void __launch_bounds__(256) book_kernel(const __grid_constant__ Batch
   if (m >= 2 && feasible) {
     if (tid == 0) {
       // two-queue Huffman: leaves sorted by (count, symbol), internal nodes in
-      // creation order; on equal weight the leaf wins (its id is smaller)
+      // creation order; on equal weight the leaf wins (its id is smaller).
+      // The next leaf and the next internal weight are kept in registers.
       int i = 0, j = 0, nint = 0;
+      uint64_t li = lw[0], ij = 0;  // ij is iw[j] while j < nint
       for (int step = 0; step < m - 1; step++) {
         uint64_t w = 0;
         #pragma unroll
         for (int pick = 0; pick < 2; pick++) {
-          if (i < m && (j >= nint || lw[i] <= iw[j])) {
-            w += lw[i];
+          if (i < m && (j >= nint || li <= ij)) {
+            w += li;
             lpar[i++] = (uint16_t)nint;
+            li = i < m ? lw[i] : 0ull;
           } else {
-            w += iw[j];
+            w += ij;
             ipar[j++] = (uint16_t)nint;
+            ij = j < nint ? iw[j] : 0ull;
           }
         }
-        iw[nint++] = w;
+        iw[nint] = w;
+        if (j == nint) ij = w;  // the queue was empty: the new node is next
+        nint++;
       }
-      idep[nint - 1] = 0;
-      for (int k = nint - 2; k >= 0; k--) idep[k] = (uint8_t)(idep[ipar[k]] + 1);
+      nint_s = (uint32_t)nint;
     }
     __syncthreads();
+    // internal node depths by pointer jumping: depth += depth(parent),
+    // parent = parent(parent); the root (last node) is its own parent
+    const uint32_t nint = nint_s;
+    uint32_t dep = 0, par = 0;
+    if (tid < nint) {
+      const bool root = tid == nint - 1;
+      dep = root ? 0u : 1u;
+      par = root ? tid : ipar[tid];
+      idep[tid] = (uint8_t)dep;
+      ipar[tid] = (uint16_t)par;
+    }
+    __syncthreads();
+    for (int round = 0; round < 8; round++) {  // 2^8 levels cover any tree of 256 leaves
+      uint32_t pd = 0, pp = 0;
+      if (tid < nint) {
+        pd = idep[par];
+        pp = ipar[par];
+      }
+      __syncthreads();
+      if (tid < nint) {
+        dep += pd;
+        par = pp;
+        idep[tid] = (uint8_t)dep;
+        ipar[tid] = (uint16_t)par;
+      }
+      __syncthreads();
+    }
     if (tid < m) {
       d = idep[lpar[tid]] + 1u;
       atomicMax(&maxd, d);
@@ -269,12 +310,7 @@ __global__ void __launch_bounds__(256) book_kernel(const __grid_constant__ Batch
   // rank assignment: the r-th shortest length goes to the symbol of rank r in
   // (count descending, symbol ascending) order
   if (c > 0 && feasible) {
-    uint32_t r = 0;
-    for (int j = 0; j < m; j++) {
-      const int s2 = ps[j];
-      const uint64_t c2 = cnt[s2];
-      r += (c2 > c) || (c2 == c && s2 < tid);
-    }
+    const uint32_t r = r_desc;
     uint32_t cum = 0, L = 1;
     for (; L <= 32; L++) {
       cum += nlen[L];
@@ -282,22 +318,30 @@ __global__ void __launch_bounds__(256) book_kernel(const __grid_constant__ Batch
     }
     len[tid] = (uint8_t)L;
   }
-  if (tid == 0) {
-    uint64_t code = 0;
-    for (int L = 1; L <= 32; L++) {
-      firstc[L] = (uint32_t)code;
-      code = (code + nlen[L]) << 1;
+  if (tid < 32) {
+    // first canonical code of each length L (lane L-1): the exclusive prefix
+    // of nlen[L'] << (32 - L'), shifted down by 32 - L
+    const uint32_t L = tid + 1;
+    const uint64_t aL = (uint64_t)nlen[L] << (32 - L);
+    uint64_t inc = aL;
+    #pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint64_t y = __shfl_up_sync(0xffffffffu, inc, o);
+      if (tid >= (uint32_t)o) inc += y;
     }
+    firstc[L] = (uint32_t)((inc - aL) >> (32 - L));
   }
+  __syncthreads();
+  if (tid < m) plen[tid] = len[ps[tid]];
   __syncthreads();
   if (tid < A) {
     uint32_t l = len[tid], code = 0;
     if (l) {
+      // symbols of the same length below this one (present symbols are in
+      // increasing order, so the first pidx entries are the smaller ones)
       uint32_t k = 0;
-      for (int j = 0; j < m; j++) {
-        const int s2 = ps[j];
-        k += s2 < tid && len[s2] == l;
-      }
+      #pragma unroll 4
+      for (uint32_t j = 0; j < pidx; j++) k += plen[j] == l;
       code = firstc[l] + k;
     }
     I.code_len[tid] = (uint8_t)l;
@@ -317,6 +361,8 @@ constexpr int kOffPerThread = 4;           // chunks per thread in the final sca
 constexpr int kOffTile = kOffThreads * kOffPerThread;
 
 __global__ void __launch_bounds__(kOffThreads) offsets_kernel(const __grid_constant__ Batch b) {
+  pdl_trigger();
+  pdl_wait();  // the code lengths
   const int A = alphabet_of(b.dtype);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const uint32_t g = blockIdx.x * (kOffThreads / 32) + warp;
@@ -618,8 +664,9 @@ __global__ void __launch_bounds__(kThreads, 2) encode_kernel(const __grid_consta
   const uint32_t c = g - I.chunk0;
   const uint64_t i0 = (uint64_t)c * b.chunk_elems;
   const uint32_t cnt = (uint32_t)min((uint64_t)b.chunk_elems, I.n - i0);
-  load_code_table<DT>(tab, I.code_len, I.code);
   for (int i = threadIdx.x; i < kRingWords; i += kThreads) ring[i] = 0u;
+  pdl_wait();  // the codebook and the chunk offsets
+  load_code_table<DT>(tab, I.code_len, I.code);
   const uint8_t *in = (const uint8_t *)I.in + i0 * (DT == EH_BF16 ? 2 : 1);
   __syncthreads();
   encode_range<DT>(tab, in, cnt, I.off[c], I.off[c + 1], (uint32_t *)I.stream, ring, wsum, false);
@@ -720,15 +767,13 @@ cudaError_t launch_hist(const Batch &b, cudaStream_t s) {
 }
 
 cudaError_t launch_book(const Batch &b, cudaStream_t s) {
-  book_kernel<<<b.k, 256, 0, s>>>(b);
-  return cudaGetLastError();
+  return launch_pdl(book_kernel, dim3(b.k), dim3(256), 0, s, b);
 }
 
 cudaError_t launch_offsets(const Batch &b, cudaStream_t s) {
   uint32_t grid = (b.total_chunks + kOffThreads / 32 - 1) / (kOffThreads / 32);
   if (grid == 0) grid = 1;  // the last CTA still writes off[0] = 0 and the bit totals
-  offsets_kernel<<<grid, kOffThreads, 0, s>>>(b);
-  return cudaGetLastError();
+  return launch_pdl(offsets_kernel, dim3(grid), dim3(kOffThreads), 0, s, b);
 }
 
 cudaError_t configure_encode() {
@@ -758,9 +803,9 @@ cudaError_t launch_page_append(const PageLaunch &pl, cudaStream_t s) {
 cudaError_t launch_encode(const Batch &b, cudaStream_t s) {
   if (b.total_chunks == 0) return cudaSuccess;
   const size_t smem = kRingWords * sizeof(uint32_t);
-  if (b.dtype == EH_BF16) encode_kernel<EH_BF16><<<b.total_chunks, kThreads, smem, s>>>(b);
-  else if (b.dtype == EH_BYTES) encode_kernel<EH_BYTES><<<b.total_chunks, kThreads, smem, s>>>(b);
-  else encode_kernel<EH_FP8_E4M3><<<b.total_chunks, kThreads, smem, s>>>(b);
+  if (b.dtype == EH_BF16) return launch_pdl(encode_kernel<EH_BF16>, dim3(b.total_chunks), dim3(kThreads), smem, s, b);
+  if (b.dtype == EH_BYTES) return launch_pdl(encode_kernel<EH_BYTES>, dim3(b.total_chunks), dim3(kThreads), smem, s, b);
+  return launch_pdl(encode_kernel<EH_FP8_E4M3>, dim3(b.total_chunks), dim3(kThreads), smem, s, b);
   return cudaGetLastError();
 }
 

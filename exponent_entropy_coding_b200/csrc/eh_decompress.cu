@@ -62,50 +62,62 @@ __global__ void __launch_bounds__(256) tables_kernel(const __grid_constant__ Bat
   __shared__ uint32_t cntL[33], firstL[33], baseL[33];
   __shared__ uint64_t limL[33];
   __shared__ uint8_t srt[256];
-  __shared__ unsigned long long kraft;
   __shared__ uint32_t err;
   __shared__ uint32_t wlen[8][33];  // per warp: symbols of each length
 
+  pdl_trigger();
+  pdl_wait();  // the codebooks may come from the kernels just before
   if (blockIdx.x == 0 && tid == 0) {
     *b.status = 0u;  // this call's status starts clean
     *b.ticket = 0u;
   }
   if (tid <= 32) cntL[tid] = 0;
   for (int i = tid; i < 8 * 33; i += 256) (&wlen[0][0])[i] = 0;
-  if (tid == 0) { kraft = 0; err = 0; }
+  if (tid == 0) err = 0;
   const uint32_t l = tid < A ? I.code_len[tid] : 0u;
   __syncthreads();
   if (l > 32) atomicOr(&err, 1u);
   else if (l) {
     atomicAdd(&cntL[l], 1u);
     atomicAdd(&wlen[tid >> 5][l], 1u);
-    atomicAdd(&kraft, 1ull << (32 - l));
   }
   const uint32_t nsym = __syncthreads_count(l > 0 && l <= 32);
-  if (tid == 0) {
-    uint64_t code = 0;
-    uint32_t idx = 0, g = 0, maxlen = 0;
-    for (int L = 1; L <= 32; L++) {
-      firstL[L] = (uint32_t)code;
-      baseL[L] = idx;
-      limL[L] = (code + cntL[L]) << (32 - L);
-      code = (code + cntL[L]) << 1;
-      idx += cntL[L];
-      if (cntL[L]) {
-        uint32_t a = g, c = (uint32_t)L;
-        while (c) { uint32_t t = a % c; a = c; c = t; }
-        g = a;
-        maxlen = (uint32_t)L;
+  if (tid < 32) {
+    // Canonical limits by one warp, lane L-1 for length L: with
+    // a_L = count_L << (32 - L), the inclusive prefix of a is lim[L] and the
+    // exclusive one, shifted down, is the first code of length L.
+    const uint32_t L = tid + 1, cL = cntL[L];
+    const uint64_t aL = (uint64_t)cL << (32 - L);
+    uint64_t inc = aL;
+    uint32_t idx = cL;
+    #pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint64_t y = __shfl_up_sync(0xffffffffu, inc, o);
+      const uint32_t z = __shfl_up_sync(0xffffffffu, idx, o);
+      if (tid >= (uint32_t)o) {
+        inc += y;
+        idx += z;
       }
     }
-    limL[0] = 0;
-    firstL[0] = baseL[0] = cntL[0] = 0;
-    if (kraft > (1ull << 32)) err = 1;
-    if (I.n > 0 && nsym == 0) err = 1;
-    if (part == 0) {
-      T->gcd = g ? g : 1;
-      T->maxlen = maxlen;
-      T->nsym = nsym;
+    limL[L] = inc;
+    firstL[L] = (uint32_t)((inc - aL) >> (32 - L));
+    baseL[L] = idx - cL;
+    // lengths in use: their gcd (largest d dividing all of them) and maximum
+    const uint32_t used = __ballot_sync(0xffffffffu, cL != 0);
+    uint32_t mult = 0;  // lengths that are multiples of d = L
+    for (uint32_t k = L; k <= 32; k += L) mult |= 1u << (k - 1);
+    const uint32_t divides = __ballot_sync(0xffffffffu, used && (used & ~mult) == 0);
+    const uint64_t kraft = __shfl_sync(0xffffffffu, inc, 31);  // every lane takes part
+    if (tid == 0 && kraft > (1ull << 32)) err = 1;
+    if (tid == 0) {
+      limL[0] = 0;
+      firstL[0] = baseL[0] = cntL[0] = 0;
+      if (I.n > 0 && nsym == 0) err = 1;
+      if (part == 0) {
+        T->gcd = divides ? 32u - __clz(divides) : 1u;
+        T->maxlen = used ? 32u - __clz(used) : 0u;
+        T->nsym = nsym;
+      }
     }
   }
   __syncthreads();
@@ -702,6 +714,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (tid == 0) S.abort_flag = 0;
+  pdl_wait();  // the decode tables (and everything before them)
   __syncthreads();
   uint32_t parity = 0, timeout = 0;
   bool pending = false;  // a stage copy of this group is in flight
@@ -894,8 +907,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
 }  // namespace
 
 cudaError_t launch_tables(const Batch &b, cudaStream_t s) {
-  tables_kernel<<<b.k * kTabParts, 256, 0, s>>>(b);
-  return cudaGetLastError();
+  return launch_pdl(tables_kernel, dim3(b.k * kTabParts), dim3(256), 0, s, b);
 }
 
 cudaError_t launch_decode(const Batch &b, cudaStream_t s, int num_sms) {
@@ -903,10 +915,9 @@ cudaError_t launch_decode(const Batch &b, cudaStream_t s, int num_sms) {
   const size_t smem = sizeof(DecodeSmem) + 128;
   uint32_t grid = (uint32_t)num_sms;
   if (grid > b.total_chunks) grid = b.total_chunks;
-  if (b.dtype == EH_BF16) decode_kernel<EH_BF16><<<grid, kDecThreads, smem, s>>>(b);
-  else if (b.dtype == EH_BYTES) decode_kernel<EH_BYTES><<<grid, kDecThreads, smem, s>>>(b);
-  else decode_kernel<EH_FP8_E4M3><<<grid, kDecThreads, smem, s>>>(b);
-  return cudaGetLastError();
+  if (b.dtype == EH_BF16) return launch_pdl(decode_kernel<EH_BF16>, dim3(grid), dim3(kDecThreads), smem, s, b);
+  if (b.dtype == EH_BYTES) return launch_pdl(decode_kernel<EH_BYTES>, dim3(grid), dim3(kDecThreads), smem, s, b);
+  return launch_pdl(decode_kernel<EH_FP8_E4M3>, dim3(grid), dim3(kDecThreads), smem, s, b);
 }
 
 cudaError_t configure_decode() {

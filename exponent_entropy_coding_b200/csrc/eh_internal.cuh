@@ -6,6 +6,7 @@
 #pragma once
 
 #include <cuda_runtime.h>
+#include <utility>
 #include <stdint.h>
 
 #include "exphuff.h"
@@ -139,6 +140,29 @@ constexpr uint64_t kLutBytes = (sizeof(DecodeTables) + 255) & ~uint64_t(255);
 __host__ __device__ inline uint64_t align256(uint64_t x) { return (x + 255) & ~uint64_t(255); }
 
 // ---- host-side launch wrappers (defined in the .cu files)
+// Programmatic dependent launch: a kernel launched with launch_pdl may start
+// while the previous kernel of the stream is still running; it calls
+// pdl_wait() before touching anything that kernel (or an earlier one) wrote.
+// pdl_trigger() lets the next such kernel start before this one ends.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                              Args &&...args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 cudaError_t launch_hist(const Batch &b, cudaStream_t s);
 cudaError_t launch_book(const Batch &b, cudaStream_t s);
 cudaError_t launch_offsets(const Batch &b, cudaStream_t s);
