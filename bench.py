@@ -32,7 +32,7 @@ FALLBACK_HBM_GBS = 6650.0
 # DRAM traffic per decode launch on the full block, from one ncu capture
 # (dram__bytes_read.sum + dram__bytes_write.sum), valid only for the decoder
 # source it was taken on.
-DECODE_TRAFFIC = {"bytes": 293231616 + 374882304, "source_sha": "531e4b32324d2310"}
+DECODE_TRAFFIC = {"bytes": 292652032 + 374814976, "source_sha": "61288420b0d80077"}
 
 
 def decoder_source_sha():
@@ -52,7 +52,9 @@ def hbm_peak():
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons during the timed region."""
+    """nvidia-smi clocks and throttle reasons during the timed region.  The
+    sampler is started first and the timed region begins once its first
+    sample has arrived, so that short regions are still sampled."""
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
@@ -60,8 +62,16 @@ class ClockSampler:
     def __init__(self, gpu_index):
         self.gpu = gpu_index
         self.proc = None
+        self.lines = []
+        self.mark = 0
+
+    def _read(self):
+        for line in self.proc.stdout:
+            if line.strip():
+                self.lines.append(line)
 
     def __enter__(self):
+        import threading
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
@@ -69,23 +79,31 @@ class ClockSampler:
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except (OSError, ValueError):
             self.proc = None
+            return self
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+        t0 = time.time()
+        while not self.lines and time.time() - t0 < 10 and self.proc.poll() is None:
+            time.sleep(0.01)
+        self.mark = len(self.lines)  # samples from here on fall in the timed region
         return self
 
     def __exit__(self, *exc):
-        self.lines = []
         if self.proc is not None:
             self.proc.terminate()
             try:
-                out, _ = self.proc.communicate(timeout=5)
+                self.proc.wait(timeout=5)
             except subprocess.TimeoutExpired:
                 self.proc.kill()
-                out, _ = self.proc.communicate()
-            self.lines = [l for l in out.splitlines() if l.strip()]
+            self.thread.join(timeout=5)
+        # the sample taken just before the region ended is kept; earlier ones
+        # (before the region started) are not
+        self.lines = self.lines[max(self.mark - 1, 0):]
 
     def summary(self):
         sm, mx, reasons = [], [], set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for l in getattr(self, "lines", []):
+        for l in self.lines:
             f = [x.strip() for x in l.split(",")]
             if len(f) < 9:
                 continue
@@ -371,6 +389,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--no-side", action="store_true",
+                    help="skip the side measurements (FP4 scales, K/V pages, ZipFloat, prefetch ring)")
     ap.add_argument("--ncu-case", action="store_true",
                     help="one compress + one decompress of gate_proj (14336x4096), for ncu captures")
     args = ap.parse_args()
@@ -487,11 +507,13 @@ def main():
 
     # side measurement (outside the timed region): the codec on the block's
     # FP4 block scale factors (NVFP4-style E4M3 scales, one per 16 values)
-    fp4 = measure_fp4_scales(eh, synth, items, dev, stream)
-    kv_pages = measure_kv_pages(eh, synth, dev, stream)
-    # decompression into the operand buffers of the next GEMMs (prefetch ring)
-    prefetch = [measure_prefetch(eh, xs, outs, p, dev, t) for t in (1, 8192)]
-    zipfloat = measure_zipfloat(eh, xs, dev, stream)
+    fp4 = kv_pages = prefetch = zipfloat = None
+    if not args.no_side:
+        fp4 = measure_fp4_scales(eh, synth, items, dev, stream)
+        kv_pages = measure_kv_pages(eh, synth, dev, stream)
+        # decompression into the operand buffers of the next GEMMs (prefetch ring)
+        prefetch = [measure_prefetch(eh, xs, outs, p, dev, t) for t in (1, 8192)]
+        zipfloat = measure_zipfloat(eh, xs, dev, stream)
 
     if rank == 0:
         peak, peak_kind = hbm_peak()
