@@ -179,6 +179,53 @@ def cpu_baseline_oracle(items, budget_s=12.0):
                       f" on one host core, {dt:.1f} s"}
 
 
+_start_barrier = None
+
+
+def _oracle_worker_init(barrier):
+    global _start_barrier
+    _start_barrier = barrier
+
+
+def _oracle_round_trip(index, parts):
+    """Slice `index` of `parts` equal runs of whole chunks of q_proj through
+    the oracle as a tensor of its own, timed from a barrier that all workers
+    pass together once their inputs exist; returns (BF16 bytes moved both
+    ways, start time, end time)."""
+    from exponent_entropy_coding_b200 import synth
+    from oracle import ehref
+    ehref.lib()
+    _, x = synth.llama8b_block(seed=2, scale=1, count=1)[0]
+    chunks = x.size // 65536
+    lo, hi = index * chunks // parts * 65536, (index + 1) * chunks // parts * 65536
+    x = np.ascontiguousarray(x[lo:hi])
+    _start_barrier.wait()
+    t0 = time.perf_counter()
+    c = ehref.compress(ehref.BF16, x)
+    y = ehref.decompress(c)
+    t1 = time.perf_counter()
+    assert np.array_equal(y, x)
+    return 2 * 2 * x.size, t0, t1
+
+
+def cpu_baseline_oracle_parallel():
+    """The oracle as it stands on T host cores ("oracle x T"): T spawned
+    workers each round-trip an equal run of whole chunks of q_proj (16.8 M
+    values) as their own tensor, side by side; the value is all their bytes
+    over the time from the common start to the last finish."""
+    import multiprocessing as mp
+    T = max(1, min(16, os.cpu_count() or 1))
+    ctx = mp.get_context("spawn")
+    barrier = ctx.Barrier(T)
+    with ctx.Pool(T, initializer=_oracle_worker_init, initargs=(barrier,)) as pool:
+        res = pool.starmap(_oracle_round_trip, [(i, T) for i in range(T)], chunksize=1)
+    nbytes = sum(r[0] for r in res)
+    dt = max(r[2] for r in res) - min(r[1] for r in res)
+    return {"value": nbytes / dt / 1e9, "unit": "GB/s", "cores": T, "kind": "oracle",
+            "sample": f"q_proj (16.8 M values) in {T} runs of whole chunks, one per process, compress+decompress "
+                      f"started together, {dt:.2f} s"}
+
+
 def run_ncu_case():
     """Small case for profiler captures: gate_proj alone (117 MB of BF16, more
     than the 126 MB L2 once its compressed form is counted), compressed once
@@ -561,6 +608,7 @@ def main():
         }
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline_oracle(items)
+            line["cpu_baseline_parallel"] = cpu_baseline_oracle_parallel()
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()
