@@ -553,18 +553,19 @@ __device__ __forceinline__ uint32_t exp_of(const uint4 &p, const uint4 &q, int j
 
 // ORs the `nbits` (<= 32) code bits held right-aligned in `acc` into the
 // ring at stream bit `pos`.
-__device__ __forceinline__ void ring_or(uint32_t *ring, uint64_t pos, uint32_t acc, uint32_t nbits) {
-  const uint32_t s = (uint32_t)(pos & 31);
-  const uint64_t w = pos >> 5;
+// Ring positions are bits relative to the start of the stream word that
+// holds the range's first bit (32-bit arithmetic; a range is one chunk or
+// page).  Ring word k is stream word (bit0 >> 5) + k, at slot k & kRingMask.
+__device__ __forceinline__ void ring_or(uint32_t *ring, uint32_t pos, uint32_t acc, uint32_t nbits) {
+  const uint32_t s = pos & 31, w = pos >> 5;
   const uint64_t y = (uint64_t)acc << (64 - s - nbits);
   atomicOr(&ring[w & kRingMask], (uint32_t)(y >> 32));
   if (s + nbits > 32) atomicOr(&ring[(w + 1) & kRingMask], (uint32_t)y);
 }
 
-// ORs the low nbits (1..64) of (hi:lo) into the ring at stream bit pos.
-__device__ __forceinline__ void ring_or64(uint32_t *ring, uint64_t pos, uint32_t hi, uint32_t lo, uint32_t nbits) {
-  const uint32_t s = (uint32_t)(pos & 31);
-  const uint64_t w = pos >> 5;
+// ORs the low nbits (1..64) of (hi:lo) into the ring at relative bit pos.
+__device__ __forceinline__ void ring_or64(uint32_t *ring, uint32_t pos, uint32_t hi, uint32_t lo, uint32_t nbits) {
+  const uint32_t s = pos & 31, w = pos >> 5;
   const uint64_t L = (((uint64_t)hi << 32) | lo) << (64 - nbits);  // left-aligned
   atomicOr(&ring[w & kRingMask], (uint32_t)(L >> (32 + s)));
   if (s + nbits > 32) atomicOr(&ring[(w + 1) & kRingMask], (uint32_t)(L >> s));
@@ -579,8 +580,11 @@ template <int DT>
 __device__ void encode_range(const uint2 *tab, const uint8_t *in, uint32_t cnt, uint64_t bit0, uint64_t bit1,
                              uint32_t *gs, uint32_t *ring, uint32_t *wsum, bool exclusive) {
   const int tid = threadIdx.x;
-  uint64_t tile_base = bit0;           // stream bit where the current tile starts
-  uint64_t wdone = bit0 >> 5;          // first stream word not yet written out
+  const uint64_t gw0 = bit0 >> 5;             // stream word of relative word 0
+  const uint32_t r0 = (uint32_t)(bit0 & 31);  // relative bit of the range's first code
+  const uint32_t rend = r0 + (uint32_t)(bit1 - bit0);
+  uint32_t tile_base = r0;  // relative bit where the current tile starts
+  uint32_t wdone = 0;       // first relative word not yet written out
   uint4 np, nq;
   load_exps<DT>(in, tid * kEncPerThread, cnt, np, nq);
   for (uint32_t t0 = 0; t0 < cnt; t0 += kEncTile) {
@@ -611,14 +615,14 @@ __device__ void encode_range(const uint2 *tab, const uint8_t *in, uint32_t cnt, 
     }
     uint32_t total;
     const uint32_t excl = block_excl_scan1(tot[0] + tot[1], wsum, &total);
-    uint64_t pos = tile_base + excl;
+    uint32_t pos = tile_base + excl;
     #pragma unroll
     for (int h = 0; h < 2; h++) {
       if (tot[h] == 0) continue;
       if (tot[h] <= 64) {
         ring_or64(ring, pos, hi[h], lo[h], tot[h]);
       } else {
-        uint64_t pp = pos;
+        uint32_t pp = pos;
         for (int j = 8 * h; j < 8 * h + 8; j++) {
           uint2 cl = tab[exp_of<DT>(p, q, j)];
           if (idx + j >= cnt || cl.y == 0) continue;
@@ -631,14 +635,15 @@ __device__ void encode_range(const uint2 *tab, const uint8_t *in, uint32_t cnt, 
     __syncthreads();
     tile_base += total;
     const bool last = t0 + kEncTile >= cnt;
-    const uint64_t wend = last ? (bit1 + 31) >> 5 : tile_base >> 5;
-    for (uint64_t wi = wdone + tid; wi < wend; wi += kThreads) {
-      const uint32_t slot = (uint32_t)(wi & kRingMask);
+    const uint32_t wend = last ? (rend + 31) >> 5 : tile_base >> 5;
+    for (uint32_t wi = wdone + tid; wi < wend; wi += kThreads) {
+      const uint32_t slot = wi & kRingMask;
       const uint32_t val = bswap32(ring[slot]);
       ring[slot] = 0u;
-      const bool edge = !exclusive && ((wi << 5) < bit0 || ((wi + 1) << 5) > bit1);
-      if (edge) atomicOr(gs + wi, val);
-      else gs[wi] = val;
+      // the first and last words may hold bits of the neighbouring ranges
+      const bool edge = !exclusive && ((wi == 0 && r0 != 0) || ((wi + 1) << 5) > rend);
+      if (edge) atomicOr(gs + gw0 + wi, val);
+      else gs[gw0 + wi] = val;
     }
     wdone = wend;
   }
