@@ -371,6 +371,30 @@ int ehref_encode(int dtype, const void *in, uint64_t n, uint32_t chunk,
   return EHREF_OK;
 }
 
+int ehref_value_index(int dtype, const void *in, uint64_t n, uint32_t chunk,
+                      const uint8_t *len, uint32_t *index) {
+  if (!alphabet_of(dtype) || chunk == 0 || chunk % EHREF_INDEX_STRIDE) return EHREF_EINVAL;
+  const uint64_t C = ehref_num_chunks(n, chunk);
+  const uint32_t per = chunk / EHREF_INDEX_STRIDE;
+  for (uint64_t c = 0; c < C; c++) {
+    uint32_t bits = 0;  // from the chunk's first bit
+    for (uint64_t j = 0; j < chunk; j++) {
+      const uint64_t i = c * chunk + j;
+      if (j % EHREF_INDEX_STRIDE == 0) index[c * per + j / EHREF_INDEX_STRIDE] = bits;
+      if (i < n) {
+        uint8_t e, sm;
+        split_one(dtype, load_elem(dtype, in, i), &e, &sm);
+        if (len[e] == 0) return EHREF_EINVAL;
+        bits += len[e];
+      }
+    }
+    // entries past the last value of a short chunk: the chunk's total bits
+    for (uint32_t k = 0; k < per; k++)
+      if (c * chunk + (uint64_t)k * EHREF_INDEX_STRIDE >= n) index[c * per + k] = bits;
+  }
+  return EHREF_OK;
+}
+
 int ehref_compress(int dtype, const void *in, uint64_t n, uint32_t chunk,
                    int Lmax, uint8_t *len, uint32_t *code, uint64_t *off,
                    uint8_t *stream, uint64_t cap, uint8_t *sm_packed,

@@ -111,6 +111,18 @@ int ehref_decompress(int dtype, uint64_t n, uint32_t chunk, const uint8_t *len,
                      const uint8_t *stream, uint64_t stream_bytes,
                      const uint8_t *sm_packed, void *out);
 
+/* Optional value index (an auxiliary position array in the spirit of the
+ * DFloat11 article's per-thread position variables, "方法介绍", kept outside
+ * the stream): for chunk c and k = 0 .. chunk/EHREF_INDEX_STRIDE - 1, entry
+ * index[c * (chunk / EHREF_INDEX_STRIDE) + k] is the bit offset, from the
+ * chunk's first bit, of the code of value k * EHREF_INDEX_STRIDE of the
+ * chunk; entries past the chunk's last value hold the chunk's total bits.
+ * With it a decoder can start every run of EHREF_INDEX_STRIDE values at a
+ * known bit without first finding code boundaries. */
+#define EHREF_INDEX_STRIDE 128
+int ehref_value_index(int dtype, const void *in, uint64_t n, uint32_t chunk,
+                      const uint8_t *len, uint32_t *index);
+
 /* Fixed-slot page store (online K/V cache compression).  A page of n values
  * (one chunk; 64 tokens x 8 heads x 128 dims = 65,536 for Llama-3.1-8B K/V) is
  * coded with a FROZEN codebook (len/code from earlier data) into a slot of

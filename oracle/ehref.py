@@ -52,6 +52,7 @@ def lib():
             "ehref_decompress": (i32, [i32, u64, u32, vp, vp, vp, vp, u64, vp, vp]),
             "ehref_page_encode": (i32, [i32, vp, u64, vp, vp, vp, u64, vp, vp, vp, vp]),
             "ehref_page_decode": (i32, [i32, u64, vp, vp, vp, u64, u64, i32, vp, vp, vp]),
+            "ehref_value_index": (i32, [i32, vp, u64, u32, vp, vp]),
             "zfref_blocks": (u64, [u64]),
             "zfref_block_base": (i32, [vp, u32, vp, vp]),
             "zfref_compress": (i32, [vp, u64, vp, vp, vp, vp, vp, u64, vp]),
@@ -176,6 +177,19 @@ def encode(dtype, x, chunk, lengths, codes):
     _check(lib().ehref_encode(dtype, _p(x), n, chunk, _p(ln), _p(cd), _p(off), _p(stream),
                               cap, C.byref(bits)))
     return off, stream[: (bits.value + 7) // 8].copy(), bits.value
+
+
+INDEX_STRIDE = 128
+
+
+def value_index(dtype, x, lengths, chunk=65536):
+    """Bit offset of every INDEX_STRIDE-th value of each chunk (format in ehref.h)."""
+    x = np.ascontiguousarray(x, dtype=elem_dtype(dtype))
+    nc = num_chunks(x.size, chunk)
+    idx = np.zeros(max(nc * (chunk // INDEX_STRIDE), 1), np.uint32)
+    _check(lib().ehref_value_index(dtype, _p(x), x.size, chunk,
+                                   _p(np.ascontiguousarray(lengths, np.uint8)), _p(idx)))
+    return idx[: nc * (chunk // INDEX_STRIDE)]
 
 
 def compress(dtype, x, chunk=65536, lmax=32):
