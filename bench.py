@@ -326,6 +326,47 @@ def measure_kv_pages(eh, synth, dev, stream, reps=20):
             "slot_bytes": 28 * 1024}
 
 
+def measure_indexed(eh, p, xs, dev, stream, reps=50):
+    """The block with the optional value index (4 bytes per 128 values beside
+    the stream): compress writes it, decompress starts every run of 128 values
+    at its recorded bit instead of finding code boundaries.  CUDA events;
+    GB/s of BF16 bytes, the decoder's fraction of the measured HBM bandwidth
+    in algorithmic bytes (the index read counted), and the size ratio with
+    the index."""
+    import torch
+    outs = [eh.alloc_compressed(p, x.numel(), dev, index=True) for x in xs]
+    ys = [torch.empty_like(x) for x in xs]
+    wsc = torch.empty(eh.compress_batch_workspace(p, [x.numel() for x in xs]), dtype=torch.uint8, device=dev)
+    wsd = torch.empty(eh.decompress_workspace(p, len(xs)), dtype=torch.uint8, device=dev)
+    bits = torch.zeros(len(xs), dtype=torch.int64, device=dev)
+    eh.compress_batch(p, xs, outs, wsc)
+    eh.decompress_batch(p, outs, ys, wsd)
+    assert eh.get_status(wsd) == eh.EH_OK and all(torch.equal(x, y) for x, y in zip(xs, ys))
+    in_bytes = sum(2 * x.numel() for x in xs)
+    comp = sum(o.compressed_bytes() for o in outs)
+    alg = sum(o.stream_bytes() + o.sign_mant.numel() + 8 * o.chunk_bit_off.numel() + 4 * o.value_index.numel()
+              for o in outs) + in_bytes
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+    for _ in range(3):
+        eh.compress_batch(p, xs, outs, wsc, bits_dev=bits)
+        eh.decompress_batch(p, outs, ys, wsd)
+    ev[0].record(stream)
+    for _ in range(reps):
+        eh.compress_batch(p, xs, outs, wsc, bits_dev=bits)
+    ev[1].record(stream)
+    for _ in range(reps):
+        eh.decompress_batch(p, outs, ys, wsd)
+    ev[2].record(stream)
+    torch.cuda.synchronize()
+    assert eh.get_status(wsd) == eh.EH_OK and all(torch.equal(x, y) for x, y in zip(xs, ys))
+    enc = ev[0].elapsed_time(ev[1]) / reps * 1e-3
+    dec = ev[1].elapsed_time(ev[2]) / reps * 1e-3
+    peak, _ = hbm_peak()
+    return {"kind": "value index beside the stream (bit offset of every 128th value of each chunk)",
+            "encode_gbs": in_bytes / enc / 1e9, "decode_gbs": in_bytes / dec / 1e9,
+            "decode_frac": alg / dec / 1e9 / peak, "size_ratio": comp / in_bytes}
+
+
 def measure_zipfloat(eh, xs, dev, stream, reps=20):
     """The ZipFloat comparison codec on the same block (seven calls each way
     per repetition, CUDA events): GB/s of BF16 bytes and the size ratio."""
@@ -554,8 +595,9 @@ def main():
 
     # side measurement (outside the timed region): the codec on the block's
     # FP4 block scale factors (NVFP4-style E4M3 scales, one per 16 values)
-    fp4 = kv_pages = prefetch = zipfloat = None
+    fp4 = kv_pages = prefetch = zipfloat = indexed = None
     if not args.no_side:
+        indexed = measure_indexed(eh, p, xs, dev, stream)
         fp4 = measure_fp4_scales(eh, synth, items, dev, stream)
         kv_pages = measure_kv_pages(eh, synth, dev, stream)
         # decompression into the operand buffers of the next GEMMs (prefetch ring)
@@ -600,6 +642,7 @@ def main():
             "gpu_launches": 6 * args.steps,
             "fp4_scales": fp4,
             "kv_pages": kv_pages,
+            "indexed": indexed,
             "zipfloat": zipfloat,
             "prefetch": {"workload": "8 layers of Llama-3.1-8B block linears (q,k,v,o,gate,up,down) "
                                      "on `tokens` BF16 rows; weights decoded into a 2-slot ring",

@@ -139,7 +139,8 @@ eh_status prepare_compress(const eh_plan_t *plan, int k, const void *const *ins,
     const uint64_t n = o.n;
     if (o.dtype != plan->dtype || n > (1ull << 40)) return EH_ERR_INVALID_ARG;
     if (!o.code_len || !o.code || !o.chunk_bit_off) return EH_ERR_INVALID_ARG;
-    if (((uintptr_t)o.code & 3u) || ((uintptr_t)o.chunk_bit_off & 7u)) return EH_ERR_INVALID_ARG;
+    if (((uintptr_t)o.code & 3u) || ((uintptr_t)o.chunk_bit_off & 7u) || ((uintptr_t)o.value_index & 3u))
+      return EH_ERR_INVALID_ARG;
     const bool has_sm = plan->dtype != EH_BYTES;
     if (n > 0 && (!ins[i] || !o.exp_stream || (has_sm && !o.sign_mant))) return EH_ERR_INVALID_ARG;
     if (n > 0 && (!aligned16(ins[i]) || !aligned16(o.exp_stream) || (has_sm && !aligned16(o.sign_mant))))
@@ -180,6 +181,7 @@ eh_status prepare_compress(const eh_plan_t *plan, int k, const void *const *ins,
     it.stream = o.exp_stream;
     it.stream_cap = o.exp_stream_cap;
     it.sm = o.sign_mant;
+    it.vindex = o.value_index;
     it.counts = (uint64_t *)(ws + kHeader + (uint64_t)i * kCountsBytes);
     it.bits_out = bits_ws + i;
     it.bits_dev = bits_dev ? bits_dev + i : nullptr;
@@ -305,7 +307,9 @@ eh_status eh::decompress_impl(const eh_plan_t *plan, int k, const eh_compressed_
     const uint32_t first = firsts ? firsts[i] : 0u;
     const uint32_t count = counts ? counts[i] : (uint32_t)C;
     if ((uint64_t)first + count > C) return EH_ERR_INVALID_ARG;
-    if (!c.code_len || !c.code || !c.chunk_bit_off || ((uintptr_t)c.chunk_bit_off & 7u)) return EH_ERR_INVALID_ARG;
+    if (!c.code_len || !c.code || !c.chunk_bit_off || ((uintptr_t)c.chunk_bit_off & 7u) ||
+        ((uintptr_t)c.value_index & 3u))
+      return EH_ERR_INVALID_ARG;
     if (count > 0) {
       const bool has_sm = plan->dtype != EH_BYTES;
       if (!outs[i] || !c.exp_stream || (has_sm && !c.sign_mant)) return EH_ERR_INVALID_ARG;
@@ -326,6 +330,7 @@ eh_status eh::decompress_impl(const eh_plan_t *plan, int k, const eh_compressed_
     it.stream = c.exp_stream;
     it.stream_cap = c.exp_stream_cap;
     it.sm = c.sign_mant;
+    it.vindex = c.value_index;
     it.lut = ws + kHeader + (uint64_t)i * kLutBytes;
     chunk0 += count;
   }

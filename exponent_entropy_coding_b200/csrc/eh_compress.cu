@@ -578,7 +578,8 @@ __device__ __forceinline__ void ring_or64(uint32_t *ring, uint32_t pos, uint32_t
 // words unless `exclusive`, when the range owns every word it touches.
 template <int DT>
 __device__ void encode_range(const uint2 *tab, const uint8_t *in, uint32_t cnt, uint64_t bit0, uint64_t bit1,
-                             uint32_t *gs, uint32_t *ring, uint32_t *wsum, bool exclusive) {
+                             uint32_t *gs, uint32_t *ring, uint32_t *wsum, bool exclusive,
+                             uint32_t *vindex = nullptr) {
   const int tid = threadIdx.x;
   const uint64_t gw0 = bit0 >> 5;             // stream word of relative word 0
   const uint32_t r0 = (uint32_t)(bit0 & 31);  // relative bit of the range's first code
@@ -616,6 +617,9 @@ __device__ void encode_range(const uint2 *tab, const uint8_t *in, uint32_t cnt, 
     uint32_t total;
     const uint32_t excl = block_excl_scan1(tot[0] + tot[1], wsum, &total);
     uint32_t pos = tile_base + excl;
+    // value index: where every kIndexStride-th value's code starts, from the
+    // range's first bit
+    if (vindex && (idx % kIndexStride) == 0 && idx < cnt) vindex[idx / kIndexStride] = pos - r0;
     #pragma unroll
     for (int h = 0; h < 2; h++) {
       if (tot[h] == 0) continue;
@@ -674,7 +678,15 @@ __global__ void __launch_bounds__(kThreads, 2) encode_kernel(const __grid_consta
   load_code_table<DT>(tab, I.code_len, I.code);
   const uint8_t *in = (const uint8_t *)I.in + i0 * (DT == EH_BF16 ? 2 : 1);
   __syncthreads();
-  encode_range<DT>(tab, in, cnt, I.off[c], I.off[c + 1], (uint32_t *)I.stream, ring, wsum, false);
+  uint32_t *vindex = I.vindex ? I.vindex + (uint64_t)c * (b.chunk_elems / kIndexStride) : nullptr;
+  encode_range<DT>(tab, in, cnt, I.off[c], I.off[c + 1], (uint32_t *)I.stream, ring, wsum, false, vindex);
+  if (vindex) {
+    // entries past a short last chunk's end: the chunk's bit count
+    const uint32_t bits = (uint32_t)(I.off[c + 1] - I.off[c]);
+    for (uint32_t k = (cnt + kIndexStride - 1) / kIndexStride + threadIdx.x; k < b.chunk_elems / kIndexStride;
+         k += kThreads)
+      vindex[k] = bits;
+  }
 }
 
 // ---------------------------------------------------------------- pages

@@ -610,6 +610,86 @@ __device__ bool decode_chunk(GroupSmem &G, const DecodeTables &T, const uint32_t
   return true;
 }
 
+// Bits taken by the first r (1..4) of the codes that start at the set bits
+// of bm (offsets from the lookup position), when the lookup holds kk >= r
+// complete codes ending at bit nb.
+__device__ __forceinline__ uint32_t bits_of_first(uint32_t bm, uint32_t r, uint32_t kk, uint32_t nb) {
+  if (r >= kk) return nb;
+  #pragma unroll
+  for (int i = 0; i < 4; i++)
+    if ((uint32_t)i < r) bm &= bm - 1u;  // drop the first r code starts
+  return __ffs(bm) - 1u;                  // the start of code r + 1
+}
+
+// Steps 2-5 with a value index: thread t writes values [128t, 128t + 128) of
+// the chunk from the bit vidx[t] on; no boundary search, no count, no scan.
+// The run must end exactly at the next entry (or the chunk's end), else the
+// chunk is reported corrupt.  Returns false (group-uniform) if corrupt.
+template <bool kSmem>
+__device__ bool decode_chunk_indexed(GroupSmem &G, const DecodeTables &T, const uint32_t *words, uint32_t rel0,
+                                     uint32_t nbits, uint32_t cnt, uint32_t id, uint32_t gtid,
+                                     const uint32_t *vidx, uint32_t per) {
+  Peek<kSmem> peek{words};
+  const uint32_t j0 = gtid * kIndexStride;
+  uint32_t start = 0, stop = 0, n = 0;
+  bool bad = false;
+  if (gtid < per && j0 < cnt) {
+    n = min(kIndexStride, cnt - j0);
+    start = __ldg(vidx + gtid);
+    stop = (gtid + 1 < per && j0 + kIndexStride < cnt) ? __ldg(vidx + gtid + 1) : nbits;
+    bad = start > stop || stop > nbits || stop - start < n || stop - start > 32u * n;
+  }
+  // also orders the caller's clearing of the exponent buffer before the writes
+  if (gsync_or(id, bad)) return false;
+
+  ExpWriter out;
+  out.init(G.exps, j0);
+  uint32_t pos = start, rem8 = 8 * n;
+  while (rem8 && pos < stop) {
+    const uint32_t x = peek(rel0 + pos);
+    const uint32_t i1 = lut_index(x);
+    const uint32_t m1 = T.l1meta[i1];
+    const uint32_t k1 = (m1 >> 1) & 0x38u, nb1 = m1 & 15u;  // k1: 8 * codes
+    if (!k1) {
+      uint32_t syms, nb;
+      if (!decode_long(T, x, m1, syms, nb)) { bad = true; break; }
+      pos += nb;
+      out.put(syms, 8);
+      rem8 -= 8;
+      continue;
+    }
+    const uint32_t s1 = T.l1sym[i1];
+    if (k1 >= rem8) {  // the run's last codes
+      out.put(s1 & low_bytes_mask(rem8), rem8);
+      pos += bits_of_first((m1 >> 7) & 0xFFFu, rem8 >> 3, k1 >> 3, nb1);
+      rem8 = 0;
+      break;
+    }
+    out.put(s1, k1);
+    rem8 -= k1;
+    const uint32_t i2 = lut_index(x << nb1);
+    const uint32_t m2 = T.l1meta[i2];
+    const uint32_t k2 = (m2 >> 1) & 0x38u, nb2 = m2 & 15u;
+    if (!k2) {
+      pos += nb1;
+      continue;
+    }
+    const uint32_t s2 = T.l1sym[i2];
+    if (k2 >= rem8) {
+      out.put(s2 & low_bytes_mask(rem8), rem8);
+      pos += nb1 + bits_of_first((m2 >> 7) & 0xFFFu, rem8 >> 3, k2 >> 3, nb2);
+      rem8 = 0;
+      break;
+    }
+    out.put(s2, k2);
+    rem8 -= k2;
+    pos += nb1 + nb2;
+  }
+  out.finish();
+  bad = bad || rem8 != 0 || pos != stop;
+  return !gsync_or(id, bad);
+}
+
 // (sign+mantissa, exponent) byte pairs [s0, e0, s1, e1] -> two BF16 values
 __device__ __forceinline__ uint32_t bf16_merge2(uint32_t p) {
   return (p & 0x007F007Fu) | ((p >> 1) & 0x7F807F80u) | ((p & 0x00800080u) << 8);
@@ -791,10 +871,17 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
         // the exponent words are OR-ed in: clear them (ordered before the
         // writing pass by the decoder's barriers)
         for (uint32_t i = gtid; i < kExpBytes / 16; i += kGroupThreads) ((uint4 *)G.exps)[i] = make_uint4(0, 0, 0, 0);
-        if (ci.fits) ok = decode_chunk<true>(G, S.tabs, G.stage, ci.rel0, ci.nbits, cnt, id, gtid, &timeout);
-        else
-          ok = decode_chunk<false>(G, S.tabs, (const uint32_t *)(I.stream + ci.lo), ci.rel0, ci.nbits, cnt, id,
-                                   gtid, &timeout);
+        const uint32_t per = b.chunk_elems / kIndexStride;
+        const uint32_t *vidx = (I.vindex && !I.page_meta) ? I.vindex + (uint64_t)ci.c * per : nullptr;
+        const uint32_t *gw = (const uint32_t *)(I.stream + ci.lo);
+        if (vidx) {
+          if (ci.fits) ok = decode_chunk_indexed<true>(G, S.tabs, G.stage, ci.rel0, ci.nbits, cnt, id, gtid, vidx, per);
+          else ok = decode_chunk_indexed<false>(G, S.tabs, gw, ci.rel0, ci.nbits, cnt, id, gtid, vidx, per);
+        } else if (ci.fits) {
+          ok = decode_chunk<true>(G, S.tabs, G.stage, ci.rel0, ci.nbits, cnt, id, gtid, &timeout);
+        } else {
+          ok = decode_chunk<false>(G, S.tabs, gw, ci.rel0, ci.nbits, cnt, id, gtid, &timeout);
+        }
         if (!ok && gtid == 0) set_status(b.status, timeout ? kFlagTimeout | kFlagCorrupt : kFlagCorrupt);
       } else if (gtid == 0 && !S.abort_flag) {
         set_status(b.status, kFlagCorrupt);

@@ -28,6 +28,8 @@ constexpr uint32_t kFlagNoRoom = 8u;   // raw page pool exhausted
 __host__ __device__ inline int alphabet_of(int dtype) { return dtype == EH_FP8_E4M3 ? 16 : 256; }
 
 // Per-tensor part of a launch.
+constexpr uint32_t kIndexStride = EH_INDEX_STRIDE;  // values per value-index entry
+
 struct Item {
   const void *in;          // compress: raw values
   void *out;               // decompress: output values
@@ -43,6 +45,7 @@ struct Item {
   uint8_t *stream;         // exp_stream
   uint64_t stream_cap;     // bytes
   uint8_t *sm;             // sign_mant
+  uint32_t *vindex;        // optional value index [total_chunks][chunk_elems / kIndexStride]
   // workspace views
   uint64_t *counts;        // compress: [256] global histogram
   uint32_t *chist;         // compress: [total_chunks][A] per-chunk histograms

@@ -58,7 +58,8 @@ class eh_compressed_t(C.Structure):
     _fields_ = [("dtype", C.c_int32), ("n_chunks", C.c_uint32), ("n", C.c_uint64),
                 ("code_len", C.c_void_p), ("code", C.c_void_p), ("chunk_bit_off", C.c_void_p),
                 ("exp_stream", C.c_void_p), ("exp_stream_cap", C.c_uint64),
-                ("sign_mant", C.c_void_p), ("exp_stream_bits", C.c_uint64)]
+                ("sign_mant", C.c_void_p), ("exp_stream_bits", C.c_uint64),
+                ("value_index", C.c_void_p)]
 
 
 class eh_zf_t(C.Structure):
@@ -184,6 +185,7 @@ class Compressed:
     exp_stream: torch.Tensor     # uint8[cap]
     sign_mant: torch.Tensor      # uint8[n or ceil(n/2)]
     exp_stream_bits: int = 0
+    value_index: Optional[torch.Tensor] = None  # int32[C * chunk / 128] (uint32 values) or None
 
     @property
     def n_chunks(self) -> int:
@@ -193,9 +195,10 @@ class Compressed:
         return (self.exp_stream_bits + 7) // 8
 
     def compressed_bytes(self) -> int:
-        """Stored size: exponent stream + sign/mantissa + offsets + codebook."""
+        """Stored size: exponent stream + sign/mantissa + offsets + codebook
+        (+ the value index when there is one)."""
         return (self.stream_bytes() + self.sign_mant.numel() + 8 * self.chunk_bit_off.numel()
-                + self.code_len.numel())
+                + self.code_len.numel() + (4 * self.value_index.numel() if self.value_index is not None else 0))
 
     def struct(self) -> eh_compressed_t:
         s = eh_compressed_t()
@@ -209,10 +212,16 @@ class Compressed:
         s.exp_stream_cap = self.exp_stream.numel()
         s.sign_mant = self.sign_mant.data_ptr() if self.sign_mant.numel() else None
         s.exp_stream_bits = self.exp_stream_bits
+        s.value_index = self.value_index.data_ptr() if self.value_index is not None else None
         return s
 
 
-def alloc_compressed(p: eh_plan_t, n: int, device) -> Compressed:
+EH_INDEX_STRIDE = 128
+
+
+def alloc_compressed(p: eh_plan_t, n: int, device, index: bool = False) -> Compressed:
+    """Buffers for one compressed tensor; `index` adds the optional value
+    index (4 bytes per EH_INDEX_STRIDE values)."""
     cap, smb, _ = compress_bound(p, n)
     A = alphabet(p.dtype)
     nc = -(-n // p.chunk_elems)
@@ -223,7 +232,9 @@ def alloc_compressed(p: eh_plan_t, n: int, device) -> Compressed:
         code=torch.zeros(A, dtype=torch.int32, device=dev),
         chunk_bit_off=torch.zeros(nc + 1, dtype=torch.int64, device=dev),
         exp_stream=torch.empty(cap if n else 0, dtype=torch.uint8, device=dev),
-        sign_mant=torch.empty(smb, dtype=torch.uint8, device=dev))
+        sign_mant=torch.empty(smb, dtype=torch.uint8, device=dev),
+        value_index=(torch.zeros(max(nc * (p.chunk_elems // EH_INDEX_STRIDE), 1), dtype=torch.int32, device=dev)
+                     if index else None))
 
 
 def _raw(x: torch.Tensor) -> torch.Tensor:
@@ -251,13 +262,14 @@ def compress_batch(p: eh_plan_t, xs: List[torch.Tensor], outs: List[Compressed],
 
 
 def compress(x: torch.Tensor, p: Optional[eh_plan_t] = None, workspace: Optional[torch.Tensor] = None,
-             stream=None) -> Compressed:
-    """Compresses one BF16 / FP8 E4M3 tensor (or its raw uint16 / uint8 bits)."""
+             stream=None, index: bool = False) -> Compressed:
+    """Compresses one BF16 / FP8 E4M3 tensor (or its raw uint16 / uint8 bits);
+    `index` also writes the optional value index."""
     x = _raw(x)
     if p is None:
         p = plan(dtype_code(x.dtype))
     n = x.numel()
-    out = alloc_compressed(p, n, x.device)
+    out = alloc_compressed(p, n, x.device, index=index)
     if workspace is None:
         workspace = torch.empty(compress_bound(p, n)[2], dtype=torch.uint8, device=x.device)
     s = out.struct()

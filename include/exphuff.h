@@ -111,7 +111,20 @@ typedef struct {
   uint64_t exp_stream_cap;  /* bytes; >= eh_compress_bound's stream_cap      */
   uint8_t *sign_mant;       /* device, n (BF16), ceil(n/2) (FP8), 0 (BYTES)  */
   uint64_t exp_stream_bits; /* total code bits (host copy)                   */
+  uint32_t *value_index;    /* device, optional (NULL: none); see below      */
 } eh_compressed_t;
+
+/* Optional value index, outside the stream: entry c * (chunk_elems /
+ * EH_INDEX_STRIDE) + k is the bit offset, from chunk c's first bit, of the
+ * code of value k * EH_INDEX_STRIDE of the chunk; entries past a short last
+ * chunk's end hold that chunk's bit count.  n_chunks * chunk_elems /
+ * EH_INDEX_STRIDE u32 entries (4 bytes per 128 values, +1.6 % on BF16).
+ * eh_compress fills it when value_index is non-NULL; eh_decompress then
+ * starts every run of EH_INDEX_STRIDE values at its recorded bit instead of
+ * finding code boundaries first (the DFloat11 article's per-thread position
+ * variables, "方法介绍", kept beside the format rather than in it).  An index
+ * that does not match the stream is reported as EH_ERR_CORRUPT. */
+#define EH_INDEX_STRIDE 128
 
 /* Fills *plan.  chunk_elems = 0 selects 65536; max_code_len = 0 selects 32.
  * Returns EH_ERR_UNSUPPORTED for other chunk sizes or limits. */
