@@ -395,6 +395,7 @@ __device__ __forceinline__ uint32_t group_excl_scan_or(uint32_t v, bool pred, ui
 // Packs decoded exponents four to a word into the exponent buffer, which
 // is zeroed before each chunk.  Words are combined with OR, so the words a run
 // shares with its neighbours need no special case.
+template <bool kOwn = false>
 struct ExpWriter {
   uint32_t *words;  // exponent buffer as words
   uint32_t wi;      // word being filled (exponents 4*wi .. 4*wi+3)
@@ -406,13 +407,19 @@ struct ExpWriter {
     s = 8 * (j & 3u);
     acc = 0;
   }
+  // kOwn: the run owns every word it touches (it starts on a word), so the
+  // words are stored, not OR-ed into a cleared buffer
+  __device__ __forceinline__ void store(uint32_t v) {
+    if (kOwn) words[wi + (wi >> 5)] = v;  // word wi of the padded rows
+    else atomicOr(words + wi + (wi >> 5), v);
+  }
   // up to four symbols, first in the low byte, zero above; k8 = 8 * count
   __device__ __forceinline__ void put(uint32_t syms, uint32_t k8) {
     const uint32_t lo = acc | (syms << s);
     const uint32_t hi = __funnelshift_l(syms, 0u, s);  // the bytes past the word; none for s = 0
     s += k8;
     if (s >= 32) {
-      atomicOr(words + wi + (wi >> 5), lo);  // word wi of the padded rows
+      store(lo);
       wi++;
       acc = hi;
       s -= 32;
@@ -421,7 +428,7 @@ struct ExpWriter {
     }
   }
   __device__ __forceinline__ void finish() {
-    if (s) atomicOr(words + wi + (wi >> 5), acc);
+    if (s) store(acc);
   }
 };
 
@@ -565,7 +572,7 @@ __device__ bool decode_chunk(GroupSmem &G, const DecodeTables &T, const uint32_t
 
   // 5. decode again from the true start, writing exactly the thread's my_n
   //    exponents (a count, not the window end, stops the loop)
-  ExpWriter out;
+  ExpWriter<> out;
   out.init(G.exps, o);
   pos = gtid == 0 ? 0u : G.ends[gtid - 1];
   uint32_t rem8 = 8 * my_n;  // exponent bits still to write
@@ -642,7 +649,7 @@ __device__ bool decode_chunk_indexed(GroupSmem &G, const DecodeTables &T, const 
   // also orders the caller's clearing of the exponent buffer before the writes
   if (gsync_or(id, bad)) return false;
 
-  ExpWriter out;
+  ExpWriter<true> out;  // runs start on multiples of 128 values: whole words
   out.init(G.exps, j0);
   uint32_t pos = start, rem8 = 8 * n;
   while (rem8 && pos < stop) {
@@ -868,11 +875,12 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
         for (uint32_t i = cnt / 16 * 16 + gtid; i < cnt; i += kGroupThreads) G.exps[exp_slot(i)] = src[i];
         gsync(id);
       } else if (ok) {
-        // the exponent words are OR-ed in: clear them (ordered before the
-        // writing pass by the decoder's barriers)
-        for (uint32_t i = gtid; i < kExpBytes / 16; i += kGroupThreads) ((uint4 *)G.exps)[i] = make_uint4(0, 0, 0, 0);
         const uint32_t per = b.chunk_elems / kIndexStride;
         const uint32_t *vidx = (I.vindex && !I.page_meta) ? I.vindex + (uint64_t)ci.c * per : nullptr;
+        // the search path ORs exponent words in: clear them (ordered before the
+        // writing pass by the decoder's barriers); indexed runs store whole words
+        if (!vidx)
+          for (uint32_t i = gtid; i < kExpBytes / 16; i += kGroupThreads) ((uint4 *)G.exps)[i] = make_uint4(0, 0, 0, 0);
         const uint32_t *gw = (const uint32_t *)(I.stream + ci.lo);
         if (vidx) {
           if (ci.fits) ok = decode_chunk_indexed<true>(G, S.tabs, G.stage, ci.rel0, ci.nbits, cnt, id, gtid, vidx, per);
