@@ -32,7 +32,7 @@ FALLBACK_HBM_GBS = 6650.0
 # DRAM traffic per decode launch on the full block, from one ncu capture
 # (dram__bytes_read.sum + dram__bytes_write.sum), valid only for the decoder
 # source it was taken on.
-DECODE_TRAFFIC = {"bytes": 292652032 + 374814976, "source_sha": "61288420b0d80077"}
+DECODE_TRAFFIC = {"bytes": 292758528 + 376947200, "source_sha": "4284ede2754d4c5f"}
 
 
 def decoder_source_sha():
@@ -187,7 +187,7 @@ def _oracle_worker_init(barrier):
     _start_barrier = barrier
 
 
-def _oracle_round_trip(index, parts):
+def _oracle_round_trip(index, parts, repeats):
     """Slice `index` of `parts` equal runs of whole chunks of q_proj through
     the oracle as a tensor of its own, timed from a barrier that all workers
     pass together once their inputs exist; returns (BF16 bytes moved both
@@ -201,29 +201,30 @@ def _oracle_round_trip(index, parts):
     x = np.ascontiguousarray(x[lo:hi])
     _start_barrier.wait()
     t0 = time.perf_counter()
-    c = ehref.compress(ehref.BF16, x)
-    y = ehref.decompress(c)
+    for _ in range(repeats):
+        c = ehref.compress(ehref.BF16, x)
+        y = ehref.decompress(c)
     t1 = time.perf_counter()
     assert np.array_equal(y, x)
-    return 2 * 2 * x.size, t0, t1
+    return repeats * 2 * 2 * x.size, t0, t1
 
 
-def cpu_baseline_oracle_parallel():
+def cpu_baseline_oracle_parallel(repeats=8):
     """The oracle as it stands on T host cores ("oracle x T"): T spawned
     workers each round-trip an equal run of whole chunks of q_proj (16.8 M
-    values) as their own tensor, side by side; the value is all their bytes
-    over the time from the common start to the last finish."""
+    values) as their own tensor `repeats` times, side by side; the value is
+    all their bytes over the time from the common start to the last finish."""
     import multiprocessing as mp
     T = max(1, min(16, os.cpu_count() or 1))
     ctx = mp.get_context("spawn")
     barrier = ctx.Barrier(T)
     with ctx.Pool(T, initializer=_oracle_worker_init, initargs=(barrier,)) as pool:
-        res = pool.starmap(_oracle_round_trip, [(i, T) for i in range(T)], chunksize=1)
+        res = pool.starmap(_oracle_round_trip, [(i, T, repeats) for i in range(T)], chunksize=1)
     nbytes = sum(r[0] for r in res)
     dt = max(r[2] for r in res) - min(r[1] for r in res)
     return {"value": nbytes / dt / 1e9, "unit": "GB/s", "cores": T, "kind": "oracle",
-            "sample": f"q_proj (16.8 M values) in {T} runs of whole chunks, one per process, compress+decompress "
-                      f"started together, {dt:.2f} s"}
+            "sample": f"q_proj (16.8 M values) in {T} runs of whole chunks, one per process, {repeats} "
+                      f"compress+decompress each, started together, {dt:.2f} s"}
 
 
 def run_ncu_case():
