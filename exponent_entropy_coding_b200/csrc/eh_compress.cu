@@ -59,6 +59,7 @@ __global__ void __launch_bounds__(kThreads, 2) hist_kernel(const __grid_constant
   for (int i = tid; i < A * 32; i += kThreads) h[i] = 0;
   __syncthreads();
   uint32_t *hl = h + lane;
+  uint8_t *hb = (uint8_t *)hl;
   if (DT == EH_BF16) {
     const uint16_t *in = (const uint16_t *)I.in + i0;
     uint8_t *smo = I.sm + i0;
@@ -71,11 +72,18 @@ __global__ void __launch_bounds__(kThreads, 2) hist_kernel(const __grid_constant
       uint32_t o[4];
       #pragma unroll
       for (int j = 0; j < 8; j++) {
-        atomicAdd(hl + (((w[j] >> 7) & 0xFFu) << 5), 1u);
-        atomicAdd(hl + (((w[j] >> 23) & 0xFFu) << 5), 1u);
+        // exponent e sits in bits 7..14 of each half: e << 7 is the byte
+        // offset of row e (32 counters of 4 bytes) in the lane's column
+        atomicAdd((uint32_t *)(hb + (w[j] & 0x7F80u)), 1u);
+        atomicAdd((uint32_t *)(hb + ((w[j] >> 16) & 0x7F80u)), 1u);
       }
       #pragma unroll
-      for (int j = 0; j < 4; j++) o[j] = bf16x2_sm(w[2 * j]) | (bf16x2_sm(w[2 * j + 1]) << 16);
+      for (int j = 0; j < 4; j++) {
+        // low bytes carry the mantissas, high bytes the signs (bit 7)
+        const uint32_t lows = __byte_perm(w[2 * j], w[2 * j + 1], 0x6420);
+        const uint32_t highs = __byte_perm(w[2 * j], w[2 * j + 1], 0x7531);
+        o[j] = (lows & 0x7F7F7F7Fu) | (highs & 0x80808080u);
+      }
       *(uint4 *)(smo + 16 * (uint64_t)v) = make_uint4(o[0], o[1], o[2], o[3]);
     }
     for (uint32_t i = nvec * 16 + tid; i < cnt; i += kThreads) {
