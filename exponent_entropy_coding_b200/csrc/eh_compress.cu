@@ -559,11 +559,24 @@ __device__ __forceinline__ uint32_t exp_of(const uint4 &p, const uint4 &q, int j
   }
 }
 
-// ORs the `nbits` (<= 32) code bits held right-aligned in `acc` into the
-// ring at stream bit `pos`.
+// (code left-aligned, length) of value j's exponent.  BF16: the exponent
+// sits in bits 7..14 of each half, so (e << 3), the entry's byte offset, is
+// one shift and one mask away.
+template <int DT>
+__device__ __forceinline__ uint2 code_of(const uint2 *tab, const uint4 &p, const uint4 &q, int j) {
+  if (DT == EH_BF16) {
+    const uint32_t w[8] = {p.x, p.y, p.z, p.w, q.x, q.y, q.z, q.w};
+    const uint32_t off = (w[j >> 1] >> ((j & 1) ? 20 : 4)) & 0x7F8u;
+    return *(const uint2 *)((const uint8_t *)tab + off);
+  }
+  return tab[exp_of<DT>(p, q, j)];
+}
+
 // Ring positions are bits relative to the start of the stream word that
 // holds the range's first bit (32-bit arithmetic; a range is one chunk or
 // page).  Ring word k is stream word (bit0 >> 5) + k, at slot k & kRingMask.
+// ring_or ORs the `nbits` (<= 32) code bits held right-aligned in `acc` in at
+// relative bit `pos`.
 __device__ __forceinline__ void ring_or(uint32_t *ring, uint32_t pos, uint32_t acc, uint32_t nbits) {
   const uint32_t s = pos & 31, w = pos >> 5;
   const uint64_t y = (uint64_t)acc << (64 - s - nbits);
@@ -607,7 +620,7 @@ __device__ void encode_range(const uint2 *tab, const uint8_t *in, uint32_t cnt, 
     if (idx + kEncPerThread <= cnt) {
       #pragma unroll
       for (int j = 0; j < kEncPerThread; j++) {
-        const uint2 cl = tab[exp_of<DT>(p, q, j)];
+        const uint2 cl = code_of<DT>(tab, p, q, j);
         hi[j >> 3] = __funnelshift_lc(lo[j >> 3], hi[j >> 3], cl.y);
         lo[j >> 3] = __funnelshift_lc(cl.x, lo[j >> 3], cl.y);
         tot[j >> 3] += cl.y;
@@ -615,7 +628,7 @@ __device__ void encode_range(const uint2 *tab, const uint8_t *in, uint32_t cnt, 
     } else {
       #pragma unroll
       for (int j = 0; j < kEncPerThread; j++) {
-        uint2 cl = tab[exp_of<DT>(p, q, j)];
+        uint2 cl = code_of<DT>(tab, p, q, j);
         if (idx + j >= cnt) cl = make_uint2(0u, 0u);
         hi[j >> 3] = __funnelshift_lc(lo[j >> 3], hi[j >> 3], cl.y);
         lo[j >> 3] = __funnelshift_lc(cl.x, lo[j >> 3], cl.y);
@@ -636,7 +649,7 @@ __device__ void encode_range(const uint2 *tab, const uint8_t *in, uint32_t cnt, 
       } else {
         uint32_t pp = pos;
         for (int j = 8 * h; j < 8 * h + 8; j++) {
-          uint2 cl = tab[exp_of<DT>(p, q, j)];
+          uint2 cl = code_of<DT>(tab, p, q, j);
           if (idx + j >= cnt || cl.y == 0) continue;
           ring_or(ring, pp, cl.x >> (32 - cl.y), cl.y);
           pp += cl.y;
