@@ -13,8 +13,13 @@
 //            stream words that two chunks share;
 //   encode   one CTA per chunk: code lookup, CTA-wide exclusive scan of code
 //            lengths, bit packing into a shared-memory word ring, coalesced
-//            stores of whole words and atomic OR of the two edge words.
-// Every kernel is HBM-bound; no tensor cores are involved.
+//            stores of whole words and atomic OR of the two edge words (and,
+//            when asked for, the value index).
+// Each kernel after hist is a programmatic dependent launch: it starts while
+// its predecessor finishes and waits for it before reading its results.
+// All of this is integer work (no dense contraction, no tensor cores); the
+// histogram runs near the HBM bound, the encoder is bound by instruction
+// issue.
 #include "eh_internal.cuh"
 
 namespace eh {
