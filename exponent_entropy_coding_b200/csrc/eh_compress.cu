@@ -67,14 +67,12 @@ __global__ void __launch_bounds__(kThreads, 2) hist_kernel(const __grid_constant
   uint8_t *hb = (uint8_t *)hl;
   if (DT == EH_BF16) {
     const uint16_t *in = (const uint16_t *)I.in + i0;
-    uint8_t *smo = I.sm + i0;
-    const uint32_t nvec = cnt / 16;  // 16 values per step: 32 B in, 16 B out
+    const uint32_t nvec = cnt / 16;  // 16 values per step: 32 B in
     #pragma unroll 2
     for (uint32_t v = tid; v < nvec; v += kThreads) {
       uint4 p = ld_stream(in + 16 * (uint64_t)v);
       uint4 q = ld_stream(in + 16 * (uint64_t)v + 8);
       uint32_t w[8] = {p.x, p.y, p.z, p.w, q.x, q.y, q.z, q.w};
-      uint32_t o[4];
       #pragma unroll
       for (int j = 0; j < 8; j++) {
         // exponent e sits in bits 7..14 of each half: e << 7 is the byte
@@ -82,20 +80,8 @@ __global__ void __launch_bounds__(kThreads, 2) hist_kernel(const __grid_constant
         atomicAdd((uint32_t *)(hb + (w[j] & 0x7F80u)), 1u);
         atomicAdd((uint32_t *)(hb + ((w[j] >> 16) & 0x7F80u)), 1u);
       }
-      #pragma unroll
-      for (int j = 0; j < 4; j++) {
-        // low bytes carry the mantissas, high bytes the signs (bit 7)
-        const uint32_t lows = __byte_perm(w[2 * j], w[2 * j + 1], 0x6420);
-        const uint32_t highs = __byte_perm(w[2 * j], w[2 * j + 1], 0x7531);
-        o[j] = (lows & 0x7F7F7F7Fu) | (highs & 0x80808080u);
-      }
-      *(uint4 *)(smo + 16 * (uint64_t)v) = make_uint4(o[0], o[1], o[2], o[3]);
     }
-    for (uint32_t i = nvec * 16 + tid; i < cnt; i += kThreads) {
-      uint32_t x = in[i];
-      atomicAdd(hl + (((x >> 7) & 0xFFu) << 5), 1u);
-      smo[i] = (uint8_t)bf16x2_sm(x);
-    }
+    for (uint32_t i = nvec * 16 + tid; i < cnt; i += kThreads) atomicAdd(hl + (((in[i] >> 7) & 0xFFu) << 5), 1u);
   } else if (DT == EH_BYTES) {
     // every byte is a symbol; there is no sign/mantissa to write
     const uint8_t *in = (const uint8_t *)I.in + i0;
@@ -114,33 +100,19 @@ __global__ void __launch_bounds__(kThreads, 2) hist_kernel(const __grid_constant
     for (uint32_t i = nvec * 32 + tid; i < cnt; i += kThreads) atomicAdd(hl + ((uint32_t)in[i] << 5), 1u);
   } else {
     const uint8_t *in = (const uint8_t *)I.in + i0;
-    uint8_t *smo = I.sm + i0 / 2;
-    const uint32_t nvec = cnt / 32;  // 32 values per step: 32 B in, 16 B out
+    const uint32_t nvec = cnt / 32;  // 32 values per step: 32 B in
     #pragma unroll 2
     for (uint32_t v = tid; v < nvec; v += kThreads) {
       uint4 p = ld_stream(in + 32 * (uint64_t)v);
       uint4 q = ld_stream(in + 32 * (uint64_t)v + 16);
       uint32_t w[8] = {p.x, p.y, p.z, p.w, q.x, q.y, q.z, q.w};
-      uint32_t o[4];
       #pragma unroll
       for (int j = 0; j < 8; j++) {
         #pragma unroll
         for (int k = 0; k < 4; k++) atomicAdd(hl + (((w[j] >> (8 * k + 3)) & 0xFu) << 5), 1u);
       }
-      #pragma unroll
-      for (int j = 0; j < 4; j++) o[j] = fp8x4_sm(w[2 * j]) | (fp8x4_sm(w[2 * j + 1]) << 16);
-      *(uint4 *)(smo + 16 * (uint64_t)v) = make_uint4(o[0], o[1], o[2], o[3]);
     }
-    // tail: one sign/mantissa byte (two values) per thread step
-    for (uint32_t pidx = nvec * 16 + tid; 2 * pidx < cnt; pidx += kThreads) {
-      uint32_t x0 = in[2 * pidx];
-      uint32_t x1 = (2 * pidx + 1 < cnt) ? in[2 * pidx + 1] : 0u;
-      atomicAdd(hl + (((x0 >> 3) & 0xFu) << 5), 1u);
-      if (2 * pidx + 1 < cnt) atomicAdd(hl + (((x1 >> 3) & 0xFu) << 5), 1u);
-      uint32_t s = fp8x4_sm(x0 | (x1 << 8));
-      if (2 * pidx + 1 >= cnt) s &= 0xFu;
-      smo[pidx] = (uint8_t)s;
-    }
+    for (uint32_t i = nvec * 32 + tid; i < cnt; i += kThreads) atomicAdd(hl + (((in[i] >> 3) & 0xFu) << 5), 1u);
   }
   __syncthreads();
   if (tid < A) {
@@ -577,6 +549,46 @@ __device__ __forceinline__ uint2 code_of(const uint2 *tab, const uint4 &p, const
   return tab[exp_of<DT>(p, q, j)];
 }
 
+// The sign/mantissa array of values [idx, idx + 16) of a chunk (held in p, q
+// as loaded by load_exps), written by the encoder beside the code packing.
+// BF16: one byte per value (s << 7 | m7); FP8: one nibble (s << 3 | m3),
+// value 2i in the low nibble of byte i, the high nibble of an odd tail zero.
+template <int DT>
+__device__ __forceinline__ void store_sm(uint8_t *smo, uint32_t idx, uint32_t cnt, const uint4 &p, const uint4 &q) {
+  if (DT == EH_BF16) {
+    const uint32_t w[8] = {p.x, p.y, p.z, p.w, q.x, q.y, q.z, q.w};
+    if (idx + 16 <= cnt) {
+      uint32_t o[4];
+      #pragma unroll
+      for (int j = 0; j < 4; j++) {
+        // low bytes carry the mantissas, high bytes the signs (bit 7)
+        const uint32_t lows = __byte_perm(w[2 * j], w[2 * j + 1], 0x6420);
+        const uint32_t highs = __byte_perm(w[2 * j], w[2 * j + 1], 0x7531);
+        o[j] = (lows & 0x7F7F7F7Fu) | (highs & 0x80808080u);
+      }
+      *(uint4 *)(smo + idx) = make_uint4(o[0], o[1], o[2], o[3]);
+    } else {
+      for (int j = 0; j < 16; j++)
+        if (idx + j < cnt) smo[idx + j] = (uint8_t)(bf16x2_sm(w[j >> 1] >> (16 * (j & 1))) & 0xFFu);
+    }
+  } else if (DT == EH_FP8_E4M3) {
+    if (idx + 16 <= cnt) {
+      const uint32_t lo = fp8x4_sm(p.x) | (fp8x4_sm(p.y) << 16);
+      const uint32_t hi = fp8x4_sm(p.z) | (fp8x4_sm(p.w) << 16);
+      *(uint2 *)(smo + idx / 2) = make_uint2(lo, hi);
+    } else {
+      const uint32_t w[4] = {p.x, p.y, p.z, p.w};
+      for (int j = 0; j < 16; j += 2) {
+        if (idx + j >= cnt) break;
+        const uint32_t pair = (w[j >> 2] >> (8 * (j & 3))) & 0xFFFFu;  // values j, j + 1
+        uint32_t sm = fp8x4_sm(pair) & 0xFFu;
+        if (idx + j + 1 >= cnt) sm &= 0xFu;
+        smo[(idx + j) / 2] = (uint8_t)sm;
+      }
+    }
+  }
+}
+
 // Ring positions are bits relative to the start of the stream word that
 // holds the range's first bit (32-bit arithmetic; a range is one chunk or
 // page).  Ring word k is stream word (bit0 >> 5) + k, at slot k & kRingMask.
@@ -605,7 +617,7 @@ __device__ __forceinline__ void ring_or64(uint32_t *ring, uint32_t pos, uint32_t
 template <int DT>
 __device__ void encode_range(const uint2 *tab, const uint8_t *in, uint32_t cnt, uint64_t bit0, uint64_t bit1,
                              uint32_t *gs, uint32_t *ring, uint32_t *wsum, bool exclusive,
-                             uint32_t *vindex = nullptr) {
+                             uint32_t *vindex = nullptr, uint8_t *smo = nullptr) {
   const int tid = threadIdx.x;
   const uint64_t gw0 = bit0 >> 5;             // stream word of relative word 0
   const uint32_t r0 = (uint32_t)(bit0 & 31);  // relative bit of the range's first code
@@ -618,6 +630,7 @@ __device__ void encode_range(const uint2 *tab, const uint8_t *in, uint32_t cnt, 
     const uint32_t idx = t0 + tid * kEncPerThread;
     const uint4 p = np, q = nq;
     if (t0 + kEncTile < cnt) load_exps<DT>(in, idx + kEncTile, cnt, np, nq);
+    if (smo && idx < cnt) store_sm<DT>(smo, idx, cnt, p, q);
     // two groups of 8 codes, each concatenated in a 64-bit accumulator
     // (hi:lo) when it fits (all but pathological codes); longer groups take
     // the per-code path
@@ -705,7 +718,8 @@ __global__ void __launch_bounds__(kThreads, 2) encode_kernel(const __grid_consta
   const uint8_t *in = (const uint8_t *)I.in + i0 * (DT == EH_BF16 ? 2 : 1);
   __syncthreads();
   uint32_t *vindex = I.vindex ? I.vindex + (uint64_t)c * (b.chunk_elems / kIndexStride) : nullptr;
-  encode_range<DT>(tab, in, cnt, I.off[c], I.off[c + 1], (uint32_t *)I.stream, ring, wsum, false, vindex);
+  uint8_t *smo = DT == EH_BF16 ? I.sm + i0 : (DT == EH_FP8_E4M3 ? I.sm + i0 / 2 : nullptr);
+  encode_range<DT>(tab, in, cnt, I.off[c], I.off[c + 1], (uint32_t *)I.stream, ring, wsum, false, vindex, smo);
   if (vindex) {
     // entries past a short last chunk's end: the chunk's bit count
     const uint32_t bits = (uint32_t)(I.off[c + 1] - I.off[c]);
