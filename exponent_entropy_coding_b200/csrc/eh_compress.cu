@@ -1,17 +1,17 @@
 // eh_compress.cu -- compression kernels of libexphuff (sm_100a).
 //
 // Steps, in launch order (one launch per step for a whole batch of tensors):
-//   hist     split every value into exponent field and sign+mantissa, write
-//            the packed sign/mantissa array, and count exponents per chunk and
-//            per tensor (DFloat11 article, "方法介绍": the Huffman code is built
-//            from the exponent distribution; sign and mantissa stay raw);
+//   hist     count the exponent fields per chunk and per tensor (DFloat11
+//            article, "方法介绍": the Huffman code is built from the exponent
+//            distribution);
 //   book     one CTA per tensor: code lengths (minimum-variance Huffman,
 //            package-merge when the depth exceeds the limit), rank assignment,
 //            canonical codes;
 //   offsets  code bits per chunk from its histogram, then (last CTA) an
 //            exclusive scan into the chunk bit offsets and the clearing of the
 //            stream words that two chunks share;
-//   encode   one CTA per chunk: code lookup, CTA-wide exclusive scan of code
+//   encode   one CTA per chunk: the packed sign/mantissa array (sign and
+//            mantissa stay raw), code lookup, CTA-wide exclusive scan of code
 //            lengths, bit packing into a shared-memory word ring, coalesced
 //            stores of whole words and atomic OR of the two edge words (and,
 //            when asked for, the value index).
