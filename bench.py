@@ -43,6 +43,17 @@ def decoder_source_sha():
     return h.hexdigest()[:16]
 
 
+def host_cpu_model():
+    try:
+        with open("/proc/cpuinfo") as fh:
+            for ln in fh:
+                if ln.startswith("model name"):
+                    return ln.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
 def hbm_peak():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -121,6 +132,15 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
+def workload_config(world, elements=218103808, chunk_elems=65536, max_code_len=32):
+    """The bench line's `config`: the same for both arms."""
+    return {"workload": "llama8b_block: q,k,v,o 4096/1024x4096, gate/up 14336x4096, "
+                        "down 4096x14336 BF16, Student-t(5) std 0.02, seed 2",
+            "elements": elements, "chunk_elems": chunk_elems, "max_code_len": max_code_len,
+            "parallelism": f"replicas x{world}",
+            "l2": "no flush: inputs (436 MB) larger than L2 (126 MB)"}
+
+
 def run_reference(args):
     """The CPU oracle on the host cores, on a bounded sample of the workload."""
     rank = int(os.environ.get("RANK", "0"))
@@ -150,9 +170,9 @@ def run_reference(args):
         "impl": "reference", "metric": METRIC, "value": v, "unit": "GB/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "u16",
-        "data": "synthetic", "config": {"workload": "llama8b_block (k_proj sample)",
-                                        "dims": "1024x4096", "threads": 1},
-        "cpu_baseline": {"value": v, "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": desc},
+        "data": "synthetic", "config": workload_config(args.gpus),
+        "cpu_baseline": {"value": v, "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": desc,
+                         "cpu": host_cpu_model(), "host_cores": os.cpu_count()},
         "e2e": {"value": v, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         "size_ratio": (c.stream.size + c.sign_mant.size + 8 * c.chunk_bit_off.size + 256) / nbytes,
     }
@@ -623,13 +643,12 @@ def main():
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "u16",
             "data": "synthetic",
-            "config": {"workload": "llama8b_block: q,k,v,o 4096/1024x4096, gate/up 14336x4096, "
-                                   "down 4096x14336 BF16, Student-t(5) std 0.02, seed 2",
-                       "elements": sum(ns), "chunk_elems": p.chunk_elems, "max_code_len": p.max_code_len,
-                       "parallelism": f"replicas x{world}",
-                       "l2": "no flush: inputs (436 MB) larger than L2 (126 MB)"},
+            "config": workload_config(world, sum(ns), p.chunk_elems, p.max_code_len),
             "decode_gbs": dec_gbs, "encode_gbs": enc_gbs,
             "pct_hbm": {"decode": dec_achieved / peak, "encode": enc_achieved / peak,
+                        # the compressor's real traffic reads the input twice (the
+                        # histogram must be complete before any code is known)
+                        "encode_with_second_read": (enc_alg + in_bytes) / (enc_ms * 1e-3) / 1e9 / peak,
                         "peak_gbs": peak, "peak_kind": peak_kind},
             "size_ratio": comp_bytes / in_bytes,
             "bits_per_exponent": 8 * stream_bytes / sum(ns),
@@ -653,6 +672,9 @@ def main():
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline_oracle(items)
             line["cpu_baseline_parallel"] = cpu_baseline_oracle_parallel()
+            for k in ("cpu_baseline", "cpu_baseline_parallel"):
+                line[k]["cpu"] = host_cpu_model()
+                line[k]["host_cores"] = os.cpu_count()
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()
