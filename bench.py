@@ -673,8 +673,9 @@ def main():
             line["cpu_baseline"] = cpu_baseline_oracle(items)
             line["cpu_baseline_parallel"] = cpu_baseline_oracle_parallel()
             for k in ("cpu_baseline", "cpu_baseline_parallel"):
-                line[k]["cpu"] = host_cpu_model()
-                line[k]["host_cores"] = os.cpu_count()
+                if isinstance(line.get(k), dict):
+                    line[k]["cpu"] = host_cpu_model()
+                    line[k]["host_cores"] = os.cpu_count()
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()
