@@ -145,8 +145,8 @@ EH_API eh_status eh_compress_batch_workspace(const eh_plan_t *plan, int k,
                                       const uint64_t *ns,
                                       uint64_t *workspace_bytes);
 
-/* Compresses one tensor (steps: split + histogram + sign/mantissa pack,
- * codebook, chunk offsets, encode).  `in` holds n raw BF16 (uint16) or FP8
+/* Compresses one tensor (steps: split + histogram, codebook, chunk offsets,
+ * encode + sign/mantissa pack).  `in` holds n raw BF16 (uint16) or FP8
  * (uint8) values.  `out` is a host struct whose dtype, n and device pointers
  * the caller has set; the call writes the device arrays, out->n_chunks and
  * out->exp_stream_bits.  Waits for `stream` once, to return the bit count. */
