@@ -7,6 +7,7 @@ import ctypes as C
 import os
 import re
 import subprocess
+import sys
 
 import pytest
 
@@ -88,3 +89,19 @@ def test_invalid_arguments_rejected_before_any_launch(lib):
     assert lib.eh_compress(C.byref(p), None, 10, C.byref(s), None, 0, None) == eh.EH_ERR_INVALID_ARG
     assert lib.eh_decompress(C.byref(p), C.byref(s), None, None, 0, None) == eh.EH_ERR_INVALID_ARG
     assert lib.eh_get_status(None, None) == eh.EH_ERR_INVALID_ARG
+
+
+def test_missing_library_fails_loudly():
+    """Without libexphuff.so the binding raises; there is no CPU fallback."""
+    code = ("import sys; sys.path.insert(0, %r)\n"
+            "from exponent_entropy_coding_b200 import exphuff as eh\n"
+            "eh.LIB_PATH = '/nonexistent/libexphuff.so'\n"
+            "try:\n"
+            "    eh.plan(0)\n"
+            "except RuntimeError as e:\n"
+            "    print('raised:', e)\n"
+            "    sys.exit(0)\n"
+            "sys.exit(3)\n") % ROOT
+    r = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, timeout=120)
+    assert r.returncode == 0, (r.stdout, r.stderr)
+    assert "not built" in r.stdout
