@@ -457,16 +457,28 @@ __global__ void __launch_bounds__(kOffThreads) offsets_kernel(const __grid_const
 }
 
 // ---------------------------------------------------------------- encode
-constexpr int kEncPerThread = 16;                       // values per thread per tile
-constexpr int kEncTile = kThreads * kEncPerThread;       // 8192 values
-constexpr int kRingWords = 16384;                        // > one tile of 32-bit codes + carry
-constexpr uint32_t kRingMask = kRingWords - 1;
+constexpr int kEncPerThread = 16;  // values per thread per tile
+
+// An encoding CTA of NT threads takes tiles of NT * 16 values and packs them
+// into a shared ring of twice as many 32-bit words (more than one tile of
+// 32-bit codes plus the partial word carried over).
+template <int NT>
+struct Enc {
+  static constexpr int kTile = NT * kEncPerThread;
+  static constexpr int kRingWords = 2 * kTile;
+  static constexpr uint32_t kRingMask = kRingWords - 1;
+  static constexpr int kMinBlocks = NT == 256 ? 4 : 2;  // CTAs per SM (64 registers a thread)
+};
+// Calls with at least a full wave of 256-thread CTAs (four per SM) use them;
+// calls with fewer chunks use 512-thread CTAs, which finish a chunk sooner.
+constexpr int kEncSmall = 256, kEncLarge = 512;
 
 // Exclusive scan over the CTA with a single barrier: every warp publishes
 // its total, then each thread adds up the totals of the warps before its own.
 // The caller must separate two uses of `wsum` by a barrier.
+template <int NT>
 __device__ __forceinline__ uint32_t block_excl_scan1(uint32_t v, uint32_t *wsum, uint32_t *total) {
-  constexpr int kWarps = kThreads / 32;
+  constexpr int kWarps = NT / 32;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   uint32_t x = v;
   #pragma unroll
@@ -594,7 +606,9 @@ __device__ __forceinline__ void store_sm(uint8_t *smo, uint32_t idx, uint32_t cn
 // page).  Ring word k is stream word (bit0 >> 5) + k, at slot k & kRingMask.
 // ring_or ORs the `nbits` (<= 32) code bits held right-aligned in `acc` in at
 // relative bit `pos`.
+template <int NT>
 __device__ __forceinline__ void ring_or(uint32_t *ring, uint32_t pos, uint32_t acc, uint32_t nbits) {
+  constexpr uint32_t kRingMask = Enc<NT>::kRingMask;
   const uint32_t s = pos & 31, w = pos >> 5;
   const uint64_t y = (uint64_t)acc << (64 - s - nbits);
   atomicOr(&ring[w & kRingMask], (uint32_t)(y >> 32));
@@ -602,7 +616,9 @@ __device__ __forceinline__ void ring_or(uint32_t *ring, uint32_t pos, uint32_t a
 }
 
 // ORs the low nbits (1..64) of (hi:lo) into the ring at relative bit pos.
+template <int NT>
 __device__ __forceinline__ void ring_or64(uint32_t *ring, uint32_t pos, uint32_t hi, uint32_t lo, uint32_t nbits) {
+  constexpr uint32_t kRingMask = Enc<NT>::kRingMask;
   const uint32_t s = pos & 31, w = pos >> 5;
   const uint64_t L = (((uint64_t)hi << 32) | lo) << (64 - nbits);  // left-aligned
   atomicOr(&ring[w & kRingMask], (uint32_t)(L >> (32 + s)));
@@ -614,10 +630,12 @@ __device__ __forceinline__ void ring_or64(uint32_t *ring, uint32_t pos, uint32_t
 // of gs.  The ring must be zero on entry and is zero on return.  Words that
 // the range shares with its neighbours are OR-ed into (pre-cleared) stream
 // words unless `exclusive`, when the range owns every word it touches.
-template <int DT>
+template <int DT, int NT>
 __device__ void encode_range(const uint2 *tab, const uint8_t *in, uint32_t cnt, uint64_t bit0, uint64_t bit1,
                              uint32_t *gs, uint32_t *ring, uint32_t *wsum, bool exclusive,
                              uint32_t *vindex = nullptr, uint8_t *smo = nullptr) {
+  constexpr int kEncTile = Enc<NT>::kTile;
+  constexpr uint32_t kRingMask = Enc<NT>::kRingMask;
   const int tid = threadIdx.x;
   const uint64_t gw0 = bit0 >> 5;             // stream word of relative word 0
   const uint32_t r0 = (uint32_t)(bit0 & 31);  // relative bit of the range's first code
@@ -654,7 +672,7 @@ __device__ void encode_range(const uint2 *tab, const uint8_t *in, uint32_t cnt, 
       }
     }
     uint32_t total;
-    const uint32_t excl = block_excl_scan1(tot[0] + tot[1], wsum, &total);
+    const uint32_t excl = block_excl_scan1<NT>(tot[0] + tot[1], wsum, &total);
     uint32_t pos = tile_base + excl;
     // value index: where every kIndexStride-th value's code starts, from the
     // range's first bit
@@ -663,13 +681,13 @@ __device__ void encode_range(const uint2 *tab, const uint8_t *in, uint32_t cnt, 
     for (int h = 0; h < 2; h++) {
       if (tot[h] == 0) continue;
       if (tot[h] <= 64) {
-        ring_or64(ring, pos, hi[h], lo[h], tot[h]);
+        ring_or64<NT>(ring, pos, hi[h], lo[h], tot[h]);
       } else {
         uint32_t pp = pos;
         for (int j = 8 * h; j < 8 * h + 8; j++) {
           uint2 cl = code_of<DT>(tab, p, q, j);
           if (idx + j >= cnt || cl.y == 0) continue;
-          ring_or(ring, pp, cl.x >> (32 - cl.y), cl.y);
+          ring_or<NT>(ring, pp, cl.x >> (32 - cl.y), cl.y);
           pp += cl.y;
         }
       }
@@ -679,7 +697,7 @@ __device__ void encode_range(const uint2 *tab, const uint8_t *in, uint32_t cnt, 
     tile_base += total;
     const bool last = t0 + kEncTile >= cnt;
     const uint32_t wend = last ? (rend + 31) >> 5 : tile_base >> 5;
-    for (uint32_t wi = wdone + tid; wi < wend; wi += kThreads) {
+    for (uint32_t wi = wdone + tid; wi < wend; wi += NT) {
       const uint32_t slot = wi & kRingMask;
       const uint32_t val = bswap32(ring[slot]);
       ring[slot] = 0u;
@@ -695,36 +713,36 @@ __device__ void encode_range(const uint2 *tab, const uint8_t *in, uint32_t cnt, 
 template <int DT>
 __device__ __forceinline__ void load_code_table(uint2 *tab, const uint8_t *code_len, const uint32_t *code) {
   constexpr int A = DT == EH_FP8_E4M3 ? 16 : 256;
-  for (int s2 = threadIdx.x; s2 < A; s2 += kThreads) {
+  for (int s2 = threadIdx.x; s2 < A; s2 += blockDim.x) {
     const uint32_t l = code_len[s2];
     tab[s2] = make_uint2(l ? code[s2] << (32 - l) : 0u, l);
   }
 }
 
-template <int DT>
-__global__ void __launch_bounds__(kThreads, 2) encode_kernel(const __grid_constant__ Batch b) {
+template <int DT, int NT>
+__global__ void __launch_bounds__(NT, Enc<NT>::kMinBlocks) encode_kernel(const __grid_constant__ Batch b) {
   constexpr int A = DT == EH_FP8_E4M3 ? 16 : 256;
-  extern __shared__ uint32_t ring[];  // kRingWords words, code bits in MSB-first order
+  extern __shared__ uint32_t ring[];  // Enc<NT>::kRingWords words, code bits in MSB-first order
   __shared__ uint2 tab[A];            // (code left-aligned in 32 bits, length)
-  __shared__ uint32_t wsum[kThreads / 32];
+  __shared__ uint32_t wsum[NT / 32];
   const uint32_t g = blockIdx.x;
   const Item &I = b.item[find_item(b, g)];
   const uint32_t c = g - I.chunk0;
   const uint64_t i0 = (uint64_t)c * b.chunk_elems;
   const uint32_t cnt = (uint32_t)min((uint64_t)b.chunk_elems, I.n - i0);
-  for (int i = threadIdx.x; i < kRingWords; i += kThreads) ring[i] = 0u;
+  for (int i = threadIdx.x; i < Enc<NT>::kRingWords; i += NT) ring[i] = 0u;
   pdl_wait();  // the codebook and the chunk offsets
   load_code_table<DT>(tab, I.code_len, I.code);
   const uint8_t *in = (const uint8_t *)I.in + i0 * (DT == EH_BF16 ? 2 : 1);
   __syncthreads();
   uint32_t *vindex = I.vindex ? I.vindex + (uint64_t)c * (b.chunk_elems / kIndexStride) : nullptr;
   uint8_t *smo = DT == EH_BF16 ? I.sm + i0 : (DT == EH_FP8_E4M3 ? I.sm + i0 / 2 : nullptr);
-  encode_range<DT>(tab, in, cnt, I.off[c], I.off[c + 1], (uint32_t *)I.stream, ring, wsum, false, vindex, smo);
+  encode_range<DT, NT>(tab, in, cnt, I.off[c], I.off[c + 1], (uint32_t *)I.stream, ring, wsum, false, vindex, smo);
   if (vindex) {
     // entries past a short last chunk's end: the chunk's bit count
     const uint32_t bits = (uint32_t)(I.off[c + 1] - I.off[c]);
     for (uint32_t k = (cnt + kIndexStride - 1) / kIndexStride + threadIdx.x; k < b.chunk_elems / kIndexStride;
-         k += kThreads)
+         k += NT)
       vindex[k] = bits;
   }
 }
@@ -754,12 +772,12 @@ __global__ void __launch_bounds__(kThreads, 2) page_append_kernel(const __grid_c
   const uint64_t sm_page = DT == EH_BF16 ? n : (DT == EH_FP8_E4M3 ? n / 2 : 0);
   uint8_t *smo = pl.sm + (uint64_t)slot * sm_page;
   load_code_table<DT>(tab, pl.code_len, pl.code);
-  for (int i = tid; i < kRingWords; i += kThreads) ring[i] = 0u;
+  for (int i = tid; i < Enc<kThreads>::kRingWords; i += kThreads) ring[i] = 0u;
   __syncthreads();
 
   // pass 1: code bits, missing codes, sign/mantissa
   uint32_t bits = 0, missing = 0;
-  for (uint32_t idx = tid * kEncPerThread; idx < n; idx += kEncTile) {
+  for (uint32_t idx = tid * kEncPerThread; idx < n; idx += Enc<kThreads>::kTile) {
     uint4 p, q;
     load_exps<DT>(in, idx, n, p, q);
     #pragma unroll
@@ -782,12 +800,12 @@ __global__ void __launch_bounds__(kThreads, 2) page_append_kernel(const __grid_c
     }
   }
   uint32_t total;
-  (void)block_excl_scan1(bits, wsum, &total);
+  (void)block_excl_scan1<kThreads>(bits, wsum, &total);
   const bool any_missing = __syncthreads_or(missing != 0);
   const bool coded = !any_missing && (total + 7) / 8 + 16 <= pl.slot_bytes;
   if (coded) {
     const uint64_t b0 = (uint64_t)slot * pl.slot_bytes * 8;
-    encode_range<DT>(tab, in, n, b0, b0 + total, (uint32_t *)pl.slots, ring, wsum, true);
+    encode_range<DT, kThreads>(tab, in, n, b0, b0 + total, (uint32_t *)pl.slots, ring, wsum, true);
     if (tid == 0) pl.page_meta[slot] = total;
     return;
   }
@@ -799,7 +817,7 @@ __global__ void __launch_bounds__(kThreads, 2) page_append_kernel(const __grid_c
   __syncthreads();
   if (raw_idx >= pl.raw_cap) return;
   uint8_t *dst = pl.raw_pool + (uint64_t)raw_idx * n;
-  for (uint32_t idx = tid * kEncPerThread; idx < n; idx += kEncTile) {
+  for (uint32_t idx = tid * kEncPerThread; idx < n; idx += Enc<kThreads>::kTile) {
     uint4 p, q;
     load_exps<DT>(in, idx, n, p, q);
     uint32_t o[4];
@@ -834,12 +852,16 @@ cudaError_t launch_offsets(const Batch &b, cudaStream_t s) {
 }
 
 cudaError_t configure_encode() {
-  const int smem = kRingWords * (int)sizeof(uint32_t);
-  cudaError_t e = cudaFuncSetAttribute(encode_kernel<EH_BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(encode_kernel<EH_BYTES>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(encode_kernel<EH_FP8_E4M3>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  const int smem = Enc<kThreads>::kRingWords * (int)sizeof(uint32_t);
+  const int small = Enc<kEncSmall>::kRingWords * (int)sizeof(uint32_t);
+  const int large = Enc<kEncLarge>::kRingWords * (int)sizeof(uint32_t);
+  const cudaFuncAttribute dyn = cudaFuncAttributeMaxDynamicSharedMemorySize;
+  cudaError_t e = cudaFuncSetAttribute(encode_kernel<EH_BF16, kEncSmall>, dyn, small);
+  if (e == cudaSuccess) e = cudaFuncSetAttribute(encode_kernel<EH_BYTES, kEncSmall>, dyn, small);
+  if (e == cudaSuccess) e = cudaFuncSetAttribute(encode_kernel<EH_FP8_E4M3, kEncSmall>, dyn, small);
+  if (e == cudaSuccess) e = cudaFuncSetAttribute(encode_kernel<EH_BF16, kEncLarge>, dyn, large);
+  if (e == cudaSuccess) e = cudaFuncSetAttribute(encode_kernel<EH_BYTES, kEncLarge>, dyn, large);
+  if (e == cudaSuccess) e = cudaFuncSetAttribute(encode_kernel<EH_FP8_E4M3, kEncLarge>, dyn, large);
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(page_append_kernel<EH_BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
@@ -850,20 +872,30 @@ cudaError_t configure_encode() {
 
 cudaError_t launch_page_append(const PageLaunch &pl, cudaStream_t s) {
   if (pl.n_pages == 0) return cudaSuccess;
-  const size_t smem = kRingWords * sizeof(uint32_t);
+  const size_t smem = Enc<kThreads>::kRingWords * sizeof(uint32_t);
   if (pl.dtype == EH_BF16) page_append_kernel<EH_BF16><<<pl.n_pages, kThreads, smem, s>>>(pl);
   else if (pl.dtype == EH_BYTES) page_append_kernel<EH_BYTES><<<pl.n_pages, kThreads, smem, s>>>(pl);
   else page_append_kernel<EH_FP8_E4M3><<<pl.n_pages, kThreads, smem, s>>>(pl);
   return cudaGetLastError();
 }
 
+template <int NT>
+cudaError_t launch_encode_nt(const Batch &b, cudaStream_t s) {
+  const size_t smem = Enc<NT>::kRingWords * sizeof(uint32_t);
+  const dim3 grid(b.total_chunks), block(NT);
+  if (b.dtype == EH_BF16) return launch_pdl(encode_kernel<EH_BF16, NT>, grid, block, smem, s, b);
+  if (b.dtype == EH_BYTES) return launch_pdl(encode_kernel<EH_BYTES, NT>, grid, block, smem, s, b);
+  return launch_pdl(encode_kernel<EH_FP8_E4M3, NT>, grid, block, smem, s, b);
+}
+
 cudaError_t launch_encode(const Batch &b, cudaStream_t s) {
   if (b.total_chunks == 0) return cudaSuccess;
-  const size_t smem = kRingWords * sizeof(uint32_t);
-  if (b.dtype == EH_BF16) return launch_pdl(encode_kernel<EH_BF16>, dim3(b.total_chunks), dim3(kThreads), smem, s, b);
-  if (b.dtype == EH_BYTES) return launch_pdl(encode_kernel<EH_BYTES>, dim3(b.total_chunks), dim3(kThreads), smem, s, b);
-  return launch_pdl(encode_kernel<EH_FP8_E4M3>, dim3(b.total_chunks), dim3(kThreads), smem, s, b);
-  return cudaGetLastError();
+  int dev = 0, sms = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return e;
+  if (b.total_chunks >= (uint32_t)(Enc<kEncSmall>::kMinBlocks * sms)) return launch_encode_nt<kEncSmall>(b, s);
+  return launch_encode_nt<kEncLarge>(b, s);
 }
 
 }  // namespace eh

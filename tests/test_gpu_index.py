@@ -43,7 +43,9 @@ def _compress_indexed(eh, p, x):
 
 
 CASES = [(0, 65536, 3 * 65536 + 3392, 1), (0, 65536, 1 << 20, 2), (0, 4096, 70000, 3), (1, 65536, 200001, 4),
-         (2, 65536, 150000, 5), (0, 65536, 100, 6)]
+         (2, 65536, 150000, 5), (0, 65536, 100, 6),
+         # enough chunks for the encoder's 256-thread CTAs (a full wave of them)
+         (0, 1024, 650 * 1024 + 77, 7), (1, 1024, 700 * 1024 + 5, 8)]
 
 
 @pytest.mark.parametrize("dtype,chunk,n,seed", CASES)

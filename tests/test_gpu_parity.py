@@ -70,7 +70,9 @@ def test_fp8_normal(eh, oracle, n):
 
 
 @pytest.mark.parametrize("dtype,chunk,n", [(0, 1024, 10 * 1024 + 3), (1, 1024, 9 * 1024 + 1),
-                                           (0, 4096, 50_000), (1, 8192, 65_537)])
+                                           (0, 4096, 50_000), (1, 8192, 65_537),
+                                           # a full wave of the encoder's 256-thread CTAs
+                                           (0, 1024, 600 * 1024 + 3), (1, 1024, 1200 * 1024 + 1)])
 def test_small_chunks(eh, oracle, dtype, chunk, n):
     x = synth.normal_bf16(n, seed=3) if dtype == 0 else synth.normal_fp8(n, seed=3)
     roundtrip(eh, oracle, dtype, x, chunk=chunk)
