@@ -10,7 +10,8 @@
 //   offsets  code bits per chunk from its histogram, then (last CTA) an
 //            exclusive scan into the chunk bit offsets and the clearing of the
 //            stream words that two chunks share;
-//   encode   one CTA per chunk: the packed sign/mantissa array (sign and
+//   encode   one CTA per chunk (256 threads when the call has a full wave
+//            of such CTAs, else 512): the packed sign/mantissa array (sign and
 //            mantissa stay raw), code lookup, CTA-wide exclusive scan of code
 //            lengths, bit packing into a shared-memory word ring, coalesced
 //            stores of whole words and atomic OR of the two edge words (and,
