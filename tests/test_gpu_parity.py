@@ -297,3 +297,31 @@ def test_bytes_every_value(eh, oracle):
     rng = np.random.default_rng(8)
     x = np.tile(np.arange(256, dtype=np.uint8), 1000)[rng.permutation(256 * 1000)]
     roundtrip(eh, oracle, 2, x)
+
+
+@pytest.mark.parametrize("name,dtype,npdt", [("handworked_bf16.txt", 0, np.uint16),
+                                             ("handworked_fp8.txt", 1, np.uint8)])
+def test_handworked_goldens(eh, name, dtype, npdt):
+    """The hand-worked examples' codes, stream and sign/mantissa bytes, straight
+    from the fixtures (no oracle in between)."""
+    import os
+    path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden", name)
+    rows = [ln.strip() for ln in open(path) if ln.strip() and not ln.startswith("#")]
+    g = dict(r.split(":", 1) for r in rows)
+    x = np.array([int(h, 16) for h in g["input_hex"].split()], npdt)
+    p = eh.plan(dtype)
+    c = eh.compress(dev(x), p)
+    lens = c.code_len.cpu().numpy()
+    codes = c.code.cpu().numpy().view(np.uint32)
+    want_lens = dict(item.split(":") for item in g["lengths"].split())
+    for s in range(lens.size):
+        assert int(lens[s]) == int(want_lens.get(str(s), 0))
+    for item in g["codes"].split():
+        s, bits = item.split(":")
+        assert format(int(codes[int(s)]), f"0{len(bits)}b") == bits
+    assert c.exp_stream_bits == int(g["bits"])
+    assert list(c.chunk_bit_off.cpu().numpy().view(np.uint64)) == [int(v) for v in g["offsets"].split()]
+    want = bytes(int(h, 16) for h in g["stream_hex"].split())
+    assert bytes(c.exp_stream[:len(want)].cpu().numpy()) == want
+    assert bytes(c.sign_mant.cpu().numpy()) == bytes(int(h, 16) for h in g["sign_mant_hex"].split())
+    assert np.array_equal(host_bits(eh.decompress(c, p), dtype), x)

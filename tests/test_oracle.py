@@ -283,6 +283,28 @@ def test_handworked_example(oracle):
     assert np.array_equal(oracle.decompress(c), x)
 
 
+def test_handworked_fp8_example(oracle):
+    g = dict(r.split(":", 1) for r in read_golden("handworked_fp8.txt"))
+    x = np.array([int(h, 16) for h in g["input_hex"].split()], np.uint8)
+    e, _ = oracle.split(oracle.FP8_E4M3, x)
+    assert list(e) == [int(v) for v in g["exponents"].split()]
+    c = oracle.compress(oracle.FP8_E4M3, x)
+    for item in g["lengths"].split():
+        s, l = item.split(":")
+        assert c.code_len[int(s)] == int(l)
+    assert int(np.count_nonzero(c.code_len)) == len(g["lengths"].split())
+    for item in g["codes"].split():
+        s, bits = item.split(":")
+        assert format(int(c.code[int(s)]), f"0{len(bits)}b") == bits
+    assert c.bits == int(g["bits"])
+    assert list(c.chunk_bit_off) == [int(v) for v in g["offsets"].split()]
+    assert bytes(c.stream) == bytes(int(h, 16) for h in g["stream_hex"].split())
+    assert bytes(c.sign_mant) == bytes(int(h, 16) for h in g["sign_mant_hex"].split())
+    cnt = oracle.histogram(oracle.FP8_E4M3, x)
+    assert abs(entropy_bits(cnt) - float(g["entropy_bits"])) < 1e-12
+    assert np.array_equal(oracle.decompress(c), x)
+
+
 def _bits_of(stream, nbits):
     return np.unpackbits(stream, bitorder="big")[:nbits]
 
