@@ -10,6 +10,8 @@ python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
 --impl reference times the CPU oracle (single-threaded C++) on the host on a
 bounded sample of the same workload, with the same metric.
+--all-configs prints one line per workload of the codec's table (the BF16
+1M and FP8 16M tensors, the block, the K/V layer, the LM head) instead.
 """
 import argparse
 import hashlib
@@ -269,6 +271,77 @@ def run_ncu_case():
     return 0
 
 
+def run_all_configs(reps=20):
+    """One JSON line per workload (the five of the codec's table): batched
+    compress and decompress timed with CUDA events, median of `reps` after 3
+    warm-ups, a 256 MB L2 flush before every timed call; algorithmic-byte
+    fractions of the measured copy bandwidth; the oracle's round trip of the
+    workload's first tensor on one host core beside it."""
+    import torch
+
+    from exponent_entropy_coding_b200 import exphuff as eh
+    from exponent_entropy_coding_b200 import synth
+    from oracle import ehref
+    peak, peak_kind = hbm_peak()
+    dev = torch.device("cuda", 0)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    for name in ("bf16_1m", "fp8_16m", "llama8b_block", "kv_layer", "lm_head"):
+        dt, items = synth.workload(name)
+        dtype = {"bf16": eh.EH_BF16, "fp8_e4m3": eh.EH_FP8_E4M3}[dt]
+        view = np.int16 if dtype == eh.EH_BF16 else np.uint8
+        p = eh.plan(dtype)
+        xs = [torch.from_numpy(np.ascontiguousarray(x).view(view)).to(dev) for _, x in items]
+        outs = [eh.alloc_compressed(p, x.numel(), dev) for x in xs]
+        ys = [torch.empty_like(x) for x in xs]
+        wsc = torch.empty(eh.compress_batch_workspace(p, [x.numel() for x in xs]), dtype=torch.uint8, device=dev)
+        wsd = torch.empty(eh.decompress_workspace(p, len(xs)), dtype=torch.uint8, device=dev)
+        bits = torch.zeros(len(xs), dtype=torch.int64, device=dev)
+        eh.compress_batch(p, xs, outs, wsc)  # with a host wait: fills the stream sizes
+        t_c, t_d = [], []
+        for r in range(3 + reps):
+            ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+            flush.zero_()
+            ev[0].record()
+            eh.compress_batch(p, xs, outs, wsc, bits_dev=bits)
+            ev[1].record()
+            flush.zero_()
+            ev[2].record()
+            eh.decompress_batch(p, outs, ys, wsd)
+            ev[3].record()
+            torch.cuda.synchronize()
+            if r >= 3:
+                t_c.append(ev[0].elapsed_time(ev[1]) * 1e-3)
+                t_d.append(ev[2].elapsed_time(ev[3]) * 1e-3)
+        assert eh.get_status(wsd) == eh.EH_OK
+        assert all(torch.equal(x, y) for x, y in zip(xs, ys)), name
+        n = sum(x.numel() for x in xs)
+        nbytes = sum(x.numel() * x.element_size() for x in xs)
+        stream_b = sum(o.stream_bytes() for o in outs)
+        sm_b = sum(o.sign_mant.numel() for o in outs)
+        off_b = sum(8 * o.chunk_bit_off.numel() for o in outs)
+        alg = nbytes + sm_b + stream_b + off_b  # each byte once, either direction
+        tc, td = statistics.median(t_c), statistics.median(t_d)
+        x0 = np.ascontiguousarray(items[0][1])
+        a = time.perf_counter()
+        c0 = ehref.compress(dtype, x0)
+        b_ = time.perf_counter()
+        y0 = ehref.decompress(c0)
+        e_ = time.perf_counter()
+        assert np.array_equal(y0, x0)
+        print(json.dumps({
+            "config": name, "values": n, "bytes": nbytes,
+            "compress_gbs": nbytes / tc / 1e9, "decompress_gbs": nbytes / td / 1e9,
+            "compress_frac": alg / tc / 1e9 / peak, "decompress_frac": alg / td / 1e9 / peak,
+            "peak_gbs": peak, "peak_kind": peak_kind,
+            "compress_us": tc * 1e6, "decompress_us": td * 1e6,
+            "size_ratio": sum(o.compressed_bytes() for o in outs) / nbytes,
+            "bits_per_exponent": 8 * stream_b / n,
+            "oracle": {"compress_gbs": x0.nbytes / (b_ - a) / 1e9, "decompress_gbs": x0.nbytes / (e_ - b_) / 1e9,
+                       "cores": 1, "sample": f"{items[0][0]} ({x0.size} values)"},
+        }), flush=True)
+    return 0
+
+
 def measure_fp4_scales(eh, synth, items, dev, stream, reps=50):
     """Compress + decompress of the seven matrices' E4M3 block scales (byte
     alphabet) with CUDA events; returns GB/s of scale bytes and the ratio."""
@@ -500,6 +573,8 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--no-side", action="store_true",
                     help="skip the side measurements (FP4 scales, K/V pages, ZipFloat, prefetch ring)")
+    ap.add_argument("--all-configs", action="store_true",
+                    help="one line per workload of the codec's table (compress/decompress, fractions, oracle)")
     ap.add_argument("--ncu-case", action="store_true",
                     help="one compress + one decompress of gate_proj (14336x4096), for ncu captures")
     args = ap.parse_args()
@@ -507,6 +582,8 @@ def main():
         return run_reference(args)
     if args.ncu_case:
         return run_ncu_case()
+    if args.all_configs:
+        return run_all_configs()
 
     import torch
     import torch.distributed as dist
