@@ -2,10 +2,10 @@
 //
 //   tables  eight CTAs per codebook: validate the code lengths and codes and
 //           build the decode tables (a 12-bit first level giving, for the
-//           index bits, the symbols of up to four complete codes, their bits,
-//           and the number, bits and start offsets of all complete codes;
-//           8-bit second-level tables for codes of 13..20 bits; canonical
-//           limits for anything longer);
+//           index bits, the number, bits and start offsets of all complete
+//           codes and the symbols and bits of the first four; 8-bit second
+//           levels for codes of 13..20 bits; canonical limits for anything
+//           longer);
 //   decode  persistent CTAs of two independent groups, one chunk per group
 //           at a time:
 //             1. the chunk's bit range is copied into shared memory with one
@@ -14,16 +14,20 @@
 //             2. every thread counts the codes of its own window of the
 //                chunk's bits, starting speculatively at the window start and
 //                recording the code boundaries of its first 64 bits;
-//             3. fix-up rounds: each thread restarts from the true end of its
-//                predecessor and stops as soon as it lands on one of its
-//                recorded boundaries (Huffman codes resynchronise after a few
-//                codes), until no end moves;
+//             3. fix-up: each thread restarts from the end of its
+//                predecessor's codes and stops as soon as it lands on one of
+//                its recorded boundaries (Huffman codes resynchronise after a
+//                few codes);
 //             4. group-wide exclusive scan of the per-thread code counts
 //                gives every thread its first output index;
-//             5. the threads decode again from their true starts and write
-//                their exponents to shared memory;
-//             6. coalesced pass: exponents merged with the sign/mantissa
-//                stream and stored with 16-byte stores.
+//             5. every thread decodes again from its true start and writes a
+//                run of whole exponent words to shared memory: the run starts
+//                at the first multiple of 4 (16 for a warp's first thread) at
+//                or after its first code and ends where its successor's run
+//                starts, so no word is shared and no buffer is cleared;
+//             6. each warp merges its own runs with the sign/mantissa stream
+//                as soon as they are written (no group barrier) and stores
+//                them with 16-byte coalesced stores.
 // The DFloat11 article ("方法介绍") describes compact LUTs sized for on-chip
 // SRAM, a two-phase kernel coordinating where each thread reads and writes,
 // and block-level decompression; here the per-thread start positions are not
@@ -34,7 +38,7 @@ namespace eh {
 namespace {
 
 constexpr uint32_t kMaskBits = 64;            // code starts recorded per thread
-constexpr uint32_t kSpinLimit = 1u << 26;     // bounded mbarrier wait
+constexpr uint64_t kWaitLimitNs = 200000000ull;  // a stage copy not landed after 0.2 s is given up
 
 // ---------------------------------------------------------------- tables
 // kTabParts CTAs of 256 threads per codebook; each builds 1/kTabParts of the
@@ -51,6 +55,14 @@ __device__ __forceinline__ uint32_t code_length_of(uint32_t x, const uint64_t *l
     else lo = mid + 1;
   }
   return lo;
+}
+
+// The form in which the decoder keeps a decoded symbol.  BF16 exponents are
+// rotated right by one bit, (e >> 1) | (e & 1) << 7: the high bits then sit
+// where the high byte of the BF16 value needs them and the low bit where the
+// low byte does, so two byte permutes and one bit select rebuild two values.
+__device__ __forceinline__ uint32_t out_form(int dtype, uint32_t e) {
+  return dtype == EH_BF16 ? ((e >> 1) | ((e & 1u) << 7)) : e;
 }
 
 __global__ void __launch_bounds__(256) tables_kernel(const __grid_constant__ Batch b) {
@@ -141,17 +153,18 @@ __global__ void __launch_bounds__(256) tables_kernel(const __grid_constant__ Bat
     if (tid == 0 && part == 0) T->err = err;
     return;
   }
-  if (part == 0) T->sorted[tid] = tid < (int)nsym ? srt[tid] : (uint8_t)0;
+  if (part == 0) T->sorted[tid] = tid < (int)nsym ? (uint8_t)out_form(b.dtype, srt[tid]) : (uint8_t)0;
 
   // first level.  Codes longer than kLutBits fill the left-justified range
-  // [lim[kLutBits], lim[32]), so their prefixes are consecutive: the first
-  // kNumSub of them get a second-level table.
+  // [lim[kLutBits], lim[32]), so their prefixes are consecutive from sub0 on:
+  // the first kNumSub of them get a second-level table.
   constexpr uint32_t kShift = 32 - kLutBits;
   const uint32_t sub0 = (uint32_t)(limL[kLutBits] >> kShift);
+  if (part == 0 && tid == 0) T->sub0 = sub0;
   constexpr uint32_t kPerPart = (1u << kLutBits) / kTabParts;
   for (uint32_t p = part * kPerPart + tid; p < (part + 1) * kPerPart; p += 256) {
-    // every complete code inside the index bits: all of them for counting,
-    // the first four (their symbols fill 32 bits) for writing
+    // every complete code inside the index bits (their number, bits and
+    // starts), and the symbols of the first four
     uint32_t syms = 0, pos = 0, nc = 0, bnd = 0, pos4 = 0, nc4 = 0;
     while (pos < (uint32_t)kLutBits) {
       const uint32_t x = (p << kShift) << pos;  // next bits, left-justified, zero-filled
@@ -159,7 +172,7 @@ __global__ void __launch_bounds__(256) tables_kernel(const __grid_constant__ Bat
       if (L > (uint32_t)kLutBits - pos) break;  // not complete inside the index bits
       if (nc < 4) {
         const uint32_t v = x >> (32 - L);
-        syms |= (uint32_t)srt[baseL[L] + v - firstL[L]] << (8 * nc);
+        syms |= out_form(b.dtype, srt[baseL[L] + v - firstL[L]]) << (8 * nc);
         pos4 = pos + L;
         nc4 = nc + 1;
       }
@@ -167,10 +180,9 @@ __global__ void __launch_bounds__(256) tables_kernel(const __grid_constant__ Bat
       pos += L;
       nc++;
     }
-    uint32_t sub = kNoSub;
-    if (nc == 0 && ((uint64_t)p << kShift) < limL[32] && p - sub0 < (uint32_t)kNumSub) sub = p - sub0;
-    T->l1sym[p] = syms;
-    T->l1meta[p] = pos4 | (nc4 << 4) | (bnd << 7) | (sub << 19) | (pos << 24) | (nc << 28);
+    uint32_t meta = 0;  // a prefix without a complete code: every field zero
+    if (nc) meta = pos | ((bnd >> 1) << kMetaStartShift) | (nc << 16) | (pos4 << 20) | ((8u * nc4) << 24);
+    T->l1[p] = make_uint2(syms, meta);
   }
   if (part != 0) return;
   // second level: codes of kLutBits+1 .. kLutBits+8 bits
@@ -183,7 +195,7 @@ __global__ void __launch_bounds__(256) tables_kernel(const __grid_constant__ Bat
         if ((uint64_t)x < limL[L]) {
           if (x >= (uint32_t)(limL[L - 1])) {
             const uint32_t v = x >> (32 - L);
-            e = (uint32_t)srt[baseL[L] + v - firstL[L]] | (L << 8);
+            e = out_form(b.dtype, srt[baseL[L] + v - firstL[L]]) | (L << 8);
           }
           break;
         }
@@ -195,100 +207,89 @@ __global__ void __launch_bounds__(256) tables_kernel(const __grid_constant__ Bat
 }
 
 // ---------------------------------------------------------------- decode
-// Exponent j of a chunk is kept at byte j + 4*(j/128) of the exponent buffer:
-// every 128-byte row is followed by 4 pad bytes, so threads whose outputs
-// start about 128 values apart write to different shared-memory banks.
-constexpr uint32_t kExpBytes = kMaxChunk + 4 * (kMaxChunk / 128);
-__device__ __forceinline__ uint32_t exp_slot(uint32_t j) { return j + ((j >> 7) << 2); }
+// Accessors of a first-level meta word (see DecodeTables).
+__device__ __forceinline__ uint32_t meta_starts(uint32_t m) {  // code starts at offsets 0..11
+  return ((m >> (kMetaStartShift - 1)) & 0xFFEu) | 1u;
+}
+constexpr uint32_t kCountFields = 0x000F000Fu;  // bits of all codes | their number << 16
 
-// 32 stream bits starting at bit p.  Shared-memory stages are byte-swapped
-// once after the copy, so their words are already MSB-first; global words are
-// swapped on load.
+// 32 stream bits starting at bit q of a thread's frame.  Shared-memory stages
+// are byte-swapped once after the copy, so their words are already
+// MSB-first; global words are swapped on load.
 template <bool kSmem>
 struct Peek {
   const uint32_t *w;
   __device__ __forceinline__ uint32_t word(uint32_t i) const { return kSmem ? w[i] : bswap32(__ldg(w + i)); }
-  __device__ __forceinline__ uint32_t operator()(uint32_t p) const {
-    const uint32_t i = p >> 5;
-    return __funnelshift_l(word(i + 1), word(i), p & 31);
+  __device__ __forceinline__ uint32_t operator()(uint32_t q) const {
+    const uint32_t i = q >> 5;
+    return __funnelshift_l(word(i + 1), word(i), q);  // the shift is taken modulo 32
   }
 };
 
 __device__ __forceinline__ uint32_t lut_index(uint32_t x) { return x >> (32 - kLutBits); }
 
-// Code longer than the first-level index: second-level table, else search of
-// the canonical limits.  Returns 1 and the symbol and length, or 0 for an
-// invalid code.
-__device__ __forceinline__ uint32_t decode_long(const DecodeTables &T, uint32_t peek, uint32_t meta,
-                                                uint32_t &syms, uint32_t &nbits) {
-  const uint32_t si = (meta >> 19) & 31u;
-  if (si != kNoSub) {
-    const uint32_t e2 = T.sub[si][(peek >> (24 - kLutBits)) & 0xFFu];
-    const uint32_t l = (e2 >> 8) & 63u;
-    if (l) {
-      nbits = l;
-      syms = e2 & 0xFFu;
-      return 1;
-    }
+// A code longer than the first-level index (its prefix has no complete
+// code): second-level table, else search of the canonical limits.  Returns
+// the symbol (output form) | length << 8, or 0 for an invalid code.
+__device__ __noinline__ uint32_t decode_long(const DecodeTables &T, uint32_t x) {
+  const uint32_t si = lut_index(x) - T.sub0;
+  if (si < (uint32_t)kNumSub) {
+    const uint32_t e2 = T.sub[si][(x >> (24 - kLutBits)) & 0xFFu];
+    if (e2 >> 8) return e2;
   }
   uint32_t L = kLutBits + 1;
-  #pragma unroll 1
-  while (L <= 32 && (uint64_t)peek >= T.lim[L]) L++;
+  while (L <= 32 && (uint64_t)x >= T.lim[L]) L++;
   if (L > 32) return 0;
-  const uint32_t v = L == 32 ? peek : peek >> (32 - L);
-  syms = T.sorted[T.base[L] + (v - T.first[L])];
-  nbits = L;
-  return 1;
+  const uint32_t v = L == 32 ? x : x >> (32 - L);
+  return T.sorted[T.base[L] + (v - T.first[L])] | (L << 8);
 }
 
-// One decode step on the next 32 bits `x`, taking only codes that start in
+// One counting step on the next 32 bits `x`, taking only codes that start in
 // the next `lim` (>= 1) bits.  Returns the number of codes taken (0: invalid
-// code); their symbols (8 bits each, first in the low byte) when kSyms, the
-// bits up to the end of the last code taken, and the code starts as a bitmap.
-template <bool kSyms>
-__device__ __forceinline__ uint32_t decode_step(const DecodeTables &T, uint32_t x, uint32_t lim,
-                                                uint32_t &syms, uint32_t &nbits, uint32_t &bnd) {
-  const uint32_t idx = lut_index(x);
-  const uint32_t meta = T.l1meta[idx];
-  // writing takes the first four codes (their symbols), counting all of them
-  uint32_t k = kSyms ? (meta >> 4) & 7u : meta >> 28;
-  if (k) {
-    uint32_t nb = kSyms ? meta & 15u : (meta >> 24) & 15u;
-    uint32_t bm = (meta >> 7) & 0xFFFu;
-    if (kSyms) bm &= (1u << nb) - 1u;
-    uint32_t sy = kSyms ? T.l1sym[idx] : 0u;
-    if (nb > lim) {
-      // codes starting at or after the limit belong to the next window
-      const uint32_t keep = bm & ((1u << lim) - 1u);
-      const uint32_t rest = bm >> lim;
-      k = __popc(keep);
-      nb = rest ? lim + __ffs(rest) - 1 : nb;
-      bm = keep;
-      if (kSyms && k < 4) sy &= (1u << (8 * k)) - 1u;
-    }
-    nbits = nb;
-    bnd = bm;
-    syms = sy;
-    return k;
+// code), the bits up to the end of the last one and their starts as a bitmap.
+__device__ __forceinline__ uint32_t count_step(const DecodeTables &T, uint32_t x, uint32_t lim, uint32_t &nbits,
+                                               uint32_t &bnd) {
+  const uint32_t m = T.l1[lut_index(x)].y;
+  uint32_t k = (m >> 16) & 15u;
+  if (!k) {
+    const uint32_t d = decode_long(T, x);
+    bnd = 1u;
+    nbits = d >> 8;
+    return d ? 1u : 0u;
   }
-  bnd = 1u;
-  return decode_long(T, x, meta, syms, nbits);
+  uint32_t nb = m & 15u, bm = meta_starts(m);
+  if (nb > lim) {
+    // codes starting at or after the limit belong to the next window
+    const uint32_t keep = bm & ((1u << lim) - 1u);
+    const uint32_t rest = bm >> lim;
+    k = __popc(keep);
+    nb = rest ? lim + __ffs(rest) - 1 : nb;
+    bm = keep;
+  }
+  nbits = nb;
+  bnd = bm;
+  return k;
 }
 
 // The decoding CTA holds two independent groups of kGroupThreads threads.
 // Each group decodes its own chunk into its own exponent buffer, so one
-// group's memory-bound output pass overlaps the other's decode; the decode
-// tables are shared.
+// group's memory-bound output overlaps the other's decode; the decode tables
+// are shared.
 constexpr uint32_t kGroupThreads = 512;
+constexpr uint32_t kGroupWarps = kGroupThreads / 32;
 constexpr uint32_t kNumGroups = kDecThreads / kGroupThreads;
 constexpr uint32_t kGroupStage = 27136;  // bytes of stream staged per group
 
 struct GroupSmem {
   alignas(128) uint32_t stage[kGroupStage / 4 + 16];  // bulk-copy target (stream bytes as stored)
-  alignas(16) uint8_t exps[kExpBytes];                // decoded exponents of one chunk (padded rows)
-  uint32_t ends[kGroupThreads];
-  uint32_t wsum[kGroupThreads / 32];
+  alignas(16) uint8_t exps[kMaxChunk];                // decoded exponents (output form) of one chunk
+  uint32_t ends[kGroupThreads];                       // end bit of every thread's codes
+  uint32_t wsum[2][kGroupWarps];                      // scan: warp totals, by round parity
   alignas(8) unsigned long long mbar;
+  const uint8_t *next_src[2];                         // stage copy of the group's next chunk,
+  uint32_t next_bytes[2];                             // by chunk parity (0 bytes: none)
+  uint32_t writers_done;                              // warps done reading the stage
+  uint32_t issued;                                    // stage copies started
 };
 
 struct DecodeSmem {
@@ -321,6 +322,24 @@ __device__ __forceinline__ bool mbar_try_wait(unsigned long long *bar, uint32_t 
   return ok != 0;
 }
 
+__device__ __forceinline__ uint64_t global_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Waits for the phase `parity` of the barrier; false if it has not completed
+// within kWaitLimitNs.
+__device__ __forceinline__ bool mbar_wait_bounded(unsigned long long *bar, uint32_t parity) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_ns();
+  for (;;) {
+    for (int i = 0; i < 64; i++)
+      if (mbar_try_wait(bar, parity)) return true;
+    if (global_ns() - t0 > kWaitLimitNs) return false;
+  }
+}
+
 __device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t bytes, unsigned long long *bar) {
   asm volatile(
       "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
@@ -341,6 +360,14 @@ __device__ __forceinline__ uint2 ld_nc8(const void *p) {
   uint2 v;
   asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "l"(p));
   return v;
+}
+
+// Byte permute with the sign-replicating selector bit (PTX prmt, default
+// mode: selector nibble bit 3 set = the selected byte's top bit repeated).
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+  return d;
 }
 
 // Named barrier shared by both groups (ids 1 and 2 are the groups' own).
@@ -368,10 +395,11 @@ __device__ __forceinline__ bool gsync_or(uint32_t id, bool pred) {
 }
 
 // Exclusive scan of v over the group with one barrier, which also ORs `pred`
-// over the group (*any).  Every warp reduces the warp totals itself.
+// over the group (*any).  Every warp reduces the warp totals itself.  wsum
+// must alternate between consecutive calls (a warp may write the next call's
+// total while another still reads this one's).
 __device__ __forceinline__ uint32_t group_excl_scan_or(uint32_t v, bool pred, uint32_t *wsum, uint32_t *total,
                                                        bool *any, uint32_t id, uint32_t gtid) {
-  constexpr uint32_t kWarps = kGroupThreads / 32;
   const uint32_t lane = gtid & 31u, warp = gtid >> 5;
   uint32_t x = v;
   #pragma unroll
@@ -381,7 +409,7 @@ __device__ __forceinline__ uint32_t group_excl_scan_or(uint32_t v, bool pred, ui
   }
   if (lane == 31) wsum[warp] = x;
   *any = gsync_or(id, pred);
-  const uint32_t t = lane < kWarps ? wsum[lane] : 0u;
+  const uint32_t t = lane < kGroupWarps ? wsum[lane] : 0u;
   uint32_t pre = lane < warp ? t : 0u, all = t;
   #pragma unroll
   for (int o = 16; o; o >>= 1) {
@@ -392,252 +420,274 @@ __device__ __forceinline__ uint32_t group_excl_scan_or(uint32_t v, bool pred, ui
   return pre + x - v;
 }
 
-// Packs decoded exponents four to a word into the exponent buffer, which
-// is zeroed before each chunk.  Words are combined with OR, so the words a run
-// shares with its neighbours need no special case.
-template <bool kOwn = false>
-struct ExpWriter {
-  uint32_t *words;  // exponent buffer as words
-  uint32_t wi;      // word being filled (exponents 4*wi .. 4*wi+3)
-  uint32_t s;       // bits of that word filled so far (those below the run are zero)
-  uint32_t acc;
-  __device__ __forceinline__ void init(uint8_t *e, uint32_t j) {
-    words = (uint32_t *)e;
-    wi = j >> 2;
-    s = 8 * (j & 3u);
-    acc = 0;
-  }
-  // kOwn: the run owns every word it touches (it starts on a word), so the
-  // words are stored, not OR-ed into a cleared buffer
-  __device__ __forceinline__ void store(uint32_t v) {
-    if (kOwn) words[wi + (wi >> 5)] = v;  // word wi of the padded rows
-    else atomicOr(words + wi + (wi >> 5), v);
+// A run of decoded symbols written as whole 32-bit words of the exponent
+// buffer, which the run owns: four symbols to a word, first in the low byte.
+// The current word is stored after every append, complete or not (a later
+// append completes it), so no append branches.
+struct RunWriter {
+  uint32_t *pw;  // word being filled
+  uint32_t lo;   // its bytes so far (those above f are zero)
+  uint32_t f;    // bits of it filled: 0, 8, 16 or 24
+  __device__ __forceinline__ void init(uint8_t *exps, uint32_t j) {  // j: a multiple of 4
+    pw = (uint32_t *)(exps + j);
+    lo = 0;
+    f = 0;
   }
   // up to four symbols, first in the low byte, zero above; k8 = 8 * count
   __device__ __forceinline__ void put(uint32_t syms, uint32_t k8) {
-    const uint32_t lo = acc | (syms << s);
-    const uint32_t hi = __funnelshift_l(syms, 0u, s);  // the bytes past the word; none for s = 0
-    s += k8;
-    if (s >= 32) {
-      store(lo);
-      wi++;
-      acc = hi;
-      s -= 32;
-    } else {
-      acc = lo;
-    }
+    const uint32_t t = lo | (syms << f);
+    const uint32_t h = __funnelshift_l(syms, 0u, f);  // the bytes past the word; none for f = 0
+    *pw = t;
+    f += k8;
+    const bool full = f >= 32;
+    lo = full ? h : t;
+    pw += full ? 1 : 0;
+    f &= 31u;
   }
+  // a run that ends inside a word (a chunk's last run): its last bytes
   __device__ __forceinline__ void finish() {
-    if (s) store(acc);
+    if (f) *pw = lo;
   }
 };
 
-// the low r8 / 8 bytes of a word (r8 a multiple of 8, at most 32)
-__device__ __forceinline__ uint32_t low_bytes_mask(uint32_t r8) { return r8 >= 32 ? ~0u : (1u << r8) - 1u; }
-
 // Steps 2-5 for one chunk whose bits are [rel0, rel0 + nbits) of `words`,
 // decoded by one group.  Returns false (group-uniform) if the chunk is
-// corrupt.
+// corrupt; else *r0, *r1 receive the warp's region [r0, r1) of the chunk's
+// values (r0 a multiple of 16), whose exponents the warp's threads wrote.
 template <bool kSmem>
 __device__ bool decode_chunk(GroupSmem &G, const DecodeTables &T, const uint32_t *words, uint32_t rel0,
-                             uint32_t nbits, uint32_t cnt, uint32_t id, uint32_t gtid, uint32_t *timeout) {
+                             uint32_t nbits, uint32_t cnt, uint32_t id, uint32_t gtid, uint32_t *timeout,
+                             uint32_t *r0, uint32_t *r1) {
+  const uint32_t lane = gtid & 31u;
   // window width: a multiple of the gcd of the code lengths, so that a
   // fixed-length code starts every window on a code boundary
   const uint32_t gq = T.gcd;
   uint32_t W = (nbits + kGroupThreads - 1) / kGroupThreads;
   W = (W + gq - 1) / gq * gq;
   const uint32_t ws = min(gtid * W, nbits), we = min(ws + W, nbits);
-  Peek<kSmem> peek{words};
-  // Bulk decoding runs while 2 * kLutBits bits of the window remain: two
+  // The thread's frame: frame bit q is chunk bit ws + q - q0.
+  const uint32_t q0 = (rel0 + ws) & 31u;
+  const uint32_t qe = q0 + (we - ws);
+  Peek<kSmem> peek{words + ((rel0 + ws) >> 5)};
+  // Bulk counting runs while 2 * kLutBits bits of the window remain: two
   // first-level lookups per 32-bit peek, no window-end handling.
   constexpr uint32_t kBulk = 2 * kLutBits;
 
-  // 2. speculative decode of the own window; record where codes start in
-  //    its first kMaskBits bits
-  uint32_t pos = ws, n = 0;
+  // 2. speculative count of the own window; P = frame position | count << 16.
+  //    Record where codes start in the window's first kMaskBits bits.
+  uint32_t P = q0;
   uint64_t mask = 0;
   bool bad = false;
   // (a) while the recorded bits last
-  while (pos + kBulk <= we && pos - ws < kMaskBits) {
-    const uint32_t x = peek(rel0 + pos);
-    const uint32_t off = pos - ws;
-    const uint32_t m1 = T.l1meta[lut_index(x)];
-    const uint32_t k1 = m1 >> 28, nb1 = (m1 >> 24) & 15u;
-    if (!k1) {
-      uint32_t syms, nb;
-      if (!decode_long(T, x, m1, syms, nb)) { bad = true; break; }
+  for (;;) {
+    const uint32_t q = P & 0xFFFFu;
+    if (q + kBulk > qe || q >= q0 + kMaskBits) break;
+    const uint32_t x = peek(q);
+    const uint32_t m1 = T.l1[lut_index(x)].y;
+    const uint32_t off = q - q0;
+    if (!(m1 & 0xF0000u)) {
+      const uint32_t d = decode_long(T, x);
+      if (!d) { bad = true; break; }
       mask |= 1ull << off;
-      pos += nb;
-      n += 1;
+      P += (d >> 8) + 0x10000u;
       continue;
     }
-    // a prefix with no complete code has count, bits and starts all zero
-    const uint32_t m2 = T.l1meta[lut_index(x << nb1)];
-    mask |= (uint64_t)((m1 >> 7) & 0xFFFu) << off;
-    if (off + nb1 < kMaskBits) mask |= (uint64_t)((m2 >> 7) & 0xFFFu) << (off + nb1);
-    pos += nb1 + ((m2 >> 24) & 15u);
-    n += k1 + (m2 >> 28);
+    // a prefix with no complete code has every field zero; a code always
+    // starts right after the first lookup's codes
+    const uint32_t m2 = T.l1[lut_index(__funnelshift_l(0u, x, m1))].y;
+    mask |= (uint64_t)meta_starts(m1) << off;
+    const uint32_t off2 = off + (m1 & 15u);
+    if (off2 < kMaskBits) mask |= (uint64_t)meta_starts(m2) << off2;
+    P += (m1 & kCountFields) + (m2 & kCountFields);
   }
   // (b) the rest of the window, counting only
-  while (!bad && pos + kBulk <= we) {
-    const uint32_t x = peek(rel0 + pos);
-    const uint32_t m1 = T.l1meta[lut_index(x)];
-    const uint32_t k1 = m1 >> 28, nb1 = (m1 >> 24) & 15u;
-    if (!k1) {
-      uint32_t syms, nb;
-      if (!decode_long(T, x, m1, syms, nb)) { bad = true; break; }
-      pos += nb;
-      n += 1;
+  while (!bad) {
+    const uint32_t q = P & 0xFFFFu;
+    if (q + kBulk > qe) break;
+    const uint32_t x = peek(q);
+    const uint32_t m1 = T.l1[lut_index(x)].y;
+    if (!(m1 & 0xF0000u)) {
+      const uint32_t d = decode_long(T, x);
+      if (!d) { bad = true; break; }
+      P += (d >> 8) + 0x10000u;
       continue;
     }
-    const uint32_t m2 = T.l1meta[lut_index(x << nb1)];
-    pos += nb1 + ((m2 >> 24) & 15u);
-    n += k1 + (m2 >> 28);
+    const uint32_t m2 = T.l1[lut_index(__funnelshift_l(0u, x, m1))].y;
+    P += (m1 & kCountFields) + (m2 & kCountFields);
   }
   // (c) the window's last bits, taking only codes that start inside it
-  while (!bad && pos < we) {
-    uint32_t syms, nb, bnd;
-    const uint32_t k = decode_step<false>(T, peek(rel0 + pos), we - pos, syms, nb, bnd);
+  while (!bad) {
+    const uint32_t q = P & 0xFFFFu;
+    if (q >= qe) break;
+    uint32_t nb, bnd;
+    const uint32_t k = count_step(T, peek(q), qe - q, nb, bnd);
     if (!k) { bad = true; break; }
-    const uint32_t off = pos - ws;
+    const uint32_t off = q - q0;
     if (off < kMaskBits) mask |= (uint64_t)bnd << off;
-    pos += nb;
-    n += k;
+    P += nb + (k << 16);
   }
-  const uint32_t spec_end = bad ? we : pos, spec_n = n;
+  const uint32_t spec_end = bad ? we : ws + (P & 0xFFFFu) - q0, spec_n = P >> 16;
   const uint64_t spec_mask = bad ? 0ull : mask;
   uint32_t my_start = ws, my_end = spec_end, my_n = spec_n;
   G.ends[gtid] = my_end;
   gsync(id);
 
-  // 3. fix-up rounds: restart from the predecessor's end until a code starts
-  //    where a speculative one did (from there on the speculative decode is
-  //    right)
+  // 3-4. fix-up round: restart from the predecessor's end until a code starts
+  //    where a speculative one did (from there on the speculative count is
+  //    right); then the scan of the counts, whose barrier also tells whether
+  //    any end moved.  A successor may read an end in the round it moves,
+  //    before or after the store: an older end only costs it another round.
+  uint32_t o, total;
   for (uint32_t round = 0;; round++) {
     const uint32_t pred = gtid == 0 ? 0u : G.ends[gtid - 1];
     bool changed = false;
     if (gtid > 0 && pred != my_start) {
       my_start = pred;
-      uint32_t p = pred, k = 0;
+      uint32_t q = pred - ws + q0, k = 0;
       bool synced = false, bad2 = false;
-      while (p < we) {
-        uint32_t syms, nb, bnd;
-        const uint32_t kk = decode_step<false>(T, peek(rel0 + p), we - p, syms, nb, bnd);
+      while (q < qe) {
+        uint32_t nb, bnd;
+        const uint32_t kk = count_step(T, peek(q), qe - q, nb, bnd);
         if (!kk) { bad2 = true; break; }
-        const uint32_t off = p - ws;
+        const uint32_t off = q - q0;
         if (off < kMaskBits) {
           const uint64_t common = ((uint64_t)bnd << off) & spec_mask;
           if (common) {
-            const uint32_t q = __ffsll(common) - 1;  // offset from ws, >= off
-            k += __popc(bnd & ((1u << (q - off)) - 1u));
-            p = ws + q;
+            const uint32_t s = __ffsll(common) - 1;  // offset from q0, >= off
+            k += __popc(bnd & ((1u << (s - off)) - 1u));
+            q = q0 + s;
             synced = true;
             break;
           }
         }
-        p += nb;
+        q += nb;
         k += kk;
       }
       uint32_t new_end;
       if (synced) {
-        my_n = k + spec_n - __popcll(spec_mask & ((1ull << (p - ws)) - 1ull));
+        my_n = k + spec_n - __popcll(spec_mask & ((1ull << (q - q0)) - 1ull));
         new_end = spec_end;
         bad = false;
       } else {
         my_n = k;
-        new_end = bad2 ? we : p;
+        new_end = bad2 ? we : ws + q - q0;
         bad = bad2;
       }
       changed = new_end != my_end;
       my_end = new_end;
     }
-    // A successor may read this end in the same round, before or after the
-    // store: an older end only costs it another round, and a round in which
-    // no end moved (seen by everyone after the barrier) ends the fix-up.
     if (changed) G.ends[gtid] = my_end;
-    if (!gsync_or(id, changed)) break;
+    // a bad window adds a count no chunk has, so the total check fails
+    bool any_changed;
+    o = group_excl_scan_or(my_n + (bad ? 0x100000u : 0u), changed, G.wsum[round & 1], &total, &any_changed,
+                           id, gtid);
+    if (!any_changed) break;
     if (round > kGroupThreads + 1) {  // cannot happen for consistent data
       if (gtid == 0) *timeout = 1;
-      bad = true;
+      total = ~0u;
       break;
     }
   }
-
-  // 4. output index of every thread's first code
-  uint32_t total;
-  bool anybad;
-  const uint32_t o = group_excl_scan_or(my_n, bad, G.wsum, &total, &anybad, id, gtid);
-  const bool ok = !anybad && total == cnt && G.ends[kGroupThreads - 1] == nbits;
+  const bool ok = total == cnt && G.ends[kGroupThreads - 1] == nbits;
   if (!ok) return false;
 
-  // 5. decode again from the true start, writing exactly the thread's my_n
-  //    exponents (a count, not the window end, stops the loop)
-  ExpWriter<> out;
-  out.init(G.exps, o);
-  pos = gtid == 0 ? 0u : G.ends[gtid - 1];
-  uint32_t rem8 = 8 * my_n;  // exponent bits still to write
-  while (rem8) {
-    const uint32_t x = peek(rel0 + pos);
-    const uint32_t i1 = lut_index(x);
-    const uint32_t m1 = T.l1meta[i1];
-    const uint32_t k1 = (m1 >> 1) & 0x38u, nb1 = m1 & 15u;  // k1: 8 * codes
-    if (!k1) {
-      uint32_t syms, nb;
-      if (!decode_long(T, x, m1, syms, nb)) break;
-      pos += nb;
-      out.put(syms, 8);
-      rem8 -= 8;
-      continue;
+  // 5. the thread's run: from the first multiple of 4 (16 for a warp's first
+  //    thread, so that every warp's region is whole 16-value vectors) at or
+  //    after its first output index, to where the next thread's run starts
+  const uint32_t o1 = o + my_n;
+  const uint32_t a0 = gtid == 0 ? 0u : min(lane == 0 ? (o + 15u) & ~15u : (o + 3u) & ~3u, cnt);
+  const uint32_t a1 =
+      gtid == kGroupThreads - 1 ? cnt : min(lane == 31 ? (o1 + 15u) & ~15u : (o1 + 3u) & ~3u, cnt);
+  *r0 = __shfl_sync(0xffffffffu, a0, 0);
+  *r1 = __shfl_sync(0xffffffffu, a1, 31);
+  if (a1 > a0) {
+    uint32_t skip = a0 - o;  // codes before the run (the previous run's last ones)
+    uint32_t rem8 = 8u * (a1 - a0);
+    uint32_t q = (gtid == 0 ? 0u : G.ends[gtid - 1]) - ws + q0;
+    RunWriter out;
+    out.init(G.exps, a0);
+    // skip, then take the rest of the lookup that crosses into the run
+    while (skip) {
+      const uint32_t x = peek(q);
+      const uint2 e = T.l1[lut_index(x)];
+      uint32_t k = e.y >> 27, nb = (e.y >> 20) & 15u, syms = e.x;  // k: up to four codes
+      if (!k) {
+        const uint32_t d = decode_long(T, x);
+        if (!d) break;
+        syms = d & 0xFFu;
+        nb = d >> 8;
+        k = 1;
+      }
+      q += nb;
+      if (k <= skip) {
+        skip -= k;
+        continue;
+      }
+      const uint32_t take8 = min(8u * (k - skip), rem8);
+      out.put((syms >> (8 * skip)) & ((take8 >= 32 ? 0u : 1u << take8) - 1u), take8);
+      rem8 -= take8;
+      skip = 0;
     }
-    const uint32_t s1 = T.l1sym[i1];
-    if (k1 >= rem8) {  // the last codes of the thread
-      out.put(s1 & low_bytes_mask(rem8), rem8);
-      break;
+    // bulk: two lookups per 32-bit peek while more than eight symbols remain
+    while (rem8 > 64) {
+      const uint32_t x = peek(q);
+      const uint2 e1 = T.l1[lut_index(x)];
+      if (e1.y < (1u << 24)) {  // no complete code in the index bits
+        const uint32_t d = decode_long(T, x);
+        if (!d) break;
+        out.put(d & 0xFFu, 8);
+        rem8 -= 8;
+        q += d >> 8;
+        continue;
+      }
+      const uint32_t s1 = e1.y >> 20;  // bits of the first codes (low 4 bits) | 8 * their number << 4
+      const uint2 e2 = T.l1[lut_index(__funnelshift_l(0u, x, s1))];
+      const uint32_t s2 = e2.y >> 20;
+      out.put(e1.x, s1 >> 4);
+      out.put(e2.x, s2 >> 4);
+      q += (s1 & 15u) + (s2 & 15u);
+      rem8 -= (s1 >> 4) + (s2 >> 4);
     }
-    out.put(s1, k1);
-    rem8 -= k1;
-    const uint32_t i2 = lut_index(x << nb1);
-    const uint32_t m2 = T.l1meta[i2];
-    const uint32_t k2 = (m2 >> 1) & 0x38u, nb2 = m2 & 15u;
-    if (!k2) {
-      pos += nb1;
-      continue;
+    // the run's last symbols, one lookup at a time
+    while (rem8) {
+      const uint32_t x = peek(q);
+      const uint2 e = T.l1[lut_index(x)];
+      uint32_t k8 = e.y >> 24, nb = (e.y >> 20) & 15u, syms = e.x;
+      if (!k8) {
+        const uint32_t d = decode_long(T, x);
+        if (!d) break;
+        syms = d & 0xFFu;
+        nb = d >> 8;
+        k8 = 8;
+      }
+      if (k8 >= rem8) {
+        out.put(syms & (rem8 >= 32 ? ~0u : (1u << rem8) - 1u), rem8);
+        rem8 = 0;
+        break;
+      }
+      out.put(syms, k8);
+      rem8 -= k8;
+      q += nb;
     }
-    const uint32_t s2 = T.l1sym[i2];
-    if (k2 >= rem8) {
-      out.put(s2 & low_bytes_mask(rem8), rem8);
-      break;
-    }
-    out.put(s2, k2);
-    rem8 -= k2;
-    pos += nb1 + nb2;
+    out.finish();
+    if (rem8) *timeout |= 2u;  // an invalid code after the count accepted the chunk
   }
-  out.finish();
-  gsync(id);
+  __syncwarp();
   return true;
-}
-
-// Bits taken by the first r (1..4) of the codes that start at the set bits
-// of bm (offsets from the lookup position), when the lookup holds kk >= r
-// complete codes ending at bit nb.
-__device__ __forceinline__ uint32_t bits_of_first(uint32_t bm, uint32_t r, uint32_t kk, uint32_t nb) {
-  if (r >= kk) return nb;
-  #pragma unroll
-  for (int i = 0; i < 4; i++)
-    if ((uint32_t)i < r) bm &= bm - 1u;  // drop the first r code starts
-  return __ffs(bm) - 1u;                  // the start of code r + 1
 }
 
 // Steps 2-5 with a value index: thread t writes values [128t, 128t + 128) of
 // the chunk from the bit vidx[t] on; no boundary search, no count, no scan.
-// The run must end exactly at the next entry (or the chunk's end), else the
-// chunk is reported corrupt.  Returns false (group-uniform) if corrupt.
+// The run must end exactly at the next entry (or the chunk's end); a thread
+// whose run does not returns false.  *r0, *r1 receive the warp's region.
 template <bool kSmem>
 __device__ bool decode_chunk_indexed(GroupSmem &G, const DecodeTables &T, const uint32_t *words, uint32_t rel0,
-                                     uint32_t nbits, uint32_t cnt, uint32_t id, uint32_t gtid,
-                                     const uint32_t *vidx, uint32_t per) {
-  Peek<kSmem> peek{words};
+                                     uint32_t nbits, uint32_t cnt, uint32_t gtid, const uint32_t *vidx,
+                                     uint32_t per, uint32_t *r0, uint32_t *r1) {
   const uint32_t j0 = gtid * kIndexStride;
+  const uint32_t wbase = (gtid & ~31u) * kIndexStride;
+  *r0 = min(wbase, cnt);
+  *r1 = min(wbase + 32 * kIndexStride, cnt);
   uint32_t start = 0, stop = 0, n = 0;
   bool bad = false;
   if (gtid < per && j0 < cnt) {
@@ -646,66 +696,80 @@ __device__ bool decode_chunk_indexed(GroupSmem &G, const DecodeTables &T, const 
     stop = (gtid + 1 < per && j0 + kIndexStride < cnt) ? __ldg(vidx + gtid + 1) : nbits;
     bad = start > stop || stop > nbits || stop - start < n || stop - start > 32u * n;
   }
-  // also orders the caller's clearing of the exponent buffer before the writes
-  if (gsync_or(id, bad)) return false;
-
-  ExpWriter<true> out;  // runs start on multiples of 128 values: whole words
-  out.init(G.exps, j0);
-  uint32_t pos = start, rem8 = 8 * n;
-  while (rem8 && pos < stop) {
-    const uint32_t x = peek(rel0 + pos);
-    const uint32_t i1 = lut_index(x);
-    const uint32_t m1 = T.l1meta[i1];
-    const uint32_t k1 = (m1 >> 1) & 0x38u, nb1 = m1 & 15u;  // k1: 8 * codes
-    if (!k1) {
-      uint32_t syms, nb;
-      if (!decode_long(T, x, m1, syms, nb)) { bad = true; break; }
-      pos += nb;
-      out.put(syms, 8);
-      rem8 -= 8;
-      continue;
+  if (!bad && n) {
+    Peek<kSmem> peek{words + ((rel0 + start) >> 5)};
+    const uint32_t q0 = (rel0 + start) & 31u;
+    uint32_t q = q0;
+    const uint32_t qe = q0 + (stop - start);
+    RunWriter out;  // runs start on multiples of 128 values: whole words
+    out.init(G.exps, j0);
+    uint32_t rem8 = 8 * n;
+    while (rem8 > 64 && q < qe) {
+      const uint32_t x = peek(q);
+      const uint2 e1 = T.l1[lut_index(x)];
+      if (e1.y < (1u << 24)) {
+        const uint32_t d = decode_long(T, x);
+        if (!d) { bad = true; break; }
+        out.put(d & 0xFFu, 8);
+        rem8 -= 8;
+        q += d >> 8;
+        continue;
+      }
+      const uint32_t s1 = e1.y >> 20;
+      const uint2 e2 = T.l1[lut_index(__funnelshift_l(0u, x, s1))];
+      const uint32_t s2 = e2.y >> 20;
+      out.put(e1.x, s1 >> 4);
+      out.put(e2.x, s2 >> 4);
+      q += (s1 & 15u) + (s2 & 15u);
+      rem8 -= (s1 >> 4) + (s2 >> 4);
     }
-    const uint32_t s1 = T.l1sym[i1];
-    if (k1 >= rem8) {  // the run's last codes
-      out.put(s1 & low_bytes_mask(rem8), rem8);
-      pos += bits_of_first((m1 >> 7) & 0xFFFu, rem8 >> 3, k1 >> 3, nb1);
-      rem8 = 0;
-      break;
+    while (!bad && rem8 && q < qe) {
+      const uint32_t x = peek(q);
+      const uint2 e = T.l1[lut_index(x)];
+      uint32_t k8 = e.y >> 24, nb = (e.y >> 20) & 15u, syms = e.x;
+      if (!k8) {
+        const uint32_t d = decode_long(T, x);
+        if (!d) { bad = true; break; }
+        syms = d & 0xFFu;
+        nb = d >> 8;
+        k8 = 8;
+      }
+      if (k8 >= rem8) {
+        // bits of the first rem8 / 8 codes: up to the start of the next one
+        const uint32_t r = rem8 >> 3;
+        if (r < (k8 >> 3)) {
+          uint32_t bm = meta_starts(e.y);
+          for (uint32_t i = 0; i < r; i++) bm &= bm - 1u;  // drop the first r code starts
+          nb = __ffs(bm) - 1u;
+        }
+        out.put(syms & (rem8 >= 32 ? ~0u : (1u << rem8) - 1u), rem8);
+        q += nb;
+        rem8 = 0;
+        break;
+      }
+      out.put(syms, k8);
+      rem8 -= k8;
+      q += nb;
     }
-    out.put(s1, k1);
-    rem8 -= k1;
-    const uint32_t i2 = lut_index(x << nb1);
-    const uint32_t m2 = T.l1meta[i2];
-    const uint32_t k2 = (m2 >> 1) & 0x38u, nb2 = m2 & 15u;
-    if (!k2) {
-      pos += nb1;
-      continue;
-    }
-    const uint32_t s2 = T.l1sym[i2];
-    if (k2 >= rem8) {
-      out.put(s2 & low_bytes_mask(rem8), rem8);
-      pos += nb1 + bits_of_first((m2 >> 7) & 0xFFFu, rem8 >> 3, k2 >> 3, nb2);
-      rem8 = 0;
-      break;
-    }
-    out.put(s2, k2);
-    rem8 -= k2;
-    pos += nb1 + nb2;
+    out.finish();
+    bad = bad || rem8 != 0 || q != qe;
   }
-  out.finish();
-  bad = bad || rem8 != 0 || pos != stop;
-  return !gsync_or(id, bad);
+  return !__any_sync(0xffffffffu, bad);
 }
 
-// (sign+mantissa, exponent) byte pairs [s0, e0, s1, e1] -> two BF16 values
-__device__ __forceinline__ uint32_t bf16_merge2(uint32_t p) {
-  return (p & 0x007F007Fu) | ((p >> 1) & 0x7F807F80u) | ((p & 0x00800080u) << 8);
+// (sign+mantissa word, rotated exponent word) of four values -> four BF16
+// values: bytes [sm, sign of sm] against [r, r] under the mask 0x807F807F.
+__device__ __forceinline__ uint2 bf16_merge4(uint32_t smw, uint32_t ew) {
+  constexpr uint32_t kM = 0x807F807Fu;
+  const uint32_t x0 = prmt(smw, 0u, 0x9180u), r0 = prmt(ew, 0u, 0x1100u);
+  const uint32_t x1 = prmt(smw, 0u, 0xB3A2u), r1 = prmt(ew, 0u, 0x3322u);
+  return make_uint2((x0 & kM) | (r0 & ~kM), (x1 & kM) | (r1 & ~kM));
 }
 
 // four sign+mantissa nibbles (16 bits) and four exponent bytes -> 4 FP8 values
 __device__ __forceinline__ uint32_t fp8_merge4(uint32_t nib16, uint32_t e4) {
-  const uint32_t t = (nib16 & 0xFu) | ((nib16 & 0xF0u) << 4) | ((nib16 & 0xF00u) << 8) | ((nib16 & 0xF000u) << 12);
-  return ((t & 0x08080808u) << 4) | ((e4 << 3) & 0x78787878u) | (t & 0x07070707u);
+  const uint32_t t = prmt(nib16 & 0x0F0Fu, (nib16 >> 4) & 0x0F0Fu, 0x5140u);  // one nibble per byte
+  return ((t << 4) & 0x80808080u) | (t & 0x07070707u) | (e4 << 3);
 }
 
 // Where one chunk's bits are and whether they fit a shared-memory stage.
@@ -777,34 +841,129 @@ __device__ __forceinline__ ChunkInfo chunk_info(const Batch &b, uint32_t g) {
   return ci;
 }
 
-__device__ __forceinline__ void issue_stage(GroupSmem &G, const Batch &b, const ChunkInfo &ci) {
-  mbar_expect_tx(&G.mbar, ci.bytes);
-  bulk_g2s(G.stage, b.item[ci.item].stream + ci.lo, ci.bytes, &G.mbar);
+__device__ __forceinline__ void issue_stage(GroupSmem &G, const uint8_t *src, uint32_t bytes) {
+  mbar_expect_tx(&G.mbar, bytes);
+  bulk_g2s(G.stage, src, bytes, &G.mbar);
+  G.issued++;
+}
+
+// 6. merge the exponents of values [r0, r1) of a chunk (r0 a multiple of 16)
+// with their sign/mantissa bytes and store them: one warp, 16-byte stores.
+// `exps` holds the exponents in output form; `raw` (page store) instead
+// points at the plain exponent bytes of values [0, cnt) in global memory.
+template <int DT, bool kRaw>
+__device__ __forceinline__ void merge_region(const Item &I, const ChunkInfo &ci, const uint8_t *exps,
+                                             const uint8_t *raw, uint32_t r0, uint32_t r1, uint32_t lane) {
+  const uint32_t v0 = r0 / 16, v1 = r1 / 16;
+  const uint32_t cnt = ci.cnt;
+  auto exp_word4 = [&](uint32_t v) -> uint4 {
+    if (!kRaw) return *(const uint4 *)(exps + 16 * v);
+    uint4 w = __ldg((const uint4 *)(raw + 16 * (uint64_t)v));
+    if (DT == EH_BF16) {  // plain exponents -> output form
+      w.x = ((w.x >> 1) & 0x7F7F7F7Fu) | ((w.x << 7) & 0x80808080u);
+      w.y = ((w.y >> 1) & 0x7F7F7F7Fu) | ((w.y << 7) & 0x80808080u);
+      w.z = ((w.z >> 1) & 0x7F7F7F7Fu) | ((w.z << 7) & 0x80808080u);
+      w.w = ((w.w >> 1) & 0x7F7F7F7Fu) | ((w.w << 7) & 0x80808080u);
+    }
+    return w;
+  };
+  auto exp_byte = [&](uint32_t i) -> uint32_t {
+    if (!kRaw) return exps[i];
+    const uint32_t e = raw[i];
+    return DT == EH_BF16 ? ((e >> 1) | ((e & 1u) << 7)) : e;
+  };
+  if (DT == EH_BF16) {
+    const uint8_t *smp = I.sm + ci.sm_off;
+    uint16_t *outp = (uint16_t *)I.out + ci.out_off;
+    for (uint32_t b0 = v0 + lane; b0 < v1; b0 += 4 * 32) {
+      uint4 m[4];
+      #pragma unroll
+      for (int u = 0; u < 4; u++) {
+        const uint32_t v = b0 + u * 32;
+        m[u] = v < v1 ? ld_nc16(smp + 16 * (uint64_t)v) : make_uint4(0, 0, 0, 0);
+      }
+      #pragma unroll
+      for (int u = 0; u < 4; u++) {
+        const uint32_t v = b0 + u * 32;
+        if (v < v1) {
+          const uint4 e = exp_word4(v);
+          const uint2 a = bf16_merge4(m[u].x, e.x), c = bf16_merge4(m[u].y, e.y);
+          const uint2 d = bf16_merge4(m[u].z, e.z), f = bf16_merge4(m[u].w, e.w);
+          uint4 *dst = (uint4 *)(outp + 16 * (uint64_t)v);
+          dst[0] = make_uint4(a.x, a.y, c.x, c.y);
+          dst[1] = make_uint4(d.x, d.y, f.x, f.y);
+        }
+      }
+    }
+    if (r1 == cnt)
+      for (uint32_t i = max(v1 * 16, r0) + lane; i < cnt; i += 32) {
+        const uint32_t sm = smp[i], r = exp_byte(i);
+        outp[i] = (uint16_t)(((sm & 0x80u) << 8) | ((r & 0x7Fu) << 8) | (r & 0x80u) | (sm & 0x7Fu));
+      }
+  } else if (DT == EH_BYTES) {
+    // the decoded symbols are the output bytes
+    uint8_t *outp = (uint8_t *)I.out + ci.out_off;
+    for (uint32_t v = v0 + lane; v < v1; v += 32) *(uint4 *)(outp + 16 * (uint64_t)v) = exp_word4(v);
+    if (r1 == cnt)
+      for (uint32_t i = max(v1 * 16, r0) + lane; i < cnt; i += 32) outp[i] = (uint8_t)exp_byte(i);
+  } else {
+    const uint8_t *smp = I.sm + ci.sm_off;
+    uint8_t *outp = (uint8_t *)I.out + ci.out_off;
+    for (uint32_t b0 = v0 + lane; b0 < v1; b0 += 4 * 32) {
+      uint2 m[4];
+      #pragma unroll
+      for (int u = 0; u < 4; u++) {
+        const uint32_t v = b0 + u * 32;
+        m[u] = v < v1 ? ld_nc8(smp + 8 * (uint64_t)v) : make_uint2(0, 0);
+      }
+      #pragma unroll
+      for (int u = 0; u < 4; u++) {
+        const uint32_t v = b0 + u * 32;
+        if (v < v1) {
+          const uint4 e = exp_word4(v);
+          uint4 o;
+          o.x = fp8_merge4(m[u].x & 0xFFFFu, e.x);
+          o.y = fp8_merge4(m[u].x >> 16, e.y);
+          o.z = fp8_merge4(m[u].y & 0xFFFFu, e.z);
+          o.w = fp8_merge4(m[u].y >> 16, e.w);
+          *(uint4 *)(outp + 16 * (uint64_t)v) = o;
+        }
+      }
+    }
+    if (r1 == cnt)
+      for (uint32_t i = max(v1 * 16, r0) + lane; i < cnt; i += 32) {
+        const uint32_t sm = (smp[i / 2] >> (4 * (i & 1))) & 0xFu, e = exp_byte(i);
+        outp[i] = (uint8_t)(((sm & 8u) << 4) | (e << 3) | (sm & 7u));
+      }
+  }
 }
 
 // Persistent: CTA i of G decodes the contiguous chunk range
 // [i*C/G, (i+1)*C/G), split into runs of one tensor (one codebook); inside a
-// run the two groups take alternate chunks.  Each group copies its next
-// chunk's stream bits while it merges and stores the current one.
+// run the two groups take alternate chunks.  The last warp of a group to
+// finish writing a chunk's exponents (and so reading its stage) starts the
+// copy of the group's next chunk; every warp then merges its own region.
 template <int DT>
 __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_constant__ Batch b) {
   extern __shared__ __align__(128) uint8_t smem_raw[];
   DecodeSmem &S = *reinterpret_cast<DecodeSmem *>(smem_raw);
   const uint32_t tid = threadIdx.x;
   const uint32_t grp = tid / kGroupThreads, gtid = tid % kGroupThreads, id = 1 + grp;
+  const uint32_t lane = gtid & 31u;
   GroupSmem &G = S.grp[grp];
   const uint32_t g0 = (uint32_t)(((uint64_t)b.total_chunks * blockIdx.x) / gridDim.x);
   const uint32_t g1 = (uint32_t)(((uint64_t)b.total_chunks * (blockIdx.x + 1)) / gridDim.x);
   if (g0 >= g1) return;
   if (gtid == 0) {
     mbar_init(&G.mbar, 1);
+    G.writers_done = 0;
+    G.issued = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (tid == 0) S.abort_flag = 0;
   pdl_wait();  // the decode tables (and everything before them)
   __syncthreads();
-  uint32_t parity = 0, timeout = 0;
-  bool pending = false;  // a stage copy of this group is in flight
+  uint32_t parity = 0, timeout = 0, landed = 0;  // landed: stage copies of this group waited for
 
   for (uint32_t seg = g0; seg < g1;) {
     const Item &I = b.item[find_item(b, seg)];
@@ -822,26 +981,36 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
     ci.fits = false;
     if (g < seg_end) {
       ci = chunk_info<DT>(b, g);
-      if (ci.fits && gtid == 0) issue_stage(G, b, ci);
-      pending = ci.fits;
+      if (ci.fits && gtid == 0) issue_stage(G, b.item[ci.item].stream + ci.lo, ci.bytes);
     }
     // Stagger the groups by one decode: group 1 starts its first chunk when
     // group 0 has decoded its own and turns to the memory-bound output, so
     // one group's output overlaps the other's decode instead of coinciding.
     const bool stagger = seg_end - seg >= 2;
     if (stagger && grp == 1) named_sync(kStaggerBarrier, kDecThreads);
-    for (; g < seg_end; g += kNumGroups) {
+    for (uint32_t j = 0; g < seg_end; g += kNumGroups, j ^= 1u) {
+      if (g != seg + grp) ci = chunk_info<DT>(b, g);
       const uint32_t cnt = ci.cnt;
       bool ok = ci.ok && !terr && !S.abort_flag;
-
-      // One barrier per chunk before the decode: after it the stage holds the
-      // chunk's stream words in MSB-first order and every thread of the group
-      // is done with the previous chunk's exponent buffer.
-      if (ci.fits) {
-        uint32_t spins = 0;
-        while (!mbar_try_wait(&G.mbar, parity) && ++spins < kSpinLimit) {
+      // The group's next chunk, whose copy the last writer of this one
+      // starts.  Kept by parity: the last writer of the previous chunk may
+      // still be reading the other entry.
+      if (gtid == 0) {
+        const uint32_t gn = g + kNumGroups;
+        G.next_bytes[j] = 0;
+        if (gn < seg_end) {
+          const ChunkInfo cn = chunk_info<DT>(b, gn);
+          if (cn.fits) {
+            G.next_src[j] = b.item[cn.item].stream + cn.lo;
+            G.next_bytes[j] = cn.bytes;
+          }
         }
-        const bool late = spins >= kSpinLimit;
+      }
+
+      // One barrier per chunk before the count: after it the stage holds the
+      // chunk's stream words in MSB-first order.
+      if (ci.fits) {
+        const bool late = !mbar_wait_bounded(&G.mbar, parity);
         if (!late) {
           // stream words to MSB-first order, once, for the peeks
           for (uint32_t i = gtid; i < ci.bytes / 4; i += kGroupThreads) G.stage[i] = bswap32(G.stage[i]);
@@ -856,146 +1025,68 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
           ok = false;
         } else {
           parity ^= 1u;
-          pending = false;
+          landed++;
         }
       } else {
         gsync(id);
       }
+      uint32_t r0 = 0, r1 = 0;  // this warp's region of the chunk's values
+      const uint8_t *raw = nullptr;
       if (ok && ci.raw) {
-        // page stored raw: its exponent bytes go straight to the buffer
-        const uint8_t *src = I.raw_pool + (uint64_t)(ci.raw - 1) * b.chunk_elems;
-        for (uint32_t v = gtid; v < cnt / 16; v += kGroupThreads) {
-          const uint4 x = __ldg((const uint4 *)src + v);
-          uint32_t *d = (uint32_t *)(G.exps + exp_slot(16 * v));  // 4-byte aligned
-          d[0] = x.x;
-          d[1] = x.y;
-          d[2] = x.z;
-          d[3] = x.w;
-        }
-        for (uint32_t i = cnt / 16 * 16 + gtid; i < cnt; i += kGroupThreads) G.exps[exp_slot(i)] = src[i];
-        gsync(id);
+        // page stored raw: the merge reads its exponent bytes from the pool
+        raw = I.raw_pool + (uint64_t)(ci.raw - 1) * b.chunk_elems;
+        const uint32_t per_warp = (cnt + kGroupWarps * 16 - 1) / (kGroupWarps * 16) * 16;
+        r0 = min((gtid >> 5) * per_warp, cnt);
+        r1 = min(r0 + per_warp, cnt);
       } else if (ok) {
         const uint32_t per = b.chunk_elems / kIndexStride;
         const uint32_t *vidx = (I.vindex && !I.page_meta) ? I.vindex + (uint64_t)ci.c * per : nullptr;
-        // the search path ORs exponent words in: clear them (ordered before the
-        // writing pass by the decoder's barriers); indexed runs store whole words
-        if (!vidx)
-          for (uint32_t i = gtid; i < kExpBytes / 16; i += kGroupThreads) ((uint4 *)G.exps)[i] = make_uint4(0, 0, 0, 0);
         const uint32_t *gw = (const uint32_t *)(I.stream + ci.lo);
         if (vidx) {
-          if (ci.fits) ok = decode_chunk_indexed<true>(G, S.tabs, G.stage, ci.rel0, ci.nbits, cnt, id, gtid, vidx, per);
-          else ok = decode_chunk_indexed<false>(G, S.tabs, gw, ci.rel0, ci.nbits, cnt, id, gtid, vidx, per);
-        } else if (ci.fits) {
-          ok = decode_chunk<true>(G, S.tabs, G.stage, ci.rel0, ci.nbits, cnt, id, gtid, &timeout);
+          const bool wok = ci.fits ? decode_chunk_indexed<true>(G, S.tabs, G.stage, ci.rel0, ci.nbits, cnt, gtid,
+                                                                vidx, per, &r0, &r1)
+                                   : decode_chunk_indexed<false>(G, S.tabs, gw, ci.rel0, ci.nbits, cnt, gtid,
+                                                                 vidx, per, &r0, &r1);
+          if (!wok) {
+            if (lane == 0) set_status(b.status, kFlagCorrupt);
+            r1 = r0;  // nothing of this warp's region is written out
+          }
         } else {
-          ok = decode_chunk<false>(G, S.tabs, gw, ci.rel0, ci.nbits, cnt, id, gtid, &timeout);
+          ok = ci.fits ? decode_chunk<true>(G, S.tabs, G.stage, ci.rel0, ci.nbits, cnt, id, gtid, &timeout, &r0, &r1)
+                       : decode_chunk<false>(G, S.tabs, gw, ci.rel0, ci.nbits, cnt, id, gtid, &timeout, &r0, &r1);
+          if (!ok && gtid == 0) set_status(b.status, (timeout & 1u) ? kFlagTimeout | kFlagCorrupt : kFlagCorrupt);
+          if (timeout & 2u) set_status(b.status, kFlagCorrupt);
         }
-        if (!ok && gtid == 0) set_status(b.status, timeout ? kFlagTimeout | kFlagCorrupt : kFlagCorrupt);
       } else if (gtid == 0 && !S.abort_flag) {
         set_status(b.status, kFlagCorrupt);
       }
 
       if (stagger && grp == 0 && g == seg) named_arrive(kStaggerBarrier, kDecThreads);
-      // The stage is free: every read of it came before the decoder's last
-      // barrier, and its generic writes were fenced before the chunk's first
-      // barrier.  Start copying the group's next chunk.
-      ChunkInfo cn;
-      cn.fits = false;
-      if (g + kNumGroups < seg_end && !pending && !S.abort_flag) {
-        cn = chunk_info<DT>(b, g + kNumGroups);
-        if (cn.fits && gtid == 0) issue_stage(G, b, cn);
-        pending = cn.fits;
-      } else if (g + kNumGroups < seg_end) {
-        cn = chunk_info<DT>(b, g + kNumGroups);
-        cn.fits = false;
-      }
-
-      // 6. merge exponents with sign/mantissa, 16-byte coalesced stores
-      if (ok) {
-        const uint32_t nvec = cnt / 16;
-        if (DT == EH_BF16) {
-          const uint8_t *smp = I.sm + ci.sm_off;
-          uint16_t *outp = (uint16_t *)I.out + ci.out_off;
-          for (uint32_t v0 = gtid; v0 < nvec; v0 += 4 * kGroupThreads) {
-            uint4 m[4];
-            #pragma unroll
-            for (int u = 0; u < 4; u++) {
-              const uint32_t v = v0 + u * kGroupThreads;
-              m[u] = v < nvec ? ld_nc16(smp + 16 * (uint64_t)v) : make_uint4(0, 0, 0, 0);
-            }
-            #pragma unroll
-            for (int u = 0; u < 4; u++) {
-              const uint32_t v = v0 + u * kGroupThreads;
-              if (v < nvec) {
-                const uint32_t *ew = (const uint32_t *)(G.exps + exp_slot(16 * v));
-                const uint32_t mw[4] = {m[u].x, m[u].y, m[u].z, m[u].w};
-                uint32_t o[8];
-                #pragma unroll
-                for (int q = 0; q < 4; q++) {
-                  const uint32_t e = ew[q];
-                  o[2 * q] = bf16_merge2(__byte_perm(mw[q], e, 0x5140));
-                  o[2 * q + 1] = bf16_merge2(__byte_perm(mw[q], e, 0x7362));
-                }
-                uint4 *dst = (uint4 *)(outp + 16 * (uint64_t)v);
-                dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
-                dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
-              }
-            }
-          }
-          for (uint32_t i = nvec * 16 + gtid; i < cnt; i += kGroupThreads) {
-            const uint32_t sm = smp[i], e = G.exps[exp_slot(i)];
-            outp[i] = (uint16_t)(((sm & 0x80u) << 8) | (e << 7) | (sm & 0x7Fu));
-          }
-        } else if (DT == EH_BYTES) {
-          // the decoded symbols are the output bytes
-          uint8_t *outp = (uint8_t *)I.out + ci.out_off;
-          for (uint32_t v = gtid; v < nvec; v += kGroupThreads) {
-            const uint32_t *ew = (const uint32_t *)(G.exps + exp_slot(16 * v));
-            *(uint4 *)(outp + 16 * (uint64_t)v) = make_uint4(ew[0], ew[1], ew[2], ew[3]);
-          }
-          for (uint32_t i = nvec * 16 + gtid; i < cnt; i += kGroupThreads) outp[i] = G.exps[exp_slot(i)];
-        } else {
-          const uint8_t *smp = I.sm + ci.sm_off;
-          uint8_t *outp = (uint8_t *)I.out + ci.out_off;
-          for (uint32_t v0 = gtid; v0 < nvec; v0 += 4 * kGroupThreads) {
-            uint2 m[4];
-            #pragma unroll
-            for (int u = 0; u < 4; u++) {
-              const uint32_t v = v0 + u * kGroupThreads;
-              m[u] = v < nvec ? ld_nc8(smp + 8 * (uint64_t)v) : make_uint2(0, 0);
-            }
-            #pragma unroll
-            for (int u = 0; u < 4; u++) {
-              const uint32_t v = v0 + u * kGroupThreads;
-              if (v < nvec) {
-                const uint32_t *ew = (const uint32_t *)(G.exps + exp_slot(16 * v));
-                uint4 o;
-                o.x = fp8_merge4(m[u].x & 0xFFFFu, ew[0]);
-                o.y = fp8_merge4(m[u].x >> 16, ew[1]);
-                o.z = fp8_merge4(m[u].y & 0xFFFFu, ew[2]);
-                o.w = fp8_merge4(m[u].y >> 16, ew[3]);
-                *(uint4 *)(outp + 16 * (uint64_t)v) = o;
-              }
-            }
-          }
-          for (uint32_t i = nvec * 16 + gtid; i < cnt; i += kGroupThreads) {
-            const uint32_t sm = (smp[i / 2] >> (4 * (i & 1))) & 0xFu, e = G.exps[exp_slot(i)];
-            outp[i] = (uint8_t)(((sm & 8u) << 4) | (e << 3) | (sm & 7u));
-          }
+      // The stage is free once every warp of the group has written its runs:
+      // the last one starts copying the group's next chunk.  (The generic
+      // writes of the byte swap were fenced before the chunk's barrier.)
+      __syncwarp();
+      if (lane == 0) {
+        __threadfence_block();
+        if (atomicAdd(&G.writers_done, 1u) == kGroupWarps - 1) {
+          G.writers_done = 0;
+          if (G.next_bytes[j]) issue_stage(G, G.next_src[j], G.next_bytes[j]);
         }
       }
-      // no barrier here: the next chunk's first barrier orders these reads of
-      // the exponent buffer before it is cleared or written again
-      ci = cn;
+
+      // 6. merge this warp's region with the sign/mantissa bytes
+      if (ok && r1 > r0) {
+        if (raw) merge_region<DT, true>(I, ci, G.exps, raw, r0, r1, lane);
+        else merge_region<DT, false>(I, ci, G.exps, raw, r0, r1, lane);
+      }
+      // no barrier here: the next chunk's barriers order these reads of the
+      // exponent buffer before it is written again
     }
     seg = seg_end;
   }
   // a copy still in flight (only after an abort) must land before the exit
-  if (pending) {
-    uint32_t spins = 0;
-    while (!mbar_try_wait(&G.mbar, parity) && ++spins < kSpinLimit) {
-    }
-  }
+  __syncthreads();
+  if (gtid == 0 && G.issued != landed) mbar_wait_bounded(&G.mbar, parity);
   __syncthreads();
 }
 

@@ -17,7 +17,6 @@ constexpr int kThreads = 512;           // threads per CTA of the compress kerne
 constexpr int kDecThreads = 1024;       // threads per CTA of the decoder (one CTA per SM)
 constexpr int kMaxChunk = 65536;        // largest chunk (elements)
 constexpr int kNumSub = 4;              // second-level decode tables per codebook
-constexpr int kStageBytes = 32 * 1024;  // shared-memory window for one chunk's stream
 
 // status word flags (bitwise OR of everything a call observed)
 constexpr uint32_t kFlagCorrupt = 1u;
@@ -111,33 +110,38 @@ __device__ __forceinline__ void set_status(uint32_t *status, uint32_t flag) {
 // Decode tables for one codebook, built by the table kernel into the
 // workspace and copied to shared memory by each decoding CTA.
 //
-// First level, indexed by the next kLutBits stream bits, as two u32 arrays:
-//   l1sym:  the symbols of the first four complete codes, 8 bits each
-//   l1meta: bits  0..3  bits consumed by those (up to four) codes
-//           bits  4..6  their number (0..4)
-//           bits  7..18 bit i set when a complete code starts at offset i
-//           bits 19..23 second-level table of this prefix (kNoSub: none)
-//           bits 24..27 bits consumed by all complete codes in the index
-//           bits 28..31 their number (0..12); counting uses these
-// Second level, indexed by the 8 bits after the prefix.  u32 entry:
-//   bits 0..7 symbol, bits 8..13 code length (0: longer -> search).
-// The search path handles any length up to 32 with the canonical limits.
+// First level, indexed by the next kLutBits stream bits: .x holds the symbols
+// (in the decoder's output form) of the first four complete codes, 8 bits
+// each, first in the low byte; .y is a meta word:
+//   bits  0..3  bits of all complete codes in the index bits
+//   bit   4     zero (a wrap-mode shift by the whole word shifts by bits 0..3)
+//   bits  5..15 a complete code starts at offset 1..11 (offset 0 always does)
+//   bits 16..19 number of complete codes (0: the first code is longer than the
+//               index; then the whole entry is zero)
+//   bits 20..23 bits of the first (up to four) codes
+//   bits 24..31 8 * their number
+// Second level, for the first kNumSub prefixes (from sub0 on) of codes longer
+// than the index, indexed by the 8 bits after the prefix.  u32 entry:
+//   bits 0..7 symbol (output form), bits 8..13 code length (0: longer ->
+//   search).  The search path handles any length up to 32 with the canonical
+//   limits.
 constexpr int kLutBits = 12;
-constexpr uint32_t kNoSub = 31;
-struct DecodeTables {
-  uint32_t l1meta[1 << kLutBits];
-  uint32_t l1sym[1 << kLutBits];
+constexpr uint32_t kMetaStartShift = 5;
+struct alignas(16) DecodeTables {  // copied to shared memory in 16-byte words
+  uint2 l1[1 << kLutBits];
   uint32_t sub[kNumSub][256];
   uint64_t lim[33];        // (first[L] + count[L]) << (32 - L): left-justified limits
   uint32_t first[33];      // first canonical code of length L
   uint32_t base[33];       // index in `sorted` of the first code of length L
-  uint8_t sorted[256];     // symbols in (length, symbol) order
+  uint8_t sorted[256];     // symbols (output form) in (length, symbol) order
+  uint32_t sub0;           // first prefix of a code longer than the index
   uint32_t gcd;            // gcd of the code lengths in use
   uint32_t maxlen;
   uint32_t nsym;
   uint32_t err;            // nonzero: codebook invalid
 };
 
+static_assert(sizeof(DecodeTables) % 16 == 0, "the decoder copies the tables in 16-byte words");
 constexpr uint64_t kLutBytes = (sizeof(DecodeTables) + 255) & ~uint64_t(255);
 
 __host__ __device__ inline uint64_t align256(uint64_t x) { return (x + 255) & ~uint64_t(255); }
