@@ -213,13 +213,25 @@ __device__ __forceinline__ uint32_t meta_starts(uint32_t m) {  // code starts at
 }
 constexpr uint32_t kCountFields = 0x000F000Fu;  // bits of all codes | their number << 16
 
-// 32 stream bits starting at bit q of a thread's frame.  Shared-memory stages
-// are byte-swapped once after the copy, so their words are already
-// MSB-first; global words are swapped on load.
+// 32 stream bits starting at bit q of a thread's frame (stream words are
+// byte-swapped on load to MSB-first order).
+// Shared-memory loads by 32-bit shared address.
+__device__ __forceinline__ uint32_t lds32(uint32_t a) {
+  uint32_t v;
+  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a));
+  return v;
+}
+__device__ __forceinline__ uint2 lds64(uint32_t a) {
+  uint2 v;
+  asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(a));
+  return v;
+}
 template <bool kSmem>
 struct Peek {
   const uint32_t *w;
-  __device__ __forceinline__ uint32_t word(uint32_t i) const { return kSmem ? w[i] : bswap32(__ldg(w + i)); }
+  __device__ __forceinline__ uint32_t word(uint32_t i) const {
+    return bswap32(kSmem ? lds32((uint32_t)__cvta_generic_to_shared(w) + 4 * i) : __ldg(w + i));
+  }
   __device__ __forceinline__ uint32_t operator()(uint32_t q) const {
     const uint32_t i = q >> 5;
     return __funnelshift_l(word(i + 1), word(i), q);  // the shift is taken modulo 32
@@ -249,7 +261,8 @@ __device__ __noinline__ uint32_t decode_long(const DecodeTables &T, uint32_t x) 
 // code), the bits up to the end of the last one and their starts as a bitmap.
 __device__ __forceinline__ uint32_t count_step(const DecodeTables &T, uint32_t x, uint32_t lim, uint32_t &nbits,
                                                uint32_t &bnd) {
-  const uint32_t m = T.l1[lut_index(x)].y;
+  const uint32_t tab = (uint32_t)__cvta_generic_to_shared(&T.l1[0]);
+  const uint32_t m = lds32(tab + 8 * lut_index(x) + 4);
   uint32_t k = (m >> 16) & 15u;
   if (!k) {
     const uint32_t d = decode_long(T, x);
@@ -282,7 +295,10 @@ constexpr uint32_t kGroupStage = 27136;  // bytes of stream staged per group
 
 struct GroupSmem {
   alignas(128) uint32_t stage[kGroupStage / 4 + 16];  // bulk-copy target (stream bytes as stored)
-  alignas(16) uint8_t exps[kMaxChunk];                // decoded exponents (output form) of one chunk
+  // decoded exponents (output form) of one chunk: value j at byte
+  // j + 4 * (j / 128), so that runs starting about 128 values apart store to
+  // different banks
+  alignas(16) uint8_t exps[kMaxChunk + 4 * (kMaxChunk / 128)];
   uint32_t ends[kGroupThreads];                       // end bit of every thread's codes
   uint32_t wsum[2][kGroupWarps];                      // scan: warp totals, by round parity
   alignas(8) unsigned long long mbar;
@@ -425,11 +441,13 @@ __device__ __forceinline__ uint32_t group_excl_scan_or(uint32_t v, bool pred, ui
 // The current word is stored after every append, complete or not (a later
 // append completes it), so no append branches.
 struct RunWriter {
-  uint32_t *pw;  // word being filled
+  uint32_t *base;
+  uint32_t w;    // word being filled (exponents 4w .. 4w+3; stored at word w + w/32)
   uint32_t lo;   // its bytes so far (those above f are zero)
   uint32_t f;    // bits of it filled: 0, 8, 16 or 24
   __device__ __forceinline__ void init(uint8_t *exps, uint32_t j) {  // j: a multiple of 4
-    pw = (uint32_t *)(exps + j);
+    base = (uint32_t *)exps;
+    w = j >> 2;
     lo = 0;
     f = 0;
   }
@@ -437,16 +455,16 @@ struct RunWriter {
   __device__ __forceinline__ void put(uint32_t syms, uint32_t k8) {
     const uint32_t t = lo | (syms << f);
     const uint32_t h = __funnelshift_l(syms, 0u, f);  // the bytes past the word; none for f = 0
-    *pw = t;
+    base[w + (w >> 5)] = t;
     f += k8;
     const bool full = f >= 32;
     lo = full ? h : t;
-    pw += full ? 1 : 0;
+    w += full ? 1 : 0;
     f &= 31u;
   }
   // a run that ends inside a word (a chunk's last run): its last bytes
   __device__ __forceinline__ void finish() {
-    if (f) *pw = lo;
+    if (f) base[w + (w >> 5)] = lo;
   }
 };
 
@@ -457,8 +475,9 @@ struct RunWriter {
 template <bool kSmem>
 __device__ bool decode_chunk(GroupSmem &G, const DecodeTables &T, const uint32_t *words, uint32_t rel0,
                              uint32_t nbits, uint32_t cnt, uint32_t id, uint32_t gtid, uint32_t *timeout,
-                             uint32_t *r0, uint32_t *r1) {
+                             uint32_t *r0, uint32_t *r1, bool late) {
   const uint32_t lane = gtid & 31u;
+  const uint32_t tab = (uint32_t)__cvta_generic_to_shared(&T.l1[0]);
   // window width: a multiple of the gcd of the code lengths, so that a
   // fixed-length code starts every window on a code boundary
   const uint32_t gq = T.gcd;
@@ -483,7 +502,7 @@ __device__ bool decode_chunk(GroupSmem &G, const DecodeTables &T, const uint32_t
     const uint32_t q = P & 0xFFFFu;
     if (q + kBulk > qe || q >= q0 + kMaskBits) break;
     const uint32_t x = peek(q);
-    const uint32_t m1 = T.l1[lut_index(x)].y;
+    const uint32_t m1 = lds32(tab + 8 * lut_index(x) + 4);
     const uint32_t off = q - q0;
     if (!(m1 & 0xF0000u)) {
       const uint32_t d = decode_long(T, x);
@@ -494,7 +513,7 @@ __device__ bool decode_chunk(GroupSmem &G, const DecodeTables &T, const uint32_t
     }
     // a prefix with no complete code has every field zero; a code always
     // starts right after the first lookup's codes
-    const uint32_t m2 = T.l1[lut_index(__funnelshift_l(0u, x, m1))].y;
+    const uint32_t m2 = lds32(tab + 8 * lut_index(__funnelshift_l(0u, x, m1)) + 4);
     mask |= (uint64_t)meta_starts(m1) << off;
     const uint32_t off2 = off + (m1 & 15u);
     if (off2 < kMaskBits) mask |= (uint64_t)meta_starts(m2) << off2;
@@ -505,14 +524,14 @@ __device__ bool decode_chunk(GroupSmem &G, const DecodeTables &T, const uint32_t
     const uint32_t q = P & 0xFFFFu;
     if (q + kBulk > qe) break;
     const uint32_t x = peek(q);
-    const uint32_t m1 = T.l1[lut_index(x)].y;
+    const uint32_t m1 = lds32(tab + 8 * lut_index(x) + 4);
     if (!(m1 & 0xF0000u)) {
       const uint32_t d = decode_long(T, x);
       if (!d) { bad = true; break; }
       P += (d >> 8) + 0x10000u;
       continue;
     }
-    const uint32_t m2 = T.l1[lut_index(__funnelshift_l(0u, x, m1))].y;
+    const uint32_t m2 = lds32(tab + 8 * lut_index(__funnelshift_l(0u, x, m1)) + 4);
     P += (m1 & kCountFields) + (m2 & kCountFields);
   }
   // (c) the window's last bits, taking only codes that start inside it
@@ -530,7 +549,10 @@ __device__ bool decode_chunk(GroupSmem &G, const DecodeTables &T, const uint32_t
   const uint64_t spec_mask = bad ? 0ull : mask;
   uint32_t my_start = ws, my_end = spec_end, my_n = spec_n;
   G.ends[gtid] = my_end;
-  gsync(id);
+  if (gsync_or(id, late)) {  // the stage copy of some thread came late
+    if (gtid == 0) *timeout |= 1u;
+    return false;
+  }
 
   // 3-4. fix-up round: restart from the predecessor's end until a code starts
   //    where a speculative one did (from there on the speculative count is
@@ -591,15 +613,20 @@ __device__ bool decode_chunk(GroupSmem &G, const DecodeTables &T, const uint32_t
   const bool ok = total == cnt && G.ends[kGroupThreads - 1] == nbits;
   if (!ok) return false;
 
-  // 5. the thread's run: from the first multiple of 4 (16 for a warp's first
-  //    thread, so that every warp's region is whole 16-value vectors) at or
-  //    after its first output index, to where the next thread's run starts
+  // 5. the thread's run: from the first multiple of 4 at or after its first
+  //    output index, to where the next thread's run starts.
+  //    The warp's region [rs, re) starts at the first multiple of 16 at or
+  //    after its first thread's first output index; every run is clamped to
+  //    it, so the runs of a warp tile exactly its region and no other warp
+  //    stores into it.
   const uint32_t o1 = o + my_n;
-  const uint32_t a0 = gtid == 0 ? 0u : min(lane == 0 ? (o + 15u) & ~15u : (o + 3u) & ~3u, cnt);
-  const uint32_t a1 =
-      gtid == kGroupThreads - 1 ? cnt : min(lane == 31 ? (o1 + 15u) & ~15u : (o1 + 3u) & ~3u, cnt);
-  *r0 = __shfl_sync(0xffffffffu, a0, 0);
-  *r1 = __shfl_sync(0xffffffffu, a1, 31);
+  const uint32_t rs = __shfl_sync(0xffffffffu, gtid == 0 ? 0u : min((o + 15u) & ~15u, cnt), 0);
+  const uint32_t re =
+      __shfl_sync(0xffffffffu, gtid == kGroupThreads - 1 ? cnt : min((o1 + 15u) & ~15u, cnt), 31);
+  const uint32_t a0 = lane == 0 ? rs : min(max((o + 3u) & ~3u, rs), re);
+  const uint32_t a1 = lane == 31 ? re : min(max((o1 + 3u) & ~3u, rs), re);
+  *r0 = rs;
+  *r1 = re;
   if (a1 > a0) {
     uint32_t skip = a0 - o;  // codes before the run (the previous run's last ones)
     uint32_t rem8 = 8u * (a1 - a0);
@@ -609,7 +636,7 @@ __device__ bool decode_chunk(GroupSmem &G, const DecodeTables &T, const uint32_t
     // skip, then take the rest of the lookup that crosses into the run
     while (skip) {
       const uint32_t x = peek(q);
-      const uint2 e = T.l1[lut_index(x)];
+      const uint2 e = lds64(tab + 8 * lut_index(x));
       uint32_t k = e.y >> 27, nb = (e.y >> 20) & 15u, syms = e.x;  // k: up to four codes
       if (!k) {
         const uint32_t d = decode_long(T, x);
@@ -631,7 +658,7 @@ __device__ bool decode_chunk(GroupSmem &G, const DecodeTables &T, const uint32_t
     // bulk: two lookups per 32-bit peek while more than eight symbols remain
     while (rem8 > 64) {
       const uint32_t x = peek(q);
-      const uint2 e1 = T.l1[lut_index(x)];
+      const uint2 e1 = lds64(tab + 8 * lut_index(x));
       if (e1.y < (1u << 24)) {  // no complete code in the index bits
         const uint32_t d = decode_long(T, x);
         if (!d) break;
@@ -641,7 +668,7 @@ __device__ bool decode_chunk(GroupSmem &G, const DecodeTables &T, const uint32_t
         continue;
       }
       const uint32_t s1 = e1.y >> 20;  // bits of the first codes (low 4 bits) | 8 * their number << 4
-      const uint2 e2 = T.l1[lut_index(__funnelshift_l(0u, x, s1))];
+      const uint2 e2 = lds64(tab + 8 * lut_index(__funnelshift_l(0u, x, s1)));
       const uint32_t s2 = e2.y >> 20;
       out.put(e1.x, s1 >> 4);
       out.put(e2.x, s2 >> 4);
@@ -651,7 +678,7 @@ __device__ bool decode_chunk(GroupSmem &G, const DecodeTables &T, const uint32_t
     // the run's last symbols, one lookup at a time
     while (rem8) {
       const uint32_t x = peek(q);
-      const uint2 e = T.l1[lut_index(x)];
+      const uint2 e = lds64(tab + 8 * lut_index(x));
       uint32_t k8 = e.y >> 24, nb = (e.y >> 20) & 15u, syms = e.x;
       if (!k8) {
         const uint32_t d = decode_long(T, x);
@@ -684,6 +711,7 @@ template <bool kSmem>
 __device__ bool decode_chunk_indexed(GroupSmem &G, const DecodeTables &T, const uint32_t *words, uint32_t rel0,
                                      uint32_t nbits, uint32_t cnt, uint32_t gtid, const uint32_t *vidx,
                                      uint32_t per, uint32_t *r0, uint32_t *r1) {
+  const uint32_t tab = (uint32_t)__cvta_generic_to_shared(&T.l1[0]);
   const uint32_t j0 = gtid * kIndexStride;
   const uint32_t wbase = (gtid & ~31u) * kIndexStride;
   *r0 = min(wbase, cnt);
@@ -706,7 +734,7 @@ __device__ bool decode_chunk_indexed(GroupSmem &G, const DecodeTables &T, const 
     uint32_t rem8 = 8 * n;
     while (rem8 > 64 && q < qe) {
       const uint32_t x = peek(q);
-      const uint2 e1 = T.l1[lut_index(x)];
+      const uint2 e1 = lds64(tab + 8 * lut_index(x));
       if (e1.y < (1u << 24)) {
         const uint32_t d = decode_long(T, x);
         if (!d) { bad = true; break; }
@@ -716,7 +744,7 @@ __device__ bool decode_chunk_indexed(GroupSmem &G, const DecodeTables &T, const 
         continue;
       }
       const uint32_t s1 = e1.y >> 20;
-      const uint2 e2 = T.l1[lut_index(__funnelshift_l(0u, x, s1))];
+      const uint2 e2 = lds64(tab + 8 * lut_index(__funnelshift_l(0u, x, s1)));
       const uint32_t s2 = e2.y >> 20;
       out.put(e1.x, s1 >> 4);
       out.put(e2.x, s2 >> 4);
@@ -725,7 +753,7 @@ __device__ bool decode_chunk_indexed(GroupSmem &G, const DecodeTables &T, const 
     }
     while (!bad && rem8 && q < qe) {
       const uint32_t x = peek(q);
-      const uint2 e = T.l1[lut_index(x)];
+      const uint2 e = lds64(tab + 8 * lut_index(x));
       uint32_t k8 = e.y >> 24, nb = (e.y >> 20) & 15u, syms = e.x;
       if (!k8) {
         const uint32_t d = decode_long(T, x);
@@ -857,7 +885,10 @@ __device__ __forceinline__ void merge_region(const Item &I, const ChunkInfo &ci,
   const uint32_t v0 = r0 / 16, v1 = r1 / 16;
   const uint32_t cnt = ci.cnt;
   auto exp_word4 = [&](uint32_t v) -> uint4 {
-    if (!kRaw) return *(const uint4 *)(exps + 16 * v);
+    if (!kRaw) {
+      const uint32_t *p = (const uint32_t *)(exps + 16 * v + 4 * (v >> 3));  // padded rows
+      return make_uint4(p[0], p[1], p[2], p[3]);
+    }
     uint4 w = __ldg((const uint4 *)(raw + 16 * (uint64_t)v));
     if (DT == EH_BF16) {  // plain exponents -> output form
       w.x = ((w.x >> 1) & 0x7F7F7F7Fu) | ((w.x << 7) & 0x80808080u);
@@ -868,7 +899,7 @@ __device__ __forceinline__ void merge_region(const Item &I, const ChunkInfo &ci,
     return w;
   };
   auto exp_byte = [&](uint32_t i) -> uint32_t {
-    if (!kRaw) return exps[i];
+    if (!kRaw) return exps[i + 4 * (i >> 7)];
     const uint32_t e = raw[i];
     return DT == EH_BF16 ? ((e >> 1) | ((e & 1u) << 7)) : e;
   };
@@ -1009,26 +1040,28 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
 
       // One barrier per chunk before the count: after it the stage holds the
       // chunk's stream words in MSB-first order.
+      // Every thread waits for the chunk's stage copy itself.  The plain
+      // decode's first barrier tells the group whether a copy came late;
+      // every other path takes one barrier here, so that the warps of a
+      // group never drift more than a chunk apart.
+      const uint32_t *vidx = (ok && I.vindex && !I.page_meta) ? I.vindex + (uint64_t)ci.c * (b.chunk_elems / kIndexStride)
+                                                            : nullptr;
+      bool late = false;
       if (ci.fits) {
-        const bool late = !mbar_wait_bounded(&G.mbar, parity);
+        late = !mbar_wait_bounded(&G.mbar, parity);
         if (!late) {
-          // stream words to MSB-first order, once, for the peeks
-          for (uint32_t i = gtid; i < ci.bytes / 4; i += kGroupThreads) G.stage[i] = bswap32(G.stage[i]);
+          parity ^= 1u;
+          landed++;
         }
-        // these generic writes come before the next bulk copy into the stage
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      }
+      if (!ok || ci.raw || vidx) {
         if (gsync_or(id, late)) {
           if (gtid == 0) {
             set_status(b.status, kFlagTimeout);
             S.abort_flag = 1;
           }
           ok = false;
-        } else {
-          parity ^= 1u;
-          landed++;
         }
-      } else {
-        gsync(id);
       }
       uint32_t r0 = 0, r1 = 0;  // this warp's region of the chunk's values
       const uint8_t *raw = nullptr;
@@ -1040,7 +1073,6 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
         r1 = min(r0 + per_warp, cnt);
       } else if (ok) {
         const uint32_t per = b.chunk_elems / kIndexStride;
-        const uint32_t *vidx = (I.vindex && !I.page_meta) ? I.vindex + (uint64_t)ci.c * per : nullptr;
         const uint32_t *gw = (const uint32_t *)(I.stream + ci.lo);
         if (vidx) {
           const bool wok = ci.fits ? decode_chunk_indexed<true>(G, S.tabs, G.stage, ci.rel0, ci.nbits, cnt, gtid,
@@ -1052,8 +1084,8 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
             r1 = r0;  // nothing of this warp's region is written out
           }
         } else {
-          ok = ci.fits ? decode_chunk<true>(G, S.tabs, G.stage, ci.rel0, ci.nbits, cnt, id, gtid, &timeout, &r0, &r1)
-                       : decode_chunk<false>(G, S.tabs, gw, ci.rel0, ci.nbits, cnt, id, gtid, &timeout, &r0, &r1);
+          ok = ci.fits ? decode_chunk<true>(G, S.tabs, G.stage, ci.rel0, ci.nbits, cnt, id, gtid, &timeout, &r0, &r1, late)
+                       : decode_chunk<false>(G, S.tabs, gw, ci.rel0, ci.nbits, cnt, id, gtid, &timeout, &r0, &r1, late);
           if (!ok && gtid == 0) set_status(b.status, (timeout & 1u) ? kFlagTimeout | kFlagCorrupt : kFlagCorrupt);
           if (timeout & 2u) set_status(b.status, kFlagCorrupt);
         }

@@ -78,6 +78,26 @@ def test_small_chunks(eh, oracle, dtype, chunk, n):
     roundtrip(eh, oracle, dtype, x, chunk=chunk)
 
 
+@pytest.mark.parametrize("dtype", [0, 1])
+def test_repeated_small_chunk_decodes_are_exact(eh, oracle, dtype):
+    # 1024-value chunks are decoded in a few microseconds each, so the warps
+    # of a group run far out of step; every warp must store only into its
+    # own region of the exponent buffer, or a merge may read a word that
+    # another warp is still rewriting.  Thirty decodes of the same tensor
+    # must all be exact.
+    n = 1200 * 1024 + 1
+    x = synth.normal_bf16(n, seed=3) if dtype == 0 else synth.normal_fp8(n, seed=3)
+    p = eh.plan(dtype, 1024)
+    c = eh.compress(dev(x), p)
+    assert_same(c, oracle.compress(dtype, x, chunk=1024))
+    t = dev(x)
+    ws = torch.empty(eh.decompress_workspace(p, 1), dtype=torch.uint8, device="cuda")
+    y = torch.empty_like(t)
+    for _ in range(30):
+        eh.decompress(c, p, out=y, workspace=ws)
+        assert torch.equal(y, t)
+
+
 def test_every_bf16_pattern(eh, oracle):
     rng = np.random.default_rng(1)
     x = np.arange(1 << 16, dtype=np.uint16)[rng.permutation(1 << 16)]
