@@ -170,6 +170,10 @@ def run_reference(args):
     desc = "oracle compress+decompress of k_proj (1024x4096 BF16, 8.4 MB) per step"
     line = {
         "impl": "reference", "metric": METRIC, "value": v, "unit": "GB/s", "n_gpus": args.gpus,
+        # `config` names the workload the GPU arm runs; each step of this arm
+        # codes only a bounded sample of it (the metric is a rate)
+        "sample_per_step": {"tensor": "k_proj", "shape": [1024, 4096], "elements": int(sample.size),
+                            "of_workload_elements": 218103808},
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "u16",
         "data": "synthetic", "config": workload_config(args.gpus),

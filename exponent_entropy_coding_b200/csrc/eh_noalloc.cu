@@ -2,13 +2,14 @@
 // device memory.
 //
 // Some callers cannot call cudaMalloc (or any allocating routine) at the point
-// where they need to decompress: code running while a CUDA graph is being
-// captured, runtimes that plan all device memory up front and forbid later
-// allocations, or allocator callbacks that must not re-enter the allocator.
-// eh_decompress_batch_noalloc serves them: the decoder's scratch (the status
-// word and one set of decode tables per tensor) lives in a file-scope device
-// array of fixed size instead of a caller-provided workspace.  The caller
-// still provides the compressed inputs and the output buffers.
+// where they need to decompress: runtimes that plan all device memory up front
+// and forbid later allocations, or allocator callbacks that must not re-enter
+// the allocator.  eh_decompress_batch_noalloc serves them: the decoder's
+// scratch (the status word and one set of decode tables per tensor) lives in a
+// file-scope device array of fixed size instead of a caller-provided
+// workspace.  The caller still provides the compressed inputs and the output
+// buffers.  The call reads the status back and synchronises the stream, so it
+// is not meant for a stream that is being captured into a CUDA graph.
 //
 // The array is allocated by the CUDA runtime in every device context that
 // loads this library and stays there until the process exits.  All calls
@@ -21,29 +22,32 @@
 
 namespace {
 
+static_assert(eh::kLutBytes == 37888, "the header documents 37,888 bytes of decode tables per tensor");
 constexpr uint64_t kNoallocBytes = 256 + (uint64_t)EH_NOALLOC_MAX_BATCH * eh::kLutBytes;
 
 static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoallocBytes];
 
 constexpr int kMaxDevices = 64;
-struct ScratchAddr {
-  std::once_flag once;
-  void *ptr = nullptr;
-  cudaError_t err = cudaSuccess;
-};
-ScratchAddr g_addr[kMaxDevices];
+std::mutex g_addr_mu;
+void *g_addr[kMaxDevices];  // device address of the array, per device (null: not looked up yet)
 
-// Device address of the scratch array on the current device, looked up once
-// per device (the host-side symbol is not a device address).
+// Device address of the scratch array on the current device (the host-side
+// symbol is not a device address).  Only a successful lookup is kept, so a
+// transient failure is retried by the next call.
 cudaError_t scratch_address(void **ptr) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-  ScratchAddr &a = g_addr[dev];
-  std::call_once(a.once, [&a]() { a.err = cudaGetSymbolAddress(&a.ptr, g_noalloc_scratch); });
-  *ptr = a.ptr;
-  return a.err;
+  std::lock_guard<std::mutex> lock(g_addr_mu);
+  if (!g_addr[dev]) {
+    void *p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return e;
+    g_addr[dev] = p;
+  }
+  *ptr = g_addr[dev];
+  return cudaSuccess;
 }
 
 }  // namespace

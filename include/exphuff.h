@@ -214,17 +214,20 @@ EH_API eh_status eh_decompress_chunks(const eh_plan_t *plan, const eh_compressed
                                void *stream);
 
 /* eh_decompress_batch without a workspace, for callers that cannot allocate
- * device memory (code running during CUDA graph capture, runtimes that plan
- * all device memory ahead of time, allocator callbacks).  There is no
- * counterpart on the pages: it is a packaging variant of block decompression.
- * The decoder's scratch lives in a fixed device array inside the library
- * (256 + EH_NOALLOC_MAX_BATCH * 37,888 bytes, held by every GPU that uses the
+ * device memory where they decompress: runtimes that plan all device memory
+ * ahead of time and forbid later allocations, and allocator callbacks that
+ * must not re-enter the allocator.  There is no counterpart on the pages: it
+ * is a packaging variant of block decompression.  The decoder's scratch
+ * lives in a fixed device array inside the library (256 +
+ * EH_NOALLOC_MAX_BATCH * 37,888 bytes, held by every GPU that uses the
  * library until the process exits); nothing is allocated.  k must be in
  * [1, EH_NOALLOC_MAX_BATCH], else EH_ERR_INVALID_ARG.  The first call on a
- * device looks up the array's device address, so make that first call
- * before any stream capture.  The call waits for `stream` and returns the
- * call's status (EH_OK or a data error).  All calls share the array: calls
- * that overlap on the GPU race and must not be issued. */
+ * device looks up the array's device address (a failed lookup is retried by
+ * the next call).  The call waits for `stream` (a device-to-host copy of the
+ * status word and a stream synchronisation) and returns the call's status
+ * (EH_OK or a data error), so it cannot be issued on a stream that is being
+ * captured into a CUDA graph.  All calls share the array: calls that overlap
+ * on the GPU race and must not be issued. */
 EH_API eh_status eh_decompress_batch_noalloc(const eh_plan_t *plan, int k,
                                              const eh_compressed_t *cs,
                                              void *const *outs, void *stream);

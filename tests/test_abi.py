@@ -105,3 +105,24 @@ def test_missing_library_fails_loudly():
     r = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, timeout=120)
     assert r.returncode == 0, (r.stdout, r.stderr)
     assert "not built" in r.stdout
+
+
+def test_python_constants_match_the_header():
+    """The binding's copies of the header's macros (batch limits, index
+    stride, chunk default) are the header's values."""
+    text = open(HEADER).read()
+    macros = dict(re.findall(r"#define\s+(EH_\w+)\s+(\w+)", text))
+    for name in ("EH_NOALLOC_MAX_BATCH", "EH_MAX_BATCH", "EH_INDEX_STRIDE", "EH_PREFETCH_MAX_DEPTH",
+                 "EH_DEFAULT_CHUNK_ELEMS", "EH_MAX_CODE_LEN", "EH_PAGE_RAW"):
+        if hasattr(eh, name):
+            assert int(macros[name].rstrip("u"), 0) == getattr(eh, name), name
+
+
+def test_noalloc_scratch_size_documented(lib):
+    """The no-allocation entry point's fixed array is 256 bytes plus one
+    decompression workspace's tables per tensor: the documented 37,888 bytes
+    per tensor is what eh_decompress_workspace reports per tensor."""
+    p = eh.plan(eh.EH_BF16)
+    per_tensor = eh.decompress_workspace(p, 2) - eh.decompress_workspace(p, 1)
+    assert per_tensor == 37888
+    assert "256 +\n * EH_NOALLOC_MAX_BATCH * 37,888 bytes" in open(HEADER).read()

@@ -30,6 +30,9 @@ def test_reference_arm_line():
     assert d["impl"] == "reference"
     assert d["metric"] == bench.METRIC and d["unit"] == "GB/s" and d["higher_is_better"] is True
     assert d["config"] == bench.workload_config(1)
+    # the per-step sample is named beside the workload it is drawn from
+    assert d["sample_per_step"]["elements"] == 1024 * 4096
+    assert d["sample_per_step"]["of_workload_elements"] == d["config"]["elements"]
     assert d["value"] > 0 and d["cpu_baseline"]["value"] == d["value"]
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] == 1
     assert d["e2e"] == {"value": d["value"], "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
