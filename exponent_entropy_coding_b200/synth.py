@@ -76,6 +76,46 @@ def normal_fp8(n: int, seed: int, std: float = 0.02) -> np.ndarray:
     return to_fp8_e4m3_bits(w)
 
 
+def fibonacci_bf16(m: int, seed: int, first_field: int = 60, chunk: int = 65536) -> np.ndarray:
+    """BF16 values whose exponent fields first_field .. first_field+m-1 occur
+    F(1), F(2), ..., F(m) times (Fibonacci numbers): the histogram that gives
+    a Huffman code its largest depth, m - 1.  Each value is
+    +-(1 + k/128) * 2^(field - 127) with random sign and k.  Placement: the
+    first chunk holds one of the two rarest values, the next 14 rarest and
+    common values; the second chunk holds the other rarest value and values
+    of middle rarity (long codes on average); the rest is shuffled."""
+    rng = np.random.default_rng(seed)
+    fib = [1, 1]
+    while len(fib) < m:
+        fib.append(fib[-1] + fib[-2])
+    fib = fib[:m]
+    pools = [np.full(c, i, dtype=np.int64) for i, c in enumerate(fib)]
+    take = lambda i, k: (pools.__setitem__(i, pools[i][k:]), np.full(k, i, dtype=np.int64))[1]
+    c0 = [take(0, 1)] + [take(i, len(pools[i])) for i in range(2, 16)]
+    n0 = sum(len(a) for a in c0)
+    c0.append(take(m - 1, chunk - n0))
+    c1 = [take(1, 1)]
+    left = chunk - 1
+    for i in range(16, m):
+        k = min(left, len(pools[i]))
+        c1.append(take(i, k))
+        left -= k
+        if left == 0:
+            break
+    head = np.concatenate(c0)
+    head = head[rng.permutation(head.size)]
+    second = np.concatenate(c1)
+    second = second[rng.permutation(second.size)]
+    rest = np.concatenate(pools)
+    rest = rest[rng.permutation(rest.size)]
+    idx = np.concatenate([head, second, rest])
+    field = (idx + first_field).astype(np.float64)
+    mant = rng.integers(0, 128, idx.size)
+    sign = np.where(rng.integers(0, 2, idx.size) == 1, -1.0, 1.0)
+    v = sign * (1.0 + mant / 128.0) * np.exp2(field - 127.0)
+    return to_bf16_bits(v.astype(np.float32))
+
+
 def student_t_f32(shape, rng: np.random.Generator, df: float = 5.0,
                   std: float = 0.02) -> np.ndarray:
     # a t(df) draw has variance df/(df-2); rescale to the requested std

@@ -379,6 +379,108 @@ def test_degenerate_inputs(oracle):
     assert np.array_equal(oracle.decompress(c), odd)
 
 
+def optimal_limited_cost(cnt, lmax):
+    """Minimum of sum(count * length) over prefix codes with lengths <= lmax,
+    computed exactly level by level, independently of package-merge: with the
+    counts sorted in decreasing order the lengths are nondecreasing, so a code
+    is a choice, at each depth d, of how many of the open nodes become leaves
+    (taking the next most frequent symbols); the others become internal and
+    open twice as many nodes at depth d + 1."""
+    w = sorted((int(c) for c in cnt if c), reverse=True)
+    n = len(w)
+    if n <= 1:
+        return sum(w)
+    pre = [0]
+    for v in w:
+        pre.append(pre[-1] + v)
+    best = None
+    cur = {(0, 2): 0}  # (symbols placed, nodes open at depth d) -> cost
+    for d in range(1, lmax + 1):
+        nxt = {}
+        for (j, a), c in cur.items():
+            for k in range(0, min(a, n - j) + 1):
+                cost = c + d * (pre[j + k] - pre[j])
+                if j + k == n:
+                    best = cost if best is None else min(best, cost)
+                    continue
+                na = min(2 * (a - k), n - j - k)
+                if na and cost < nxt.get((j + k, na), cost + 1):
+                    nxt[(j + k, na)] = cost
+        cur = nxt
+    return best
+
+
+@pytest.mark.parametrize("lmax", [3, 4, 5, 7, 9])
+@pytest.mark.parametrize("seed", range(3))
+def test_length_limited_matches_exact_dp(oracle, lmax, seed):
+    rng = np.random.default_rng(300 + seed)
+    m = int(rng.integers(lmax + 1, min(2 ** lmax, 40) + 1))
+    cnt = (rng.pareto(1.0, m) * 20 + 1).astype(np.uint64)
+    lens = oracle.code_lengths(cnt, lmax)
+    assert lens.max() <= lmax and kraft(lens) == 1.0
+    assert int(np.dot(cnt.astype(np.int64), lens.astype(np.int64))) == optimal_limited_cost(cnt, lmax)
+
+
+def _fib(m):
+    f = [1, 1]
+    while len(f) < m:
+        f.append(f[-1] + f[-2])
+    return f[:m]
+
+
+def test_fibonacci_depth_32_at_the_format_limit(oracle):
+    # 33 Fibonacci counts: Huffman depth exactly 32 = the format's longest
+    # code; the limit does not bind, so the cost is the plain Huffman cost
+    cnt = np.zeros(256, np.uint64)
+    cnt[60:93] = _fib(33)
+    assert oracle.huffman_depths(cnt).max() == 32
+    lens = oracle.code_lengths(cnt, 32)
+    assert lens.max() == 32 and int((lens == 32).sum()) == 2
+    assert kraft(lens) == 1.0
+    cost = int(np.dot(cnt.astype(np.int64), lens.astype(np.int64)))
+    assert cost == huffman_cost_heapq(cnt) == optimal_limited_cost(cnt, 32)
+
+
+def test_package_merge_at_limit_32(oracle):
+    # 34 Fibonacci counts: Huffman depth 33 exceeds the format's 32, so the
+    # lengths come from package-merge; they are optimal among codes of at
+    # most 32 bits (exact level DP) and strictly costlier than Huffman
+    cnt = np.zeros(256, np.uint64)
+    cnt[60:94] = _fib(34)
+    assert oracle.huffman_depths(cnt).max() == 33
+    lens = oracle.code_lengths(cnt, 32)
+    assert lens.max() == 32
+    assert kraft(lens) == 1.0
+    cost = int(np.dot(cnt.astype(np.int64), lens.astype(np.int64)))
+    assert cost == optimal_limited_cost(cnt, 32)
+    assert cost > huffman_cost_heapq(cnt)
+
+
+@pytest.mark.parametrize("m", [33, 34])
+def test_32_bit_codes_on_the_stream(oracle, m):
+    # codes of 32 bits inside a chunk staged by the decoder (chunk 0) and in
+    # one larger than its stage (chunk 1): canonical codes prefix-free, every
+    # code readable at its offset, the stream round-trips
+    x = synth.fibonacci_bf16(m, seed=m)
+    c = oracle.compress(0, x)
+    e = (x >> 7) & 0xFF
+    assert c.code_len.max() == 32
+    assert c.code_len[e[:65536]].max() == 32 and c.code_len[e[65536:131072]].max() == 32
+    used = [(int(c.code_len[s]), int(c.code[s])) for s in range(256) if c.code_len[s]]
+    for la, ca in used:
+        for lb, cb in used:
+            if (la, ca) != (lb, cb) and la <= lb:
+                assert (cb >> (lb - la)) != ca  # no code is a prefix of another
+    off = c.chunk_bit_off.astype(np.int64)
+    bits = _bits_of(c.stream, int(c.bits))
+    for i in (0, 1, 65536, 65537):
+        j = i // 65536
+        p0 = off[j] + int(np.sum(c.code_len[e[j * 65536:i]].astype(np.int64)))
+        L = int(c.code_len[e[i]])
+        assert int("".join(map(str, bits[p0:p0 + L])), 2) == int(c.code[e[i]])
+    assert np.array_equal(oracle.decompress(c), x)
+
+
 def test_length_limit_on_stream(oracle):
     # a Fibonacci histogram forces codes longer than 8 under Lmax 32 and the
     # limit under Lmax 9; both round-trip
