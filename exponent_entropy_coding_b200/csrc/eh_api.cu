@@ -13,6 +13,10 @@ namespace {
 
 constexpr int kMaxDevices = 64;
 
+// Fix-up round limit handed to the decoder (0: its default); set only by the
+// test hook eh_debug_set_fixup_rounds.
+std::atomic<uint32_t> g_fixup_rounds{0};
+
 struct DeviceInfo {
   std::once_flag once;
   int num_sms = 0;
@@ -336,6 +340,7 @@ eh_status eh::decompress_impl(const eh_plan_t *plan, int k, const eh_compressed_
   }
   if (chunk0 > 0x7FFFFFFFull) return EH_ERR_INVALID_ARG;
   b.total_chunks = (uint32_t)chunk0;
+  b.fixup_rounds = g_fixup_rounds.load(std::memory_order_relaxed);
   int num_sms = 0;
   if (device_setup(&num_sms) != cudaSuccess) return EH_ERR_CUDA;
   cudaStream_t s = (cudaStream_t)stream;
@@ -475,6 +480,11 @@ eh_status eh_pages_read(const eh_plan_t *plan, const eh_page_store_t *store, con
   cudaStream_t s = (cudaStream_t)stream;
   if (launch_tables(b, s) != cudaSuccess) return EH_ERR_CUDA;
   if (launch_decode(b, s, num_sms) != cudaSuccess) return EH_ERR_CUDA;
+  return EH_OK;
+}
+
+eh_status eh_debug_set_fixup_rounds(uint32_t rounds) {
+  g_fixup_rounds.store(rounds, std::memory_order_relaxed);
   return EH_OK;
 }
 

@@ -396,9 +396,6 @@ __device__ __forceinline__ void named_arrive(uint32_t id, uint32_t n) {
 }
 
 // Barriers of one group: named barrier `id` over kGroupThreads threads.
-__device__ __forceinline__ void gsync(uint32_t id) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "n"(kGroupThreads) : "memory");
-}
 __device__ __forceinline__ bool gsync_or(uint32_t id, bool pred) {
   uint32_t r;
   asm volatile(
@@ -475,7 +472,7 @@ struct RunWriter {
 template <bool kSmem>
 __device__ bool decode_chunk(GroupSmem &G, const DecodeTables &T, const uint32_t *words, uint32_t rel0,
                              uint32_t nbits, uint32_t cnt, uint32_t id, uint32_t gtid, uint32_t *timeout,
-                             uint32_t *r0, uint32_t *r1, bool late) {
+                             uint32_t *r0, uint32_t *r1, bool late, uint32_t max_rounds) {
   const uint32_t lane = gtid & 31u;
   const uint32_t tab = (uint32_t)__cvta_generic_to_shared(&T.l1[0]);
   // window width: a multiple of the gcd of the code lengths, so that a
@@ -604,8 +601,8 @@ __device__ bool decode_chunk(GroupSmem &G, const DecodeTables &T, const uint32_t
     o = group_excl_scan_or(my_n + (bad ? 0x100000u : 0u), changed, G.wsum[round & 1], &total, &any_changed,
                            id, gtid);
     if (!any_changed) break;
-    if (round > kGroupThreads + 1) {  // cannot happen for consistent data
-      if (gtid == 0) *timeout = 1;
+    if (round + 1 >= max_rounds) {  // the round limit: more rounds than threads cannot happen for consistent data
+      if (gtid == 0) *timeout |= 1u;
       total = ~0u;
       break;
     }
@@ -995,6 +992,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
   pdl_wait();  // the decode tables (and everything before them)
   __syncthreads();
   uint32_t parity = 0, timeout = 0, landed = 0;  // landed: stage copies of this group waited for
+  const uint32_t max_rounds = b.fixup_rounds ? b.fixup_rounds : kGroupThreads + 3;
 
   for (uint32_t seg = g0; seg < g1;) {
     const Item &I = b.item[find_item(b, seg)];
@@ -1084,8 +1082,8 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
             r1 = r0;  // nothing of this warp's region is written out
           }
         } else {
-          ok = ci.fits ? decode_chunk<true>(G, S.tabs, G.stage, ci.rel0, ci.nbits, cnt, id, gtid, &timeout, &r0, &r1, late)
-                       : decode_chunk<false>(G, S.tabs, gw, ci.rel0, ci.nbits, cnt, id, gtid, &timeout, &r0, &r1, late);
+          ok = ci.fits ? decode_chunk<true>(G, S.tabs, G.stage, ci.rel0, ci.nbits, cnt, id, gtid, &timeout, &r0, &r1, late, max_rounds)
+                       : decode_chunk<false>(G, S.tabs, gw, ci.rel0, ci.nbits, cnt, id, gtid, &timeout, &r0, &r1, late, max_rounds);
           if (!ok && gtid == 0) set_status(b.status, (timeout & 1u) ? kFlagTimeout | kFlagCorrupt : kFlagCorrupt);
           if (timeout & 2u) set_status(b.status, kFlagCorrupt);
         }

@@ -91,6 +91,7 @@ struct Batch {
   uint32_t max_code_len;
   uint32_t *status;        // workspace status word
   uint32_t *ticket;        // workspace counter for last-block-done patterns
+  uint32_t fixup_rounds;   // decoder: fix-up rounds before giving up (0: the default)
 };
 
 // Item that owns global chunk g (linear scan; k <= 16).

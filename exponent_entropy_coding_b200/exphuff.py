@@ -38,7 +38,7 @@ EXPORTED = ["eh_plan", "eh_compress_bound", "eh_compress_batch_workspace", "eh_c
             "eh_prefetch_acquire", "eh_prefetch_release", "eh_prefetch_status",
             "eh_prefetch_destroy",
             "eh_zf_bound", "eh_zf_compress", "eh_zf_decompress",
-            "eh_get_status", "eh_status_str", "eh_version"]
+            "eh_get_status", "eh_status_str", "eh_version", "eh_debug_set_fixup_rounds"]
 EH_PREFETCH_MAX_DEPTH = 8
 EH_PAGE_RAW = 0x80000000
 
@@ -100,6 +100,7 @@ def lib():
             "eh_decompress_batch": [P(eh_plan_t), C.c_int, P(eh_compressed_t), P(vp), vp, u64, vp],
             "eh_decompress_chunks": [P(eh_plan_t), P(eh_compressed_t), u32, u32, vp, vp, u64, vp],
             "eh_decompress_batch_noalloc": [P(eh_plan_t), C.c_int, P(eh_compressed_t), P(vp), vp],
+            "eh_debug_set_fixup_rounds": [u32],
             "eh_codebook_from_counts": [P(eh_plan_t), vp, vp, vp, vp, u64, vp],
             "eh_pages_append": [P(eh_plan_t), P(eh_page_store_t), vp, u32, vp, vp, u64, vp],
             "eh_pages_read": [P(eh_plan_t), P(eh_page_store_t), vp, u32, vp, vp, u64, vp],
@@ -375,6 +376,11 @@ def decompress_chunks(c: Compressed, first: int, count: int, p: Optional[eh_plan
     return out
 
 
+def debug_set_fixup_rounds(rounds: int) -> None:
+    """Test hook: the decoder's fix-up round limit for later calls (0: default)."""
+    _check(lib().eh_debug_set_fixup_rounds(rounds), "eh_debug_set_fixup_rounds")
+
+
 def get_status(workspace: torch.Tensor, stream=None) -> int:
     return lib().eh_get_status(C.c_void_p(workspace.data_ptr()), _stream_ptr(stream))
 
@@ -383,14 +389,20 @@ def version() -> str:
     return lib().eh_version().decode()
 
 
-def codebook_from_counts(p: eh_plan_t, counts: torch.Tensor, stream=None):
+def codebook_from_counts(p: eh_plan_t, counts: torch.Tensor, stream=None, code_len: Optional[torch.Tensor] = None,
+                         code: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None):
     """(code_len uint8[A], code int32[A]) on the counts' device from
-    exponent counts (int64[A], uint64 values)."""
+    exponent counts (int64[A], uint64 values); the output arrays and the
+    workspace may be passed in."""
     counts = counts.contiguous()
     A = alphabet(p.dtype)
-    code_len = torch.zeros(A, dtype=torch.uint8, device=counts.device)
-    code = torch.zeros(A, dtype=torch.int32, device=counts.device)
-    ws = torch.empty(compress_bound(p, 0)[2], dtype=torch.uint8, device=counts.device)
+    if code_len is None:
+        code_len = torch.zeros(A, dtype=torch.uint8, device=counts.device)
+    if code is None:
+        code = torch.zeros(A, dtype=torch.int32, device=counts.device)
+    ws = workspace
+    if ws is None:
+        ws = torch.empty(compress_bound(p, 0)[2], dtype=torch.uint8, device=counts.device)
     rc = lib().eh_codebook_from_counts(C.byref(p), C.c_void_p(counts.data_ptr()),
                                        C.c_void_p(code_len.data_ptr()), C.c_void_p(code.data_ptr()),
                                        C.c_void_p(ws.data_ptr()), ws.numel(), _stream_ptr(stream))

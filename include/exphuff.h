@@ -392,6 +392,16 @@ EH_API eh_status eh_zf_decompress(const eh_zf_t *c, void *out, void *workspace,
  * recent call that used this workspace. */
 EH_API eh_status eh_get_status(void *workspace, void *stream);
 
+/* Test hook (not for production use).  The decoder finds the thread
+ * boundaries of a chunk in fix-up rounds; a chunk still unresolved after the
+ * round limit is reported as EH_ERR_TIMEOUT | corrupt, which consistent data
+ * never reaches (the default limit exceeds the rounds any chunk can need).
+ * This sets the limit for decompression calls issued afterwards from any
+ * thread (rounds >= 1; 0 restores the default), so that tests can make this
+ * bounded device-side wait give up and check that the error is reported
+ * while the kernel returns normally. */
+EH_API eh_status eh_debug_set_fixup_rounds(uint32_t rounds);
+
 /* Static description of a status code. */
 EH_API const char *eh_status_str(eh_status s);
 

@@ -165,6 +165,28 @@ def test_length_limited(eh, oracle, lmax):
     assert c.code_len.cpu().numpy().max() == lmax
 
 
+@pytest.mark.parametrize("m", [33, 34])
+def test_codes_of_32_bits(eh, oracle, m):
+    # Fibonacci counts over 33 symbols give Huffman codes of up to 32 bits
+    # (the format's limit); over 34 symbols the Huffman depth is 33 and
+    # package-merge limits it to 32.  A 32-bit code sits in a chunk the
+    # decoder stages in shared memory (chunk 0) and in one it reads from
+    # global memory (chunk 1, above 27 KB of stream).
+    x = synth.fibonacci_bf16(m, seed=m)
+    c = roundtrip(eh, oracle, 0, x)
+    lens = c.code_len.cpu().numpy()
+    e = (x >> 7) & 0xFF
+    assert lens.max() == 32
+    assert lens[e[:CHUNK]].max() == 32 and lens[e[CHUNK:2 * CHUNK]].max() == 32
+    off = c.chunk_bit_off.cpu().numpy().view(np.uint64).astype(np.int64)
+    # chunk 0 fits the 26.5 KB shared-memory stage, chunk 1 (about 100 KB) does not
+    assert (off[1] - off[0]) // 8 < 26 * 1024 < 32 * 1024 < (off[2] - off[1]) // 8
+    # chunk ranges that start on each of the two chunks decode too
+    for first, count in ((0, 1), (1, 1), (1, 3)):
+        y = eh.decompress_chunks(c, first, count, eh.plan(0))
+        assert np.array_equal(host_bits(y, 0), x[first * CHUNK:(first + count) * CHUNK])
+
+
 def test_length_limited_real_data(eh, oracle):
     roundtrip(eh, oracle, 0, synth.normal_bf16(3 * 65536, seed=8), lmax=7)
     roundtrip(eh, oracle, 1, synth.normal_fp8(3 * 65536, seed=8), lmax=4)
