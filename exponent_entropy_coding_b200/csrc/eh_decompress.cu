@@ -238,6 +238,31 @@ struct Peek {
   }
 };
 
+// The same 32 bits from two cached words: each call may move at most 32
+// bits past the previous one (one word), and loads one new word when the
+// position enters the next word.  The counting passes move at most 24 bits a
+// lookup pair and at most 32 a code, and they are bound by shared-memory
+// bandwidth: this halves their stream loads.
+template <bool kSmem>
+struct Cursor {
+  Peek<kSmem> src;
+  uint32_t i, a, b;  // a, b: stream words i, i+1
+  __device__ __forceinline__ void seek(uint32_t q) {
+    i = q >> 5;
+    a = src.word(i);
+    b = src.word(i + 1);
+  }
+  __device__ __forceinline__ uint32_t operator()(uint32_t q) {
+    const uint32_t j = q >> 5;
+    if (j != i) {  // j == i + 1
+      a = b;
+      b = src.word(j + 1);
+      i = j;
+    }
+    return __funnelshift_l(b, a, q);
+  }
+};
+
 __device__ __forceinline__ uint32_t lut_index(uint32_t x) { return x >> (32 - kLutBits); }
 
 // A code longer than the first-level index (its prefix has no complete
@@ -293,6 +318,22 @@ constexpr uint32_t kGroupWarps = kGroupThreads / 32;
 constexpr uint32_t kNumGroups = kDecThreads / kGroupThreads;
 constexpr uint32_t kGroupStage = 27136;  // bytes of stream staged per group
 
+// Where one chunk's bits are and whether they fit a shared-memory stage.
+struct ChunkInfo {
+  int item;
+  uint32_t c;       // tensor-local chunk index (page index of the call in page mode)
+  uint32_t cnt;     // values in the chunk
+  uint32_t nbits;   // code bits of the chunk
+  uint32_t rel0;    // first bit of the chunk relative to byte `lo`
+  uint32_t bytes;   // stream bytes staged (multiple of 16)
+  uint64_t lo;      // first staged stream byte (multiple of 16)
+  uint64_t sm_off;  // byte offset of the chunk's sign/mantissa array
+  uint64_t out_off; // index in `out` of the chunk's first value
+  uint32_t raw;     // page mode: raw page index + 1 (0: coded)
+  bool ok;          // offsets consistent with the buffer
+  bool fits;        // bits staged in shared memory
+};
+
 struct GroupSmem {
   alignas(128) uint32_t stage[kGroupStage / 4 + 16];  // bulk-copy target (stream bytes as stored)
   // decoded exponents (output form) of one chunk: value j at byte
@@ -302,8 +343,7 @@ struct GroupSmem {
   uint32_t ends[kGroupThreads];                       // end bit of every thread's codes
   uint32_t wsum[2][kGroupWarps];                      // scan: warp totals, by round parity
   alignas(8) unsigned long long mbar;
-  const uint8_t *next_src[2];                         // stage copy of the group's next chunk,
-  uint32_t next_bytes[2];                             // by chunk parity (0 bytes: none)
+  ChunkInfo next[2];                                  // the group's next chunk, by chunk parity
   uint32_t writers_done;                              // warps done reading the stage
   uint32_t issued;                                    // stage copies started
 };
@@ -479,12 +519,14 @@ __device__ bool decode_chunk(GroupSmem &G, const DecodeTables &T, const uint32_t
   // fixed-length code starts every window on a code boundary
   const uint32_t gq = T.gcd;
   uint32_t W = (nbits + kGroupThreads - 1) / kGroupThreads;
-  W = (W + gq - 1) / gq * gq;
+  if (gq > 1) W = (W + gq - 1) / gq * gq;
   const uint32_t ws = min(gtid * W, nbits), we = min(ws + W, nbits);
   // The thread's frame: frame bit q is chunk bit ws + q - q0.
   const uint32_t q0 = (rel0 + ws) & 31u;
   const uint32_t qe = q0 + (we - ws);
   Peek<kSmem> peek{words + ((rel0 + ws) >> 5)};
+  Cursor<kSmem> cur{peek};
+  cur.seek(q0);
   // Bulk counting runs while 2 * kLutBits bits of the window remain: two
   // first-level lookups per 32-bit peek, no window-end handling.
   constexpr uint32_t kBulk = 2 * kLutBits;
@@ -498,7 +540,7 @@ __device__ bool decode_chunk(GroupSmem &G, const DecodeTables &T, const uint32_t
   for (;;) {
     const uint32_t q = P & 0xFFFFu;
     if (q + kBulk > qe || q >= q0 + kMaskBits) break;
-    const uint32_t x = peek(q);
+    const uint32_t x = cur(q);
     const uint32_t m1 = lds32(tab + 8 * lut_index(x) + 4);
     const uint32_t off = q - q0;
     if (!(m1 & 0xF0000u)) {
@@ -520,7 +562,7 @@ __device__ bool decode_chunk(GroupSmem &G, const DecodeTables &T, const uint32_t
   while (!bad) {
     const uint32_t q = P & 0xFFFFu;
     if (q + kBulk > qe) break;
-    const uint32_t x = peek(q);
+    const uint32_t x = cur(q);
     const uint32_t m1 = lds32(tab + 8 * lut_index(x) + 4);
     if (!(m1 & 0xF0000u)) {
       const uint32_t d = decode_long(T, x);
@@ -536,7 +578,7 @@ __device__ bool decode_chunk(GroupSmem &G, const DecodeTables &T, const uint32_t
     const uint32_t q = P & 0xFFFFu;
     if (q >= qe) break;
     uint32_t nb, bnd;
-    const uint32_t k = count_step(T, peek(q), qe - q, nb, bnd);
+    const uint32_t k = count_step(T, cur(q), qe - q, nb, bnd);
     if (!k) { bad = true; break; }
     const uint32_t off = q - q0;
     if (off < kMaskBits) mask |= (uint64_t)bnd << off;
@@ -564,9 +606,10 @@ __device__ bool decode_chunk(GroupSmem &G, const DecodeTables &T, const uint32_t
       my_start = pred;
       uint32_t q = pred - ws + q0, k = 0;
       bool synced = false, bad2 = false;
+      cur.seek(q);
       while (q < qe) {
         uint32_t nb, bnd;
-        const uint32_t kk = count_step(T, peek(q), qe - q, nb, bnd);
+        const uint32_t kk = count_step(T, cur(q), qe - q, nb, bnd);
         if (!kk) { bad2 = true; break; }
         const uint32_t off = q - q0;
         if (off < kMaskBits) {
@@ -797,22 +840,6 @@ __device__ __forceinline__ uint32_t fp8_merge4(uint32_t nib16, uint32_t e4) {
   return ((t << 4) & 0x80808080u) | (t & 0x07070707u) | (e4 << 3);
 }
 
-// Where one chunk's bits are and whether they fit a shared-memory stage.
-struct ChunkInfo {
-  int item;
-  uint32_t c;       // tensor-local chunk index (page index of the call in page mode)
-  uint32_t cnt;     // values in the chunk
-  uint32_t nbits;   // code bits of the chunk
-  uint32_t rel0;    // first bit of the chunk relative to byte `lo`
-  uint32_t bytes;   // stream bytes staged (multiple of 16)
-  uint64_t lo;      // first staged stream byte (multiple of 16)
-  uint64_t sm_off;  // byte offset of the chunk's sign/mantissa array
-  uint64_t out_off; // index in `out` of the chunk's first value
-  uint32_t raw;     // page mode: raw page index + 1 (0: coded)
-  bool ok;          // offsets consistent with the buffer
-  bool fits;        // bits staged in shared memory
-};
-
 template <int DT>
 __device__ __forceinline__ ChunkInfo chunk_info(const Batch &b, uint32_t g) {
   ChunkInfo ci;
@@ -903,24 +930,45 @@ __device__ __forceinline__ void merge_region(const Item &I, const ChunkInfo &ci,
   if (DT == EH_BF16) {
     const uint8_t *smp = I.sm + ci.sm_off;
     uint16_t *outp = (uint16_t *)I.out + ci.out_off;
-    for (uint32_t b0 = v0 + lane; b0 < v1; b0 += 4 * 32) {
-      uint4 m[4];
-      #pragma unroll
-      for (int u = 0; u < 4; u++) {
-        const uint32_t v = b0 + u * 32;
-        m[u] = v < v1 ? ld_nc16(smp + 16 * (uint64_t)v) : make_uint4(0, 0, 0, 0);
+    if (kRaw) {
+      for (uint32_t v = v0 + lane; v < v1; v += 32) {
+        const uint4 m = ld_nc16(smp + 16 * (uint64_t)v), e = exp_word4(v);
+        const uint2 a = bf16_merge4(m.x, e.x), c = bf16_merge4(m.y, e.y);
+        const uint2 d = bf16_merge4(m.z, e.z), f = bf16_merge4(m.w, e.w);
+        uint4 *dst = (uint4 *)(outp + 16 * (uint64_t)v);
+        dst[0] = make_uint4(a.x, a.y, c.x, c.y);
+        dst[1] = make_uint4(d.x, d.y, f.x, f.y);
       }
-      #pragma unroll
-      for (int u = 0; u < 4; u++) {
-        const uint32_t v = b0 + u * 32;
-        if (v < v1) {
-          const uint4 e = exp_word4(v);
-          const uint2 a = bf16_merge4(m[u].x, e.x), c = bf16_merge4(m[u].y, e.y);
-          const uint2 d = bf16_merge4(m[u].z, e.z), f = bf16_merge4(m[u].w, e.w);
-          uint4 *dst = (uint4 *)(outp + 16 * (uint64_t)v);
-          dst[0] = make_uint4(a.x, a.y, c.x, c.y);
-          dst[1] = make_uint4(d.x, d.y, f.x, f.y);
-        }
+    } else if (v0 + lane < v1) {
+      // lane's vectors v0 + lane + 32k: constant strides for all three
+      // pointers (in the padded exponent rows, 32 vectors are 528 bytes)
+      const uint32_t vl = v0 + lane, K = (v1 - vl + 31) / 32;
+      const uint4 *sp = (const uint4 *)smp + vl;
+      uint4 *op = (uint4 *)outp + 2 * (uint64_t)vl;
+      uint32_t ea = (uint32_t)__cvta_generic_to_shared(exps) + 16 * vl + 4 * (vl >> 3);
+      uint32_t k = 0;
+      for (; k + 1 < K; k += 2, sp += 64, op += 128, ea += 2 * 528) {
+        const uint4 m0 = ld_nc16(sp), m1 = ld_nc16(sp + 32);
+        const uint4 e0 = make_uint4(lds32(ea), lds32(ea + 4), lds32(ea + 8), lds32(ea + 12));
+        const uint4 e1 = make_uint4(lds32(ea + 528), lds32(ea + 532), lds32(ea + 536), lds32(ea + 540));
+        uint2 a = bf16_merge4(m0.x, e0.x), c = bf16_merge4(m0.y, e0.y);
+        uint2 d = bf16_merge4(m0.z, e0.z), f = bf16_merge4(m0.w, e0.w);
+        op[0] = make_uint4(a.x, a.y, c.x, c.y);
+        op[1] = make_uint4(d.x, d.y, f.x, f.y);
+        a = bf16_merge4(m1.x, e1.x);
+        c = bf16_merge4(m1.y, e1.y);
+        d = bf16_merge4(m1.z, e1.z);
+        f = bf16_merge4(m1.w, e1.w);
+        op[64] = make_uint4(a.x, a.y, c.x, c.y);
+        op[65] = make_uint4(d.x, d.y, f.x, f.y);
+      }
+      if (k < K) {
+        const uint4 m0 = ld_nc16(sp);
+        const uint4 e0 = make_uint4(lds32(ea), lds32(ea + 4), lds32(ea + 8), lds32(ea + 12));
+        const uint2 a = bf16_merge4(m0.x, e0.x), c = bf16_merge4(m0.y, e0.y);
+        const uint2 d = bf16_merge4(m0.z, e0.z), f = bf16_merge4(m0.w, e0.w);
+        op[0] = make_uint4(a.x, a.y, c.x, c.y);
+        op[1] = make_uint4(d.x, d.y, f.x, f.y);
       }
     }
     if (r1 == cnt)
@@ -1018,22 +1066,18 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
     const bool stagger = seg_end - seg >= 2;
     if (stagger && grp == 1) named_sync(kStaggerBarrier, kDecThreads);
     for (uint32_t j = 0; g < seg_end; g += kNumGroups, j ^= 1u) {
-      if (g != seg + grp) ci = chunk_info<DT>(b, g);
+      // The group's next chunk is described once, by its first thread, in
+      // the entry of this chunk's parity: every thread reads it at the start
+      // of the next chunk, and the last writer of this chunk starts its stage
+      // copy from it.  (The entry of the other parity may still be read by
+      // the last writer of the previous chunk.)
+      if (g != seg + grp) ci = G.next[j ^ 1u];
       const uint32_t cnt = ci.cnt;
       bool ok = ci.ok && !terr && !S.abort_flag;
-      // The group's next chunk, whose copy the last writer of this one
-      // starts.  Kept by parity: the last writer of the previous chunk may
-      // still be reading the other entry.
       if (gtid == 0) {
         const uint32_t gn = g + kNumGroups;
-        G.next_bytes[j] = 0;
-        if (gn < seg_end) {
-          const ChunkInfo cn = chunk_info<DT>(b, gn);
-          if (cn.fits) {
-            G.next_src[j] = b.item[cn.item].stream + cn.lo;
-            G.next_bytes[j] = cn.bytes;
-          }
-        }
+        if (gn < seg_end) G.next[j] = chunk_info<DT>(b, gn);
+        else G.next[j].fits = false;
       }
 
       // One barrier per chunk before the count: after it the stage holds the
@@ -1100,7 +1144,8 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
         __threadfence_block();
         if (atomicAdd(&G.writers_done, 1u) == kGroupWarps - 1) {
           G.writers_done = 0;
-          if (G.next_bytes[j]) issue_stage(G, G.next_src[j], G.next_bytes[j]);
+          const ChunkInfo &cn = G.next[j];
+          if (cn.fits) issue_stage(G, b.item[cn.item].stream + cn.lo, cn.bytes);
         }
       }
 
