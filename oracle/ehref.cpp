@@ -533,4 +533,75 @@ int ehref_page_decode(int dtype, uint64_t n, const uint8_t *len,
                                  slot_bytes, sm_packed, 0, n ? 1u : 0u, out);
 }
 
+/* ---- stored form (see ehref.h) ---- */
+
+uint32_t ehref_crc32(const uint8_t *data, uint64_t len) {
+  /* bit by bit, lowest bit first, with the reflected polynomial */
+  uint32_t crc = 0xFFFFFFFFu;
+  for (uint64_t i = 0; i < len; i++) {
+    crc ^= data[i];
+    for (int b = 0; b < 8; b++) {
+      if (crc & 1u)
+        crc = (crc >> 1) ^ 0xEDB88320u;
+      else
+        crc >>= 1;
+    }
+  }
+  return ~crc;
+}
+
+static void le_store(uint8_t *p, uint64_t v, int bytes) {
+  for (int i = 0; i < bytes; i++) p[i] = (uint8_t)(v >> (8 * i));
+}
+
+int ehref_container_write(int dtype, uint64_t n, uint32_t chunk, int lmax,
+                          const uint8_t *len, const uint32_t *code,
+                          const uint64_t *chunk_bit_off, const uint8_t *stream,
+                          uint64_t bits, const uint8_t *sm_packed,
+                          const uint32_t *index, uint8_t *out, uint64_t out_cap,
+                          uint64_t *size) {
+  const int A = alphabet_of(dtype);
+  if (!A || chunk == 0 || chunk % 128 != 0 || lmax < 1 || lmax > 32 || !size) return EHREF_EINVAL;
+  const uint64_t C = ehref_num_chunks(n, chunk);
+  /* section contents, in order */
+  uint64_t slen[6];
+  const uint8_t *sptr[6];
+  slen[0] = (uint64_t)A;              sptr[0] = len;
+  slen[1] = 4 * (uint64_t)A;          sptr[1] = (const uint8_t *)code;
+  slen[2] = 8 * (C + 1);              sptr[2] = (const uint8_t *)chunk_bit_off;
+  slen[3] = (bits + 7) / 8;           sptr[3] = stream;
+  slen[4] = ehref_sm_bytes(dtype, n); sptr[4] = sm_packed;
+  slen[5] = index ? 4 * C * (chunk / 128) : 0;
+  sptr[5] = (const uint8_t *)index;
+  /* offsets: from 192, each section at the next multiple of 16 */
+  uint64_t soff[6], pos = 192;
+  for (int i = 0; i < 6; i++) {
+    soff[i] = pos;
+    pos += slen[i];
+    while (pos % 16) pos++;
+  }
+  *size = pos;
+  if (!out) return EHREF_OK;
+  if (out_cap < pos) return EHREF_ECAPACITY;
+  for (uint64_t i = 0; i < pos; i++) out[i] = 0;
+  out[0] = 'E'; out[1] = 'X'; out[2] = 'H'; out[3] = 'F';
+  le_store(out + 4, 1, 2);
+  out[6] = (uint8_t)dtype;
+  out[7] = (uint8_t)lmax;
+  le_store(out + 8, chunk, 4);
+  le_store(out + 12, index ? 1 : 0, 4);
+  le_store(out + 16, n, 8);
+  le_store(out + 24, C, 8);
+  le_store(out + 32, bits, 8);
+  for (int i = 0; i < 6; i++) {
+    for (uint64_t j = 0; j < slen[i]; j++) out[soff[i] + j] = sptr[i][j];
+    uint8_t *entry = out + 40 + 24 * i;
+    le_store(entry, soff[i], 8);
+    le_store(entry + 8, slen[i], 8);
+    le_store(entry + 16, ehref_crc32(out + soff[i], slen[i]), 4);
+  }
+  le_store(out + 184, ehref_crc32(out, 184), 4);
+  return EHREF_OK;
+}
+
 }  // extern "C"

@@ -146,6 +146,32 @@ int ehref_page_decode(int dtype, uint64_t n, const uint8_t *len,
                       const uint8_t *raw_exps, const uint8_t *sm_packed,
                       void *out);
 
+/* Stored form of one compressed tensor (a format of this library; the pages
+ * only say that weights are compressed offline and decompressed on the GPU:
+ * the DFloat11 article, "方法介绍", and ZipFloat §4.2).  Little-endian:
+ *   "EXHF", u16 version 1, u8 dtype, u8 lmax, u32 chunk, u32 flags (bit 0:
+ *   value index present), u64 n, u64 number of chunks C, u64 code bits;
+ *   six section entries {u64 offset, u64 length, u32 crc32, u32 0} for
+ *   lengths (A bytes), codes (A u32), chunk bit offsets (C+1 u64), stream
+ *   (ceil(bits/8) bytes), sign/mantissa bytes, value index (C*chunk/128 u32
+ *   or length 0); the crc32 of the preceding 184 bytes and a zero u32;
+ *   then the sections in that order from byte 192, each starting at a
+ *   multiple of 16, zeros between them and after the last up to a multiple
+ *   of 16.
+ * crc32 is the IEEE 802.3 / zlib CRC (reflected polynomial 0xEDB88320,
+ * initial and final XOR 0xFFFFFFFF).  index may be NULL.  Writes the
+ * container to out (out_cap bytes) and its size to *size; with out == NULL
+ * only the size is returned. */
+int ehref_container_write(int dtype, uint64_t n, uint32_t chunk, int lmax,
+                          const uint8_t *len, const uint32_t *code,
+                          const uint64_t *chunk_bit_off, const uint8_t *stream,
+                          uint64_t bits, const uint8_t *sm_packed,
+                          const uint32_t *index, uint8_t *out, uint64_t out_cap,
+                          uint64_t *size);
+
+/* The crc32 of the container format, for tests. */
+uint32_t ehref_crc32(const uint8_t *data, uint64_t len);
+
 #ifdef __cplusplus
 }
 #endif

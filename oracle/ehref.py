@@ -53,6 +53,8 @@ def lib():
             "ehref_page_encode": (i32, [i32, vp, u64, vp, vp, vp, u64, vp, vp, vp, vp]),
             "ehref_page_decode": (i32, [i32, u64, vp, vp, vp, u64, u64, i32, vp, vp, vp]),
             "ehref_value_index": (i32, [i32, vp, u64, u32, vp, vp]),
+            "ehref_container_write": (i32, [i32, u64, u32, i32, vp, vp, vp, vp, u64, vp, vp, vp, u64, vp]),
+            "ehref_crc32": (u32, [vp, u64]),
             "zfref_blocks": (u64, [u64]),
             "zfref_block_base": (i32, [vp, u32, vp, vp]),
             "zfref_compress": (i32, [vp, u64, vp, vp, vp, vp, vp, u64, vp]),
@@ -209,6 +211,25 @@ def compress(dtype, x, chunk=65536, lmax=32):
     return Compressed(dtype, n, chunk, lmax, ln, code, off,
                       stream[: (bits.value + 7) // 8].copy(),
                       sm[: sm_bytes(dtype, n)].copy(), bits.value)
+
+
+def container(c: Compressed, index=None) -> bytes:
+    """The stored form (ehref.h) of a compressed tensor; `index` is its
+    optional value index (uint32 array)."""
+    args = [c.dtype, c.n, c.chunk, c.lmax, _p(np.ascontiguousarray(c.code_len, np.uint8)),
+            _p(np.ascontiguousarray(c.code, np.uint32)), _p(np.ascontiguousarray(c.chunk_bit_off, np.uint64)),
+            _p(np.ascontiguousarray(c.stream, np.uint8)), c.bits, _p(np.ascontiguousarray(c.sign_mant, np.uint8)),
+            _p(np.ascontiguousarray(index, np.uint32)) if index is not None else None]
+    size = C.c_uint64(0)
+    _check(lib().ehref_container_write(*args, None, 0, C.byref(size)))
+    out = np.zeros(size.value, np.uint8)
+    _check(lib().ehref_container_write(*args, _p(out), out.size, C.byref(size)))
+    return out.tobytes()
+
+
+def crc32(data: bytes) -> int:
+    a = np.frombuffer(data, np.uint8)
+    return int(lib().ehref_crc32(_p(np.ascontiguousarray(a)), a.size))
 
 
 def decompress(c: Compressed, first=None, count=None):

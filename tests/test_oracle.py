@@ -628,3 +628,48 @@ def test_page_missing_symbol_is_raw(oracle):
     pg = oracle.page_encode(0, page, book.code_len, book.code, 64 * 1024)
     assert pg.raw
     assert np.array_equal(oracle.page_decode(0, 65536, book.code_len, book.code, pg), page)
+
+
+# ------------------------------------------------------------ stored form
+
+def test_crc32_is_the_zlib_crc(oracle):
+    import zlib
+    assert oracle.crc32(b"123456789") == 0xCBF43926  # the standard check value
+    rng = np.random.default_rng(5)
+    for n in (0, 1, 7, 1000, 65537):
+        data = rng.integers(0, 256, n, dtype=np.uint8).tobytes()
+        assert oracle.crc32(data) == zlib.crc32(data)
+
+
+@pytest.mark.parametrize("dtype,n,chunk,with_index", [(0, 3 * 65536 + 123, 65536, False), (1, 70001, 1024, True),
+                                                       (2, 4097, 1024, False), (0, 0, 65536, False)])
+def test_container_layout(oracle, dtype, n, chunk, with_index):
+    """The oracle's container, parsed field by field with the layout written
+    out independently here, holds the compressed arrays and their CRCs."""
+    import struct
+    import zlib
+    if dtype == 0:
+        x = synth.normal_bf16(n, seed=3)
+    elif dtype == 1:
+        x = synth.normal_fp8(n, seed=3)
+    else:
+        x = np.random.default_rng(3).integers(0, 256, n).astype(np.uint8)
+    c = oracle.compress(dtype, x, chunk=chunk)
+    idx = oracle.value_index(dtype, x, c.code_len, chunk=chunk) if with_index else None
+    buf = oracle.container(c, idx)
+    assert buf[:4] == b"EXHF"
+    version, dt, lmax, ch, flags, n_, C, bits = struct.unpack_from("<HBBIIQQQ", buf, 4)
+    assert (version, dt, lmax, ch, flags, n_, bits) == (1, dtype, 32, chunk, int(with_index), n, c.bits)
+    assert C == -(-n // chunk)
+    parts = [c.code_len.tobytes(), c.code.astype("<u4").tobytes(), c.chunk_bit_off.astype("<u8").tobytes(),
+             c.stream.tobytes(), c.sign_mant.tobytes(), idx.astype("<u4").tobytes() if with_index else b""]
+    pos = 192
+    for i, part in enumerate(parts):
+        off, ln, crc, zero = struct.unpack_from("<QQII", buf, 40 + 24 * i)
+        assert (off, ln, zero) == (pos, len(part), 0)
+        assert buf[off:off + ln] == part and crc == zlib.crc32(part)
+        end = -(-(off + ln) // 16) * 16
+        assert buf[off + ln:end] == bytes(end - off - ln)  # zero padding
+        pos = end
+    assert len(buf) == pos
+    assert struct.unpack_from("<II", buf, 184) == (zlib.crc32(buf[:184]), 0)
