@@ -38,7 +38,8 @@ EXPORTED = ["eh_plan", "eh_compress_bound", "eh_compress_batch_workspace", "eh_c
             "eh_prefetch_acquire", "eh_prefetch_release", "eh_prefetch_status",
             "eh_prefetch_destroy",
             "eh_zf_bound", "eh_zf_compress", "eh_zf_decompress",
-            "eh_get_status", "eh_status_str", "eh_version", "eh_debug_set_fixup_rounds"]
+            "eh_get_status", "eh_status_str", "eh_version", "eh_debug_set_fixup_rounds",
+            "eh_container_size", "eh_container_write", "eh_container_read"]
 EH_PREFETCH_MAX_DEPTH = 8
 EH_PAGE_RAW = 0x80000000
 
@@ -101,6 +102,9 @@ def lib():
             "eh_decompress_chunks": [P(eh_plan_t), P(eh_compressed_t), u32, u32, vp, vp, u64, vp],
             "eh_decompress_batch_noalloc": [P(eh_plan_t), C.c_int, P(eh_compressed_t), P(vp), vp],
             "eh_debug_set_fixup_rounds": [u32],
+            "eh_container_size": [P(eh_plan_t), u64, u64, C.c_int, P(u64)],
+            "eh_container_write": [P(eh_plan_t), P(eh_compressed_t), vp, u64],
+            "eh_container_read": [vp, u64, P(eh_plan_t), P(eh_compressed_t)],
             "eh_codebook_from_counts": [P(eh_plan_t), vp, vp, vp, vp, u64, vp],
             "eh_pages_append": [P(eh_plan_t), P(eh_page_store_t), vp, u32, vp, vp, u64, vp],
             "eh_pages_read": [P(eh_plan_t), P(eh_page_store_t), vp, u32, vp, vp, u64, vp],
@@ -374,6 +378,65 @@ def decompress_chunks(c: Compressed, first: int, count: int, p: Optional[eh_plan
     if check:
         _check(get_status(workspace, stream), "eh_decompress_chunks (device status)")
     return out
+
+
+def container_size(p: eh_plan_t, n: int, exp_stream_bits: int, with_index: bool = False) -> int:
+    out = C.c_uint64()
+    _check(lib().eh_container_size(C.byref(p), n, exp_stream_bits, int(with_index), C.byref(out)),
+           "eh_container_size")
+    return out.value
+
+
+def to_container(c: Compressed, p: eh_plan_t) -> bytes:
+    """The stored form of a compressed tensor: its device arrays copied to the
+    host and written by eh_container_write."""
+    import numpy as np
+    host = {k: getattr(c, k).cpu().numpy() for k in ("code_len", "code", "chunk_bit_off", "exp_stream", "sign_mant")}
+    vi = c.value_index.cpu().numpy() if c.value_index is not None else None
+    s = eh_compressed_t()
+    s.dtype, s.n, s.n_chunks, s.exp_stream_bits = c.dtype, c.n, c.n_chunks, c.exp_stream_bits
+    ptr = lambda a: a.ctypes.data_as(C.c_void_p) if a is not None and a.size else None
+    s.code_len, s.code, s.chunk_bit_off = ptr(host["code_len"]), ptr(host["code"]), ptr(host["chunk_bit_off"])
+    s.exp_stream, s.exp_stream_cap = ptr(host["exp_stream"]), host["exp_stream"].size
+    s.sign_mant = ptr(host["sign_mant"])
+    s.value_index = ptr(vi)
+    size = container_size(p, c.n, c.exp_stream_bits, vi is not None)
+    out = np.zeros(size, np.uint8)
+    _check(lib().eh_container_write(C.byref(p), C.byref(s), out.ctypes.data_as(C.c_void_p), size),
+           "eh_container_write")
+    return out.tobytes()
+
+
+def from_container(buf: bytes, device):
+    """(Compressed on `device`, plan) from a stored container; raises EhError
+    (EH_ERR_CORRUPT) if it fails its checks."""
+    import numpy as np
+    src = np.frombuffer(buf, np.uint8)
+    p, v = eh_plan_t(), eh_compressed_t()
+    _check(lib().eh_container_read(src.ctypes.data_as(C.c_void_p), src.size, C.byref(p), C.byref(v)),
+           "eh_container_read")
+    base = src.ctypes.data
+
+    def arr(ptr, count, dtype):
+        if not ptr or not count:
+            return np.zeros(0, dtype)
+        return src[ptr - base: ptr - base + count * np.dtype(dtype).itemsize].view(dtype)
+
+    A = alphabet(p.dtype)
+    nc = v.n_chunks
+    c = alloc_compressed(p, v.n, device, index=bool(v.value_index))
+    c.code_len.copy_(torch.from_numpy(arr(v.code_len, A, np.uint8).copy()))
+    c.code.copy_(torch.from_numpy(arr(v.code, A, np.int32).copy()))
+    c.chunk_bit_off.copy_(torch.from_numpy(arr(v.chunk_bit_off, nc + 1, np.int64).copy()))
+    nb = v.exp_stream_cap
+    if nb:
+        c.exp_stream[:nb].copy_(torch.from_numpy(arr(v.exp_stream, nb, np.uint8).copy()))
+    if c.sign_mant.numel():
+        c.sign_mant.copy_(torch.from_numpy(arr(v.sign_mant, c.sign_mant.numel(), np.uint8).copy()))
+    if c.value_index is not None:
+        c.value_index.copy_(torch.from_numpy(arr(v.value_index, c.value_index.numel(), np.int32).copy()))
+    c.exp_stream_bits = v.exp_stream_bits
+    return c, p
 
 
 def debug_set_fixup_rounds(rounds: int) -> None:

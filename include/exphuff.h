@@ -392,6 +392,41 @@ EH_API eh_status eh_zf_decompress(const eh_zf_t *c, void *out, void *workspace,
  * recent call that used this workspace. */
 EH_API eh_status eh_get_status(void *workspace, void *stream);
 
+/* ---- Stored form of one compressed tensor.  Weights are compressed once,
+ * offline, and decompressed on the GPU when used (the DFloat11 article,
+ * "方法介绍"; ZipFloat §4.2): these calls turn a compressed tensor into one
+ * self-describing byte container and back.  Layout (little-endian): the
+ * magic "EXHF", u16 version 1, u8 dtype, u8 max_code_len, u32 chunk_elems,
+ * u32 flags (bit 0: value index present), u64 n, u64 n_chunks, u64
+ * exp_stream_bits; six section entries {u64 offset, u64 length, u32 CRC-32,
+ * u32 0} for code_len (A bytes), code (A u32), chunk_bit_off (n_chunks+1
+ * u64), exp_stream (ceil(bits/8) bytes), sign_mant and value_index (length 0
+ * when absent); the CRC-32 of the 184 bytes before it; then the sections at
+ * 16-byte aligned offsets from byte 192, zero-padded, the total a multiple of
+ * 16.  CRC-32 is the IEEE 802.3 / zlib one.  All pointers are HOST pointers:
+ * the caller copies the device arrays to the host before writing and back to
+ * device buffers (eh_compress_bound sizes, for the decoder's read-ahead)
+ * after reading. */
+
+/* Size in bytes of the container of an n-element tensor with that many code
+ * bits (with_index != 0: with a value index). */
+EH_API eh_status eh_container_size(const eh_plan_t *plan, uint64_t n, uint64_t exp_stream_bits,
+                                   int with_index, uint64_t *bytes);
+
+/* Writes the container of the tensor `c` (its dtype, n, n_chunks,
+ * exp_stream_bits and HOST arrays; value_index may be NULL) to dst, which
+ * must hold eh_container_size() bytes (else EH_ERR_NOMEM). */
+EH_API eh_status eh_container_write(const eh_plan_t *plan, const eh_compressed_t *c, void *dst,
+                                    uint64_t dst_bytes);
+
+/* Checks a container (magic, version, plan, sizes, section layout, every
+ * CRC-32; EH_ERR_CORRUPT on any mismatch) and fills *plan and *view, whose
+ * array pointers point into src (exp_stream_cap = the stream's byte
+ * length).  Padding and reserved bytes must be zero, so that a change to any
+ * byte of a container is detected. */
+EH_API eh_status eh_container_read(const void *src, uint64_t src_bytes, eh_plan_t *plan,
+                                   eh_compressed_t *view);
+
 /* Test hook (not for production use).  The decoder finds the thread
  * boundaries of a chunk in fix-up rounds; a chunk still unresolved after the
  * round limit is reported as EH_ERR_TIMEOUT | corrupt, which consistent data
