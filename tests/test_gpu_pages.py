@@ -50,17 +50,17 @@ def _setup(eh, oracle, n_prefill=8, n_new=24, smooth=True):
     return p, book, prefill, new
 
 
-def _check_against_oracle(eh, oracle, store, book, new, slot_ids):
+def _check_against_oracle(eh, oracle, store, book, new, slot_ids, dtype=0):
     lens = book.code_len.cpu().numpy()
     codes = book.code.cpu().numpy().view(np.uint32)
     meta = store.page_meta.cpu().numpy().view(np.uint32)
     slots = store.slots.cpu().numpy().reshape(store.n_slots, store.slot_bytes)
-    sm = store.sign_mant.cpu().numpy().reshape(store.n_slots, PAGE)
+    sm = store.sign_mant.cpu().numpy().reshape(store.n_slots, PAGE if dtype == 0 else PAGE // 2)
     pool = store.raw_pool.cpu().numpy()
     n_raw = 0
     for i, s in enumerate(slot_ids):
         page = new[i * PAGE:(i + 1) * PAGE]
-        ref = oracle.page_encode(0, page, lens, codes, store.slot_bytes)
+        ref = oracle.page_encode(dtype, page, lens, codes, store.slot_bytes)
         assert np.array_equal(sm[s], ref.sign_mant)
         if ref.raw:
             n_raw += 1
@@ -113,3 +113,42 @@ def test_raw_pool_exhaustion_is_reported(eh, oracle):
     assert store.status() == eh.EH_ERR_NOMEM
     y = store.read(torch.arange(6, dtype=torch.int32), check=False)
     assert store.status() == eh.EH_ERR_CORRUPT
+
+
+def _fp8_cache(n_pages, seed):
+    """FP8 E4M3 K/V-like values: normal with standard deviation 20, so that no
+    value reaches 256 (exponent field 15) while subnormals occur."""
+    w = np.random.default_rng(seed).standard_normal(n_pages * PAGE).astype(np.float32) * np.float32(20.0)
+    return synth.to_fp8_e4m3_bits(w)
+
+
+@pytest.mark.parametrize("smooth", [True, False])
+def test_fp8_pages_append_and_read(eh, oracle, smooth):
+    """The page store with FP8 E4M3 pages (16-symbol exponent alphabet,
+    sign/mantissa nibbles packed two per byte)."""
+    prefill, new = _fp8_cache(6, 11), _fp8_cache(20, 12)
+    assert not ((prefill >> 3) & 0xF == 15).any()
+    p = eh.plan(eh.EH_FP8_E4M3)
+    if smooth:
+        cnt = oracle.histogram(1, prefill) + np.uint64(1)
+        code_len, code = eh.codebook_from_counts(p, torch.from_numpy(cnt.view(np.int64)).cuda())
+        assert np.array_equal(code_len.cpu().numpy(), oracle.code_lengths(cnt, 32))
+        book = _Book(code_len, code)
+    else:
+        new[7 * PAGE + 4321] = 0x78                     # 256.0: exponent 15, absent from the prefill
+        book = eh.compress(torch.from_numpy(prefill).cuda(), p)
+    n_new = new.size // PAGE
+    # pages code to 21.15 - 21.30 KB (2.6 bits per exponent): with 21,248-byte
+    # slots some fit and some go to the raw pool
+    store = eh.PageStore(p, book.code_len, book.code, n_slots=32, slot_bytes=21248, raw_cap=n_new,
+                         device="cuda")
+    rng = np.random.default_rng(1)
+    slot_ids = rng.permutation(32)[:n_new]
+    store.append(torch.from_numpy(new).cuda(), torch.from_numpy(slot_ids))
+    assert store.status() == eh.EH_OK
+    n_raw = _check_against_oracle(eh, oracle, store, book, new, slot_ids, dtype=1)
+    assert 0 < n_raw < n_new
+    order = rng.permutation(n_new)
+    y = store.read(torch.from_numpy(slot_ids[order]))
+    want = np.concatenate([new[i * PAGE:(i + 1) * PAGE] for i in order])
+    assert np.array_equal(y.cpu().numpy(), want)
