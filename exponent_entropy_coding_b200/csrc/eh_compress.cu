@@ -491,14 +491,8 @@ __device__ __forceinline__ uint32_t block_excl_scan1(uint32_t v, uint32_t *wsum,
   __syncthreads();
   // lane i < kWarps holds warp i's total; prefix over lanes below `warp`
   const uint32_t t = lane < kWarps ? wsum[lane] : 0u;
-  const uint32_t before = lane < warp ? t : 0u;
-  uint32_t pre = before, all = t;
-  #pragma unroll
-  for (int o = 16; o; o >>= 1) {
-    pre += __shfl_xor_sync(0xffffffffu, pre, o);
-    all += __shfl_xor_sync(0xffffffffu, all, o);
-  }
-  *total = all;
+  *total = __reduce_add_sync(0xffffffffu, t);  // one warp reduction each
+  const uint32_t pre = __reduce_add_sync(0xffffffffu, lane < warp ? t : 0u);
   return pre + x - v;
 }
 
