@@ -463,13 +463,8 @@ __device__ __forceinline__ uint32_t group_excl_scan_or(uint32_t v, bool pred, ui
   if (lane == 31) wsum[warp] = x;
   *any = gsync_or(id, pred);
   const uint32_t t = lane < kGroupWarps ? wsum[lane] : 0u;
-  uint32_t pre = lane < warp ? t : 0u, all = t;
-  #pragma unroll
-  for (int o = 16; o; o >>= 1) {
-    pre += __shfl_xor_sync(0xffffffffu, pre, o);
-    all += __shfl_xor_sync(0xffffffffu, all, o);
-  }
-  *total = all;
+  *total = __reduce_add_sync(0xffffffffu, t);  // one warp reduction each
+  const uint32_t pre = __reduce_add_sync(0xffffffffu, lane < warp ? t : 0u);
   return pre + x - v;
 }
 
@@ -1045,14 +1040,8 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
   for (uint32_t seg = g0; seg < g1;) {
     const Item &I = b.item[find_item(b, seg)];
     const uint32_t seg_end = min(g1, I.chunk0 + I.nchunks);
-    __syncthreads();  // both groups are done with the previous tables
-    {
-      const uint4 *src = (const uint4 *)I.lut;
-      uint4 *dst = (uint4 *)&S.tabs;
-      for (uint32_t i = tid; i < sizeof(DecodeTables) / 16; i += kDecThreads) dst[i] = src[i];
-    }
-    __syncthreads();
-    const bool terr = S.tabs.err != 0;
+    __syncthreads();  // both groups are done with the previous tables and stages
+    // the first chunk's stage copy runs while the tables are copied
     uint32_t g = seg + grp;
     ChunkInfo ci;
     ci.fits = false;
@@ -1060,10 +1049,19 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
       ci = chunk_info<DT>(b, g);
       if (ci.fits && gtid == 0) issue_stage(G, b.item[ci.item].stream + ci.lo, ci.bytes);
     }
+    {
+      const uint4 *src = (const uint4 *)I.lut;
+      uint4 *dst = (uint4 *)&S.tabs;
+      for (uint32_t i = tid; i < sizeof(DecodeTables) / 16; i += kDecThreads) dst[i] = src[i];
+    }
+    __syncthreads();
+    const bool terr = S.tabs.err != 0;
     // Stagger the groups by one decode: group 1 starts its first chunk when
     // group 0 has decoded its own and turns to the memory-bound output, so
     // one group's output overlaps the other's decode instead of coinciding.
-    const bool stagger = seg_end - seg >= 2;
+    // With only two chunks there is nothing to overlap afterwards, and both
+    // groups start at once.
+    const bool stagger = seg_end - seg >= 3;
     if (stagger && grp == 1) named_sync(kStaggerBarrier, kDecThreads);
     for (uint32_t j = 0; g < seg_end; g += kNumGroups, j ^= 1u) {
       // The group's next chunk is described once, by its first thread, in
@@ -1080,12 +1078,12 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
         else G.next[j].fits = false;
       }
 
-      // One barrier per chunk before the count: after it the stage holds the
-      // chunk's stream words in MSB-first order.
       // Every thread waits for the chunk's stage copy itself.  The plain
       // decode's first barrier tells the group whether a copy came late;
       // every other path takes one barrier here, so that the warps of a
-      // group never drift more than a chunk apart.
+      // group never drift more than a chunk apart, and a chunk read from
+      // global memory (no copy to wait for) cannot overwrite the end bits
+      // that a slow warp of the previous chunk still reads.
       const uint32_t *vidx = (ok && I.vindex && !I.page_meta) ? I.vindex + (uint64_t)ci.c * (b.chunk_elems / kIndexStride)
                                                             : nullptr;
       bool late = false;
@@ -1096,7 +1094,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
           landed++;
         }
       }
-      if (!ok || ci.raw || vidx) {
+      if (!ok || ci.raw || vidx || !ci.fits) {
         if (gsync_or(id, late)) {
           if (gtid == 0) {
             set_status(b.status, kFlagTimeout);

@@ -215,6 +215,34 @@ def test_chunk_larger_than_stage(eh, oracle):
     assert (off[2] - off[1]) // 8 > 32 * 1024
 
 
+@pytest.mark.parametrize("dtype", [0, 1])
+def test_runs_of_every_length_are_exact(eh, oracle, dtype):
+    # A batch whose tensors split the decoding CTAs' chunk ranges into runs
+    # of one to eight chunks (1024-value chunks): runs of one chunk leave a
+    # group idle, runs of two start both groups at once, longer runs stagger
+    # them, and a range may change tensors (and tables) in its middle.
+    # Decoded many times, every decode must be exact.
+    p = eh.plan(dtype, 1024)
+    sizes = [148 * 3 * 1024 + 5, 7 * 1024, 149 * 1024 - 1, 1024, 3 * 148 * 1024 + 2 * 1024 + 17]
+    xs = [synth.normal_bf16(n, seed=11 + i) if dtype == 0 else synth.normal_fp8(n, seed=11 + i)
+          for i, n in enumerate(sizes)]
+    ts = [dev(x) for x in xs]
+    outs = [eh.alloc_compressed(p, t.numel(), "cuda") for t in ts]
+    ws = torch.empty(eh.compress_batch_workspace(p, sizes), dtype=torch.uint8, device="cuda")
+    eh.compress_batch(p, ts, outs, ws)
+    for x, c in zip(xs, outs):
+        assert_same(c, oracle.compress(dtype, x, chunk=1024))
+    ys = [torch.empty_like(t) for t in ts]
+    wsd = torch.empty(eh.decompress_workspace(p, len(ts)), dtype=torch.uint8, device="cuda")
+    for _ in range(10):
+        for y in ys:
+            y.fill_(0x55)
+        eh.decompress_batch(p, outs, ys, wsd)
+        assert eh.get_status(wsd) == eh.EH_OK
+        for t, y in zip(ts, ys):
+            assert torch.equal(t, y)
+
+
 def test_batch_block(eh, oracle):
     _, items = synth.workload("llama8b_block", scale=64)
     p = eh.plan(0)
