@@ -65,73 +65,103 @@ def hbm_peak():
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons during the timed region.  The
+    """SM clocks and throttle reasons during the timed region, polled through
+    NVML about every millisecond (so that a region of a few milliseconds
+    still gets several samples), else through `nvidia-smi -lms 20`.  The
     sampler is started first and the timed region begins once its first
-    sample has arrived, so that short regions are still sampled."""
+    sample has arrived."""
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
 
     def __init__(self, gpu_index):
         self.gpu = gpu_index
         self.proc = None
-        self.lines = []
+        self.samples = []  # (sm MHz, max sm MHz, set of reasons)
         self.mark = 0
+        self.source = None
+        self.stop = False
 
-    def _read(self):
+    def _nvml_handle(self):
+        import pynvml
+        import torch
+        pynvml.nvmlInit()
+        uuid = getattr(torch.cuda.get_device_properties(self.gpu), "uuid", None)
+        if uuid is not None:
+            u = str(uuid)
+            return pynvml, pynvml.nvmlDeviceGetHandleByUUID(u if u.startswith("GPU-") else "GPU-" + u)
+        return pynvml, pynvml.nvmlDeviceGetHandleByIndex(self.gpu)
+
+    def _poll_nvml(self, nv, h):
+        bits = {"hw_slowdown": nv.nvmlClocksEventReasonHwSlowdown,
+                "hw_thermal_slowdown": nv.nvmlClocksEventReasonHwThermalSlowdown,
+                "sw_thermal_slowdown": nv.nvmlClocksEventReasonSwThermalSlowdown,
+                "sw_power_cap": nv.nvmlClocksEventReasonSwPowerCap}
+        mx = float(nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM))
+        while not self.stop:
+            try:
+                sm = float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM))
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+            except Exception:
+                break
+            self.samples.append((sm, mx, {k for k, v in bits.items() if r & v}))
+            time.sleep(0.001)
+
+    def _read_smi(self):
         for line in self.proc.stdout:
-            if line.strip():
-                self.lines.append(line)
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm, mx = float(f[1]), float(f[2])
+            except ValueError:
+                continue
+            self.samples.append((sm, mx, {n for n, v in zip(self.REASONS, f[5:9]) if v.lower() == "active"}))
 
     def __enter__(self):
         import threading
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "20"],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-        except (OSError, ValueError):
-            self.proc = None
-            return self
-        self.thread = threading.Thread(target=self._read, daemon=True)
+            nv, h = self._nvml_handle()
+            self.thread = threading.Thread(target=self._poll_nvml, args=(nv, h), daemon=True)
+            self.source = "nvml, ~1 ms"
+        except Exception:
+            try:
+                self.proc = subprocess.Popen(
+                    ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                     "--format=csv,noheader,nounits", "-lms", "20"],
+                    stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            except (OSError, ValueError):
+                return self
+            self.thread = threading.Thread(target=self._read_smi, daemon=True)
+            self.source = "nvidia-smi, 20 ms"
         self.thread.start()
         t0 = time.time()
-        while not self.lines and time.time() - t0 < 10 and self.proc.poll() is None:
-            time.sleep(0.01)
-        self.mark = len(self.lines)  # samples from here on fall in the timed region
+        while not self.samples and time.time() - t0 < 10 and self.thread.is_alive():
+            time.sleep(0.001)
+        self.mark = len(self.samples)  # samples from here on fall in the timed region
         return self
 
     def __exit__(self, *exc):
+        self.stop = True
         if self.proc is not None:
             self.proc.terminate()
             try:
                 self.proc.wait(timeout=5)
             except subprocess.TimeoutExpired:
                 self.proc.kill()
+        if self.source:
             self.thread.join(timeout=5)
-        # the sample taken just before the region ended is kept; earlier ones
-        # (before the region started) are not
-        self.lines = self.lines[max(self.mark - 1, 0):]
+        # the sample taken just before the region started is kept as its first
+        self.samples = self.samples[max(self.mark - 1, 0):]
 
     def summary(self):
-        sm, mx, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for l in self.lines:
-            f = [x.strip() for x in l.split(",")]
-            if len(f) < 9:
-                continue
-            try:
-                sm.append(float(f[1]))
-                mx.append(float(f[2]))
-            except ValueError:
-                continue
-            for name, v in zip(names, f[5:9]):
-                if v.lower() == "active":
-                    reasons.add(name)
-        if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
-                "samples": len(sm)}
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0, "source": self.source}
+        reasons = set().union(*(r for _, _, r in self.samples))
+        return {"sm_mhz": statistics.median(s for s, _, _ in self.samples),
+                "sm_max_mhz": max(m for _, m, _ in self.samples), "reasons": sorted(reasons),
+                "samples": len(self.samples), "source": self.source}
 
 
 def workload_config(world, elements=218103808, chunk_elems=65536, max_code_len=32):
@@ -346,9 +376,32 @@ def run_all_configs(reps=20):
     return 0
 
 
+def graph_rate(fn, stream, reps, nbytes):
+    """Bytes per second of one call of `fn`, from `reps` calls captured in a
+    CUDA graph and replayed between CUDA events (device time only: calls that
+    only enqueue small amounts of work would otherwise be timed at the pace of
+    the host's Python loop)."""
+    import torch
+
+    def loop():
+        for _ in range(reps):
+            fn()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):  # captured on a side stream
+        loop()
+    g.replay()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    ev[0].record(stream)
+    g.replay()
+    ev[1].record(stream)
+    torch.cuda.synchronize()
+    return nbytes / (ev[0].elapsed_time(ev[1]) / reps * 1e-3) / 1e9
+
+
 def measure_fp4_scales(eh, synth, items, dev, stream, reps=50):
     """Compress + decompress of the seven matrices' E4M3 block scales (byte
-    alphabet) with CUDA events; returns GB/s of scale bytes and the ratio."""
+    alphabet), each timed as `reps` calls in a CUDA graph replay; returns GB/s
+    of scale bytes and the ratio."""
     import torch
     scales = [synth.nvfp4_block_scales(synth.bf16_bits_to_f32(x)) for _, x in items]
     xs = [torch.from_numpy(s).to(dev) for s in scales]
@@ -363,19 +416,11 @@ def measure_fp4_scales(eh, synth, items, dev, stream, reps=50):
     assert eh.get_status(wsd) == eh.EH_OK and all(torch.equal(x, y) for x, y in zip(xs, ys))
     nbytes = sum(x.numel() for x in xs)
     comp = sum(o.compressed_bytes() for o in outs)
-    ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
-    ev[0].record(stream)
-    for _ in range(reps):
-        eh.compress_batch(p, xs, outs, wsc, bits_dev=bits)
-    ev[1].record(stream)
-    for _ in range(reps):
-        eh.decompress_batch(p, outs, ys, wsd)
-    ev[2].record(stream)
-    torch.cuda.synchronize()
-    enc = ev[0].elapsed_time(ev[1]) / reps
-    dec = ev[1].elapsed_time(ev[2]) / reps
-    return {"kind": "E4M3 block scales, one per 16 BF16 values of the block", "bytes": nbytes,
-            "encode_gbs": nbytes / (enc * 1e-3) / 1e9, "decode_gbs": nbytes / (dec * 1e-3) / 1e9,
+    enc = graph_rate(lambda: eh.compress_batch(p, xs, outs, wsc, bits_dev=bits), stream, reps, nbytes)
+    dec = graph_rate(lambda: eh.decompress_batch(p, outs, ys, wsd), stream, reps, nbytes)
+    assert eh.get_status(wsd) == eh.EH_OK and all(torch.equal(x, y) for x, y in zip(xs, ys))
+    return {"kind": f"E4M3 block scales, one per 16 BF16 values of the block; {reps} calls per CUDA graph replay",
+            "bytes": nbytes, "encode_gbs": enc, "decode_gbs": dec,
             "size_ratio": comp / nbytes, "bits_per_scale": 8.0 * sum(o.stream_bytes() for o in outs) / nbytes}
 
 
@@ -383,7 +428,10 @@ def measure_kv_pages(eh, synth, dev, stream, reps=20):
     """Online K/V page store: a K cache of [2, 8192, 8, 128] (256 pages of 64
     tokens); the codebook is frozen from the first 64 pages' exponent counts
     plus one per symbol; the other 192 pages are appended into 28 KB slots in
-    one call and read back in one call (CUDA events, BF16 bytes per second)."""
+    one call and read back in one call.  Device time: `reps` calls of each
+    captured in a CUDA graph and replayed between CUDA events (the calls only
+    enqueue work, so a Python loop of them measures the host's call overhead
+    instead, reported beside as `*_gbs_host_loop`).  BF16 bytes per second."""
     import torch
     rng = np.random.default_rng(3)
     k = synth.kv_tensor(rng, 2, 8192)
@@ -403,22 +451,39 @@ def measure_kv_pages(eh, synth, dev, stream, reps=20):
     assert store.status() == eh.EH_OK
     y = store.read(ids)
     assert torch.equal(y, new)
-    ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
-    ev[0].record(stream)
-    for _ in range(reps):
+    nbytes = 2 * new.numel()
+
+    def timed(fn):
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+        ev[0].record(stream)
+        fn()
+        ev[1].record(stream)
+        torch.cuda.synchronize()
+        return nbytes / (ev[0].elapsed_time(ev[1]) / reps * 1e-3) / 1e9
+
+    def appends():  # on the current stream
+        for _ in range(reps):
+            store.raw_used.zero_()
+            store.append(new, ids)
+
+    def reads():
+        for _ in range(reps):
+            store.read(ids, out=y, check=False)
+
+    host_append, host_read = timed(appends), timed(reads)
+
+    def append1():
         store.raw_used.zero_()
         store.append(new, ids)
-    ev[1].record(stream)
-    for _ in range(reps):
-        store.read(ids, out=y, check=False)
-    ev[2].record(stream)
-    torch.cuda.synchronize()
-    nbytes = 2 * new.numel()
+    dev_append = graph_rate(append1, stream, reps, nbytes)
+    dev_read = graph_rate(lambda: store.read(ids, out=y, check=False), stream, reps, nbytes)
+    assert store.status() == eh.EH_OK and torch.equal(y, new)
     meta = store.page_meta.cpu().numpy().view(np.uint32)
     coded = meta[(meta & 0x80000000) == 0]
-    return {"kind": "K cache [2, 8192, 8, 128] BF16, 192 pages appended after a 64-page prefill",
-            "append_gbs": nbytes / (ev[0].elapsed_time(ev[1]) / reps * 1e-3) / 1e9,
-            "read_gbs": nbytes / (ev[1].elapsed_time(ev[2]) / reps * 1e-3) / 1e9,
+    return {"kind": "K cache [2, 8192, 8, 128] BF16, 192 pages appended after a 64-page prefill; "
+                    f"{reps} calls per CUDA graph replay",
+            "append_gbs": dev_append, "read_gbs": dev_read,
+            "append_gbs_host_loop": host_append, "read_gbs_host_loop": host_read,
             "raw_pages": int((meta & 0x80000000).astype(bool).sum()),
             "bits_per_exponent": float(coded.mean()) / page if coded.size else None,
             "slot_bytes": 28 * 1024}

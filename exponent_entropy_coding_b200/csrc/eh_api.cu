@@ -429,6 +429,11 @@ eh_status eh_pages_append(const eh_plan_t *plan, const eh_page_store_t *store, c
   pl.raw_used = store->raw_used;
   pl.status = (uint32_t *)workspace;
   pl.dtype = plan->dtype;
+  // Calls of fewer pages than two waves of one-CTA-per-page kernels are
+  // split into kPageParts CTAs per page when the workspace holds their part
+  // totals (16 bytes a page).
+  if (n_pages < 4u * (uint32_t)num_sms && workspace_bytes >= kHeader + 4ull * kPageParts * n_pages)
+    pl.part_bits = (uint32_t *)((uint8_t *)workspace + kHeader);
   cudaStream_t s = (cudaStream_t)stream;
   if (cudaMemsetAsync(workspace, 0, 4, s) != cudaSuccess) return EH_ERR_CUDA;
   if (launch_page_append(pl, s) != cudaSuccess) return EH_ERR_CUDA;

@@ -826,6 +826,117 @@ __global__ void __launch_bounds__(kThreads, 2) page_append_kernel(const __grid_c
   }
 }
 
+// Split append, for calls with few pages: kPageParts CTAs per page.
+// Pass 1 (one CTA per part): the part's code bits and missing codes, its
+// sign/mantissa bytes, and the clearing of its share of the page's slot.
+// Pass 2 (one CTA per part): every part reads its page's part totals, takes
+// the same coded/raw decision as the one-CTA kernel, and codes its values at
+// its offset in the slot (the words it shares with the neighbouring parts by
+// atomic OR into the cleared slot); a raw page is copied by its first part.
+constexpr int kPageThreads = 256;
+static_assert(kPageThreads == kEncSmall, "the split append's ring is sized like the small encoder's");
+
+template <int DT>
+__global__ void __launch_bounds__(kPageThreads) page_bits_kernel(const __grid_constant__ PageLaunch pl) {
+  constexpr int A = DT == EH_FP8_E4M3 ? 16 : 256;
+  __shared__ uint2 tab[A];
+  __shared__ uint32_t wsum[kPageThreads / 32];
+  pdl_trigger();
+  const int tid = threadIdx.x;
+  const uint32_t pg = blockIdx.x / kPageParts, part = blockIdx.x % kPageParts;
+  const uint32_t slot = pl.slot_ids[pg];
+  if (slot >= pl.n_slots) {
+    if (tid == 0 && part == 0) set_status(pl.status, kFlagCorrupt);
+    return;
+  }
+  const uint32_t n = pl.page_elems, pn = n / kPageParts, i0 = part * pn;
+  const uint8_t *in = (const uint8_t *)pl.in + ((uint64_t)pg * n + i0) * (DT == EH_BF16 ? 2 : 1);
+  const uint64_t sm_page = DT == EH_BF16 ? n : (DT == EH_FP8_E4M3 ? n / 2 : 0);
+  uint8_t *smo = pl.sm + (uint64_t)slot * sm_page + (DT == EH_BF16 ? i0 : i0 / 2);
+  load_code_table<DT>(tab, pl.code_len, pl.code);
+  // this part's share of the slot's words, cleared for the second pass
+  {
+    uint32_t *sw = (uint32_t *)(pl.slots + (uint64_t)slot * pl.slot_bytes);
+    const uint32_t nw = (uint32_t)(pl.slot_bytes / 4), w0 = nw * part / kPageParts, w1 = nw * (part + 1) / kPageParts;
+    for (uint32_t w = w0 + tid; w < w1; w += kPageThreads) sw[w] = 0u;
+  }
+  __syncthreads();
+  uint32_t bits = 0, missing = 0;
+  for (uint32_t idx = tid * kEncPerThread; idx < pn; idx += kPageThreads * kEncPerThread) {
+    uint4 p, q;
+    load_exps<DT>(in, idx, pn, p, q);
+    #pragma unroll
+    for (int j = 0; j < kEncPerThread; j++) {
+      const uint32_t l = tab[exp_of<DT>(p, q, j)].y;
+      bits += l;
+      missing |= l == 0;
+    }
+    store_sm<DT>(smo, idx, pn, p, q);
+  }
+  uint32_t total;
+  (void)block_excl_scan1<kPageThreads>(bits, wsum, &total);
+  const bool any_missing = __syncthreads_or(missing != 0);
+  if (tid == 0) pl.part_bits[blockIdx.x] = total | (any_missing ? 0x80000000u : 0u);
+}
+
+template <int DT>
+__global__ void __launch_bounds__(kPageThreads) page_encode_kernel(const __grid_constant__ PageLaunch pl) {
+  constexpr int A = DT == EH_FP8_E4M3 ? 16 : 256;
+  extern __shared__ uint32_t ring[];
+  __shared__ uint2 tab[A];
+  __shared__ uint32_t wsum[kPageThreads / 32];
+  __shared__ uint32_t raw_idx;
+  const int tid = threadIdx.x;
+  const uint32_t pg = blockIdx.x / kPageParts, part = blockIdx.x % kPageParts;
+  const uint32_t slot = pl.slot_ids[pg];
+  if (slot >= pl.n_slots) return;
+  const uint32_t n = pl.page_elems, pn = n / kPageParts, i0 = part * pn;
+  load_code_table<DT>(tab, pl.code_len, pl.code);
+  for (int i = tid; i < Enc<kPageThreads>::kRingWords; i += kPageThreads) ring[i] = 0u;
+  pdl_wait();  // the part totals, the cleared slot
+  uint32_t total = 0, before = 0;
+  bool missing = false;
+  #pragma unroll
+  for (uint32_t k = 0; k < kPageParts; k++) {
+    const uint32_t v = pl.part_bits[pg * kPageParts + k];
+    missing |= (v >> 31) != 0;
+    total += v & 0x7FFFFFFFu;
+    if (k < part) before += v & 0x7FFFFFFFu;
+  }
+  const uint32_t mine = pl.part_bits[blockIdx.x] & 0x7FFFFFFFu;
+  __syncthreads();
+  const uint8_t *page_in = (const uint8_t *)pl.in + (uint64_t)pg * n * (DT == EH_BF16 ? 2 : 1);
+  const bool coded = !missing && (total + 7) / 8 + 16 <= pl.slot_bytes;
+  if (coded) {
+    const uint64_t b0 = (uint64_t)slot * pl.slot_bytes * 8 + before;
+    encode_range<DT, kPageThreads>(tab, page_in + (uint64_t)i0 * (DT == EH_BF16 ? 2 : 1), pn, b0, b0 + mine,
+                                   (uint32_t *)pl.slots, ring, wsum, false);
+    if (tid == 0 && part == 0) pl.page_meta[slot] = total;
+    return;
+  }
+  if (part != 0) return;
+  if (tid == 0) {
+    raw_idx = atomicAdd(pl.raw_used, 1u);
+    if (raw_idx >= pl.raw_cap) set_status(pl.status, kFlagNoRoom);
+    pl.page_meta[slot] = EH_PAGE_RAW | (raw_idx < pl.raw_cap ? raw_idx : 0x7FFFFFFFu);
+  }
+  __syncthreads();
+  if (raw_idx >= pl.raw_cap) return;
+  uint8_t *dst = pl.raw_pool + (uint64_t)raw_idx * n;
+  for (uint32_t idx = tid * kEncPerThread; idx < n; idx += kPageThreads * kEncPerThread) {
+    uint4 p, q;
+    load_exps<DT>(page_in, idx, n, p, q);
+    uint32_t o[4];
+    #pragma unroll
+    for (int w = 0; w < 4; w++) {
+      o[w] = 0;
+      #pragma unroll
+      for (int k = 0; k < 4; k++) o[w] |= exp_of<DT>(p, q, 4 * w + k) << (8 * k);
+    }
+    *(uint4 *)(dst + idx) = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+}
+
 }  // namespace
 
 cudaError_t launch_hist(const Batch &b, cudaStream_t s) {
@@ -862,11 +973,27 @@ cudaError_t configure_encode() {
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(page_append_kernel<EH_BYTES>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  return cudaFuncSetAttribute(page_append_kernel<EH_FP8_E4M3>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  e = cudaFuncSetAttribute(page_append_kernel<EH_FP8_E4M3>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e == cudaSuccess) e = cudaFuncSetAttribute(page_encode_kernel<EH_BF16>, dyn, small);
+  if (e == cudaSuccess) e = cudaFuncSetAttribute(page_encode_kernel<EH_BYTES>, dyn, small);
+  if (e == cudaSuccess) e = cudaFuncSetAttribute(page_encode_kernel<EH_FP8_E4M3>, dyn, small);
+  return e;
 }
 
 cudaError_t launch_page_append(const PageLaunch &pl, cudaStream_t s) {
   if (pl.n_pages == 0) return cudaSuccess;
+  if (pl.part_bits) {
+    const dim3 grid(pl.n_pages * kPageParts), block(kPageThreads);
+    const size_t ring = Enc<kPageThreads>::kRingWords * sizeof(uint32_t);
+    if (pl.dtype == EH_BF16) page_bits_kernel<EH_BF16><<<grid, block, 0, s>>>(pl);
+    else if (pl.dtype == EH_BYTES) page_bits_kernel<EH_BYTES><<<grid, block, 0, s>>>(pl);
+    else page_bits_kernel<EH_FP8_E4M3><<<grid, block, 0, s>>>(pl);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    if (pl.dtype == EH_BF16) return launch_pdl(page_encode_kernel<EH_BF16>, grid, block, ring, s, pl);
+    if (pl.dtype == EH_BYTES) return launch_pdl(page_encode_kernel<EH_BYTES>, grid, block, ring, s, pl);
+    return launch_pdl(page_encode_kernel<EH_FP8_E4M3>, grid, block, ring, s, pl);
+  }
   const size_t smem = Enc<kThreads>::kRingWords * sizeof(uint32_t);
   if (pl.dtype == EH_BF16) page_append_kernel<EH_BF16><<<pl.n_pages, kThreads, smem, s>>>(pl);
   else if (pl.dtype == EH_BYTES) page_append_kernel<EH_BYTES><<<pl.n_pages, kThreads, smem, s>>>(pl);

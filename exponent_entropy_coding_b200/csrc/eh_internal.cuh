@@ -79,8 +79,10 @@ struct PageLaunch {
   uint8_t *raw_pool;
   uint32_t *raw_used;
   uint32_t *status;
+  uint32_t *part_bits;     // split append: [n_pages][kPageParts] code bits | missing << 31 (null: one CTA a page)
   int32_t dtype;
 };
+constexpr uint32_t kPageParts = 4;  // CTAs per page in the split append
 
 struct Batch {
   Item item[EH_MAX_BATCH];

@@ -270,7 +270,9 @@ EH_API eh_status eh_codebook_from_counts(const eh_plan_t *plan, const uint64_t *
 
 /* Codes n_pages full pages (in: n_pages * chunk_elems values, page i first)
  * into the slots slot_ids[i] (device array).  Stream-ordered; a full raw pool
- * sets EH_ERR_NOMEM in the workspace status word (workspace: 256 bytes). */
+ * sets EH_ERR_NOMEM in the workspace status word.  Workspace: 256 bytes;
+ * with 256 + 16 * n_pages bytes, calls of up to a few hundred pages code
+ * each page with several CTAs (the result is the same). */
 EH_API eh_status eh_pages_append(const eh_plan_t *plan, const eh_page_store_t *store,
                                  const void *in, uint32_t n_pages,
                                  const uint32_t *slot_ids, void *workspace,
