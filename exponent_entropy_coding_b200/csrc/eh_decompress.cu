@@ -1,6 +1,6 @@
 // eh_decompress.cu -- decompression kernels of libexphuff (sm_100a).
 //
-//   tables  eight CTAs per codebook: validate the code lengths and codes and
+//   tables  sixteen CTAs per codebook: validate the code lengths and codes and
 //           build the decode tables (a 12-bit first level giving, for the
 //           index bits, the number, bits and start offsets of all complete
 //           codes and the symbols and bits of the first four; 8-bit second
@@ -42,8 +42,9 @@ constexpr uint64_t kWaitLimitNs = 200000000ull;  // a stage copy not landed afte
 
 // ---------------------------------------------------------------- tables
 // kTabParts CTAs of 256 threads per codebook; each builds 1/kTabParts of the
-// first level, part 0 also writes the second levels and the limits.
-constexpr uint32_t kTabParts = 8;
+// first level (one entry a thread), parts 0..kNumSub-1 one second-level table
+// each, part 0 also the limits.
+constexpr uint32_t kTabParts = 16;
 
 // Smallest L in [1, 32] with x < lim[L], 33 if there is none (lim is
 // nondecreasing for a valid code).
@@ -184,9 +185,9 @@ __global__ void __launch_bounds__(256) tables_kernel(const __grid_constant__ Bat
     if (nc) meta = pos | ((bnd >> 1) << kMetaStartShift) | (nc << 16) | (pos4 << 20) | ((8u * nc4) << 24);
     T->l1[p] = make_uint2(syms, meta);
   }
-  if (part != 0) return;
-  // second level: codes of kLutBits+1 .. kLutBits+8 bits
-  for (uint32_t j = 0; j < (uint32_t)kNumSub; j++) {
+  // second level (one table per part): codes of kLutBits+1 .. kLutBits+8 bits
+  if (part < (uint32_t)kNumSub) {
+    const uint32_t j = part;
     uint32_t e = 0;
     const uint32_t p = sub0 + j;
     if (((uint64_t)p << kShift) < limL[32]) {
@@ -203,7 +204,7 @@ __global__ void __launch_bounds__(256) tables_kernel(const __grid_constant__ Bat
     }
     T->sub[j][tid] = e;
   }
-  if (tid == 0) T->err = err;
+  if (tid == 0 && part == 0) T->err = err;
 }
 
 // ---------------------------------------------------------------- decode
