@@ -305,6 +305,37 @@ def run_ncu_case():
     return 0
 
 
+def run_ncu_pages():
+    """Small case for profiler captures of the page store: the K/V workload's
+    192 pages (25 MB of BF16) appended once into 28 KB slots with a codebook
+    frozen from the first 64 pages, then read back once: one launch each of
+    page_bits_kernel, page_encode_kernel and (page mode) decode_kernel."""
+    import torch
+
+    from exponent_entropy_coding_b200 import exphuff as eh
+    from exponent_entropy_coding_b200 import synth
+    dev = torch.device("cuda", 0)
+    k = synth.kv_tensor(np.random.default_rng(3), 2, 8192)
+    page = 65536
+    p = eh.plan(eh.EH_BF16)
+    prefill = torch.from_numpy(k[: 64 * page].view(np.int16)).to(dev)
+    scratch = eh.alloc_compressed(p, prefill.numel(), dev)
+    ws = torch.empty(eh.compress_bound(p, prefill.numel())[2], dtype=torch.uint8, device=dev)
+    counts = torch.zeros(256, dtype=torch.int64, device=dev)
+    eh.compress_shard_begin(prefill, scratch, counts, p, ws)  # the prefill's exponent counts
+    code_len, code = eh.codebook_from_counts(p, counts + 1)
+    new = torch.from_numpy(k[64 * page:].view(np.int16)).to(dev)
+    n_new = new.numel() // page
+    store = eh.PageStore(p, code_len, code, n_slots=n_new, slot_bytes=28 * 1024, raw_cap=n_new, device=dev)
+    ids = torch.arange(n_new, dtype=torch.int32, device=dev)
+    store.append(new, ids)
+    y = store.read(ids)
+    torch.cuda.synchronize()
+    assert store.status() == eh.EH_OK and torch.equal(y, new)
+    print(json.dumps({"case": "K/V page store, 192 pages", "raw_pages": int((store.page_meta < 0).sum())}))
+    return 0
+
+
 def run_all_configs(reps=20):
     """One JSON line per workload (the five of the codec's table): batched
     compress and decompress timed with CUDA events, median of `reps` after 3
@@ -644,11 +675,14 @@ def main():
                     help="skip the side measurements (FP4 scales, K/V pages, ZipFloat, prefetch ring)")
     ap.add_argument("--all-configs", action="store_true",
                     help="one line per workload of the codec's table (compress/decompress, fractions, oracle)")
-    ap.add_argument("--ncu-case", action="store_true",
-                    help="one compress + one decompress of gate_proj (14336x4096), for ncu captures")
+    ap.add_argument("--ncu-case", nargs="?", const="gate", choices=["gate", "pages"],
+                    help="for ncu captures: one compress + one decompress of gate_proj (14336x4096), "
+                         "or (pages) one append + one read of the 192-page K/V store")
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)
+    if args.ncu_case == "pages":
+        return run_ncu_pages()
     if args.ncu_case:
         return run_ncu_case()
     if args.all_configs:

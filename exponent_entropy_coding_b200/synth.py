@@ -76,14 +76,13 @@ def normal_fp8(n: int, seed: int, std: float = 0.02) -> np.ndarray:
     return to_fp8_e4m3_bits(w)
 
 
-def fibonacci_bf16(m: int, seed: int, first_field: int = 60, chunk: int = 65536) -> np.ndarray:
-    """BF16 values whose exponent fields first_field .. first_field+m-1 occur
-    F(1), F(2), ..., F(m) times (Fibonacci numbers): the histogram that gives
-    a Huffman code its largest depth, m - 1.  Each value is
-    +-(1 + k/128) * 2^(field - 127) with random sign and k.  Placement: the
-    first chunk holds one of the two rarest values, the next 14 rarest and
-    common values; the second chunk holds the other rarest value and values
-    of middle rarity (long codes on average); the rest is shuffled."""
+def fibonacci_symbols(m: int, seed: int, chunk: int = 65536) -> np.ndarray:
+    """Symbol indices 0 .. m-1 occurring F(1), F(2), ..., F(m) times
+    (Fibonacci numbers): the histogram that gives a Huffman code its largest
+    depth, m - 1.  Placement: the first chunk holds one of the two rarest
+    symbols, the next 14 rarest and common ones; the second chunk holds the
+    other rarest symbol and symbols of middle rarity (long codes on
+    average); the rest is shuffled."""
     rng = np.random.default_rng(seed)
     fib = [1, 1]
     while len(fib) < m:
@@ -108,7 +107,15 @@ def fibonacci_bf16(m: int, seed: int, first_field: int = 60, chunk: int = 65536)
     second = second[rng.permutation(second.size)]
     rest = np.concatenate(pools)
     rest = rest[rng.permutation(rest.size)]
-    idx = np.concatenate([head, second, rest])
+    return np.concatenate([head, second, rest])
+
+
+def fibonacci_bf16(m: int, seed: int, first_field: int = 60, chunk: int = 65536) -> np.ndarray:
+    """BF16 values whose exponent fields first_field .. first_field+m-1 follow
+    fibonacci_symbols(m, seed, chunk).  Each value is
+    +-(1 + k/128) * 2^(field - 127) with random sign and k."""
+    idx = fibonacci_symbols(m, seed, chunk)
+    rng = np.random.default_rng(seed + 1000)
     field = (idx + first_field).astype(np.float64)
     mant = rng.integers(0, 128, idx.size)
     sign = np.where(rng.integers(0, 2, idx.size) == 1, -1.0, 1.0)

@@ -93,6 +93,26 @@ def test_pages_append_and_read(eh, oracle, smooth):
     assert np.array_equal(y.cpu().numpy().view(np.uint16), want)
 
 
+@pytest.mark.parametrize("smooth", [True, False])
+def test_pages_one_cta_per_page(eh, oracle, smooth):
+    # With a 256-byte workspace (no room for the part totals) every page is
+    # coded by one CTA; slots, records and raw pages must be the same.
+    p, book, prefill, new = _setup(eh, oracle, smooth=smooth)
+    n_new = new.size // PAGE
+    store = eh.PageStore(p, book.code_len, book.code, n_slots=40, slot_bytes=28 * 1024, raw_cap=24,
+                         device="cuda")
+    read_ws = store.workspace
+    store.workspace = torch.empty(256, dtype=torch.uint8, device="cuda")
+    slot_ids = np.random.default_rng(2).permutation(40)[:n_new]
+    store.append(torch.from_numpy(new.view(np.int16)).cuda(), torch.from_numpy(slot_ids))
+    assert store.status() == eh.EH_OK
+    n_raw = _check_against_oracle(eh, oracle, store, book, new, slot_ids)
+    assert n_raw == 0 if smooth else n_raw >= 1
+    store.workspace = read_ws
+    y = store.read(torch.from_numpy(slot_ids))
+    assert np.array_equal(y.cpu().numpy().view(np.uint16), new)
+
+
 def test_small_slots_go_raw(eh, oracle):
     p, book, prefill, new = _setup(eh, oracle, n_new=8)
     store = eh.PageStore(p, book.code_len, book.code, n_slots=8, slot_bytes=16 * 1024, raw_cap=8,

@@ -187,6 +187,17 @@ def test_codes_of_32_bits(eh, oracle, m):
         assert np.array_equal(host_bits(y, 0), x[first * CHUNK:(first + count) * CHUNK])
 
 
+@pytest.mark.parametrize("m", [33, 34])
+def test_byte_codes_of_32_bits(eh, oracle, m):
+    # The byte alphabet (FP4 block scales) with the same Fibonacci counts:
+    # 32-bit codes through the decoder's byte path, staged and unstaged.
+    x = (synth.fibonacci_symbols(m, seed=m) + 40).astype(np.uint8)
+    c = roundtrip(eh, oracle, 2, x)
+    lens = c.code_len.cpu().numpy()
+    assert lens.max() == 32
+    assert lens[x[:CHUNK]].max() == 32 and lens[x[CHUNK:2 * CHUNK]].max() == 32
+
+
 def test_length_limited_real_data(eh, oracle):
     roundtrip(eh, oracle, 0, synth.normal_bf16(3 * 65536, seed=8), lmax=7)
     roundtrip(eh, oracle, 1, synth.normal_fp8(3 * 65536, seed=8), lmax=4)
