@@ -425,7 +425,8 @@ EH_API eh_status eh_container_write(const eh_plan_t *plan, const eh_compressed_t
  * CRC-32; EH_ERR_CORRUPT on any mismatch) and fills *plan and *view, whose
  * array pointers point into src (exp_stream_cap = the stream's byte
  * length).  Padding and reserved bytes must be zero, so that a change to any
- * byte of a container is detected. */
+ * byte of a container is detected.  src_bytes may exceed the container's size
+ * (a container inside a larger file): the bytes after it are not read. */
 EH_API eh_status eh_container_read(const void *src, uint64_t src_bytes, eh_plan_t *plan,
                                    eh_compressed_t *view);
 

@@ -104,3 +104,14 @@ def test_container_write_needs_room(oracle):
     s.exp_stream_cap, s.sign_mant = host["exp_stream"].size, host["sign_mant"].ctypes.data
     rc = eh.lib().eh_container_write(C.byref(p), C.byref(s), out.ctypes.data_as(C.c_void_p), out.size)
     assert rc == eh.EH_ERR_NOMEM
+
+
+def test_container_inside_a_larger_buffer(oracle):
+    # bytes after the container are ignored; a container cut short is refused
+    x, r, idx, c, p = _host_compressed(oracle, 0, 70000, 65536, False)
+    buf = eh.to_container(c, p)
+    c2, _ = eh.from_container(buf + bytes(range(200)), "cpu")
+    assert torch.equal(c2.sign_mant, c.sign_mant) and c2.exp_stream_bits == c.exp_stream_bits
+    for cut in (0, 100, 191, 192, len(buf) - 16, len(buf) - 1):
+        with pytest.raises(eh.EhError):
+            eh.from_container(buf[:cut], "cpu")
