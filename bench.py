@@ -459,7 +459,9 @@ def measure_kv_pages(eh, synth, dev, stream, reps=20):
     """Online K/V page store: a K cache of [2, 8192, 8, 128] (256 pages of 64
     tokens); the codebook is frozen from the first 64 pages' exponent counts
     plus one per symbol; the other 192 pages are appended into 28 KB slots in
-    one call and read back in one call.  Device time: `reps` calls of each
+    one call and read back in one call, with the decode tables prepared once
+    (`read_gbs`; building them in every read: `read_gbs_tables_per_call`).
+    Device time: `reps` calls of each
     captured in a CUDA graph and replayed between CUDA events (the calls only
     enqueue work, so a Python loop of them measures the host's call overhead
     instead, reported beside as `*_gbs_host_loop`).  BF16 bytes per second."""
@@ -507,13 +509,15 @@ def measure_kv_pages(eh, synth, dev, stream, reps=20):
         store.raw_used.zero_()
         store.append(new, ids)
     dev_append = graph_rate(append1, stream, reps, nbytes)
+    dev_read_tables = graph_rate(lambda: store.read(ids, out=y, check=False), stream, reps, nbytes)
+    store.prepare()  # the frozen codebook's decode tables, built once
     dev_read = graph_rate(lambda: store.read(ids, out=y, check=False), stream, reps, nbytes)
     assert store.status() == eh.EH_OK and torch.equal(y, new)
     meta = store.page_meta.cpu().numpy().view(np.uint32)
     coded = meta[(meta & 0x80000000) == 0]
     return {"kind": "K cache [2, 8192, 8, 128] BF16, 192 pages appended after a 64-page prefill; "
                     f"{reps} calls per CUDA graph replay",
-            "append_gbs": dev_append, "read_gbs": dev_read,
+            "append_gbs": dev_append, "read_gbs": dev_read, "read_gbs_tables_per_call": dev_read_tables,
             "append_gbs_host_loop": host_append, "read_gbs_host_loop": host_read,
             "raw_pages": int((meta & 0x80000000).astype(bool).sum()),
             "bits_per_exponent": float(coded.mean()) / page if coded.size else None,

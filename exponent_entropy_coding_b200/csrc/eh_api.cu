@@ -440,27 +440,30 @@ eh_status eh_pages_append(const eh_plan_t *plan, const eh_page_store_t *store, c
   return EH_OK;
 }
 
-eh_status eh_pages_read(const eh_plan_t *plan, const eh_page_store_t *store, const uint32_t *slot_ids,
-                        uint32_t n_pages, void *out, void *workspace, uint64_t workspace_bytes, void *stream) {
-  if (!plan_ok(plan) || !store || !workspace) return EH_ERR_INVALID_ARG;
-  if (((uintptr_t)workspace & 255u) != 0) return EH_ERR_INVALID_ARG;
-  if (workspace_bytes < kHeader + kLutBytes) return EH_ERR_NOMEM;
-  if (n_pages == 0) return EH_OK;
+namespace {
+
+// Arguments of a page-store read that the decoder relies on.
+bool page_read_args_ok(const eh_plan_t *plan, const eh_page_store_t *store, const uint32_t *slot_ids,
+                       const void *out) {
   const bool has_sm = plan->dtype != EH_BYTES;
-  if (!out || !slot_ids || !store->code_len || !store->code || !store->slots || !store->page_meta ||
-      (has_sm && !store->sign_mant) || !aligned16(out) || !aligned16(store->slots) ||
-      (has_sm && !aligned16(store->sign_mant)) || (store->raw_pool && !aligned16(store->raw_pool)) ||
-      store->slot_bytes % 16 || store->slot_bytes == 0)
-    return EH_ERR_INVALID_ARG;
-  uint8_t *ws = (uint8_t *)workspace;
-  Batch b;
+  return out && slot_ids && store->code_len && store->code && store->slots && store->page_meta &&
+         (!has_sm || store->sign_mant) && aligned16(out) && aligned16(store->slots) &&
+         (!has_sm || aligned16(store->sign_mant)) && (!store->raw_pool || aligned16(store->raw_pool)) &&
+         store->slot_bytes % 16 == 0 && store->slot_bytes != 0;
+}
+
+// The decoder's descriptor of a read of n_pages pages, with the decode
+// tables at `lut` and the status word at `status`.
+void page_read_batch(const eh_plan_t *plan, const eh_page_store_t *store, const uint32_t *slot_ids,
+                     uint32_t n_pages, void *out, uint8_t *status, const void *lut, Batch *bp) {
+  Batch &b = *bp;
   std::memset(&b, 0, sizeof(b));
   b.k = 1;
   b.chunk_elems = plan->chunk_elems;
   b.dtype = plan->dtype;
   b.max_code_len = plan->max_code_len;
-  b.status = (uint32_t *)ws;
-  b.ticket = (uint32_t *)(ws + 4);
+  b.status = (uint32_t *)status;
+  b.ticket = (uint32_t *)(status + 4);
   b.total_chunks = n_pages;
   Item &it = b.item[0];
   it.out = out;
@@ -473,17 +476,75 @@ eh_status eh_pages_read(const eh_plan_t *plan, const eh_page_store_t *store, con
   it.stream = store->slots;
   it.stream_cap = (uint64_t)store->n_slots * store->slot_bytes;
   it.sm = store->sign_mant;
-  it.lut = ws + kHeader;
+  it.lut = const_cast<void *>(lut);
   it.slot_ids = slot_ids;
   it.page_meta = store->page_meta;
   it.raw_pool = store->raw_pool;
   it.slot_bytes = store->slot_bytes;
   it.n_slots = store->n_slots;
   it.raw_cap = store->raw_cap;
+}
+
+}  // namespace
+
+eh_status eh_pages_read(const eh_plan_t *plan, const eh_page_store_t *store, const uint32_t *slot_ids,
+                        uint32_t n_pages, void *out, void *workspace, uint64_t workspace_bytes, void *stream) {
+  if (!plan_ok(plan) || !store || !workspace) return EH_ERR_INVALID_ARG;
+  if (((uintptr_t)workspace & 255u) != 0) return EH_ERR_INVALID_ARG;
+  if (workspace_bytes < kHeader + kLutBytes) return EH_ERR_NOMEM;
+  if (n_pages == 0) return EH_OK;
+  if (!page_read_args_ok(plan, store, slot_ids, out)) return EH_ERR_INVALID_ARG;
+  uint8_t *ws = (uint8_t *)workspace;
+  Batch b;
+  page_read_batch(plan, store, slot_ids, n_pages, out, ws, ws + kHeader, &b);
   int num_sms = 0;
   if (device_setup(&num_sms) != cudaSuccess) return EH_ERR_CUDA;
   cudaStream_t s = (cudaStream_t)stream;
   if (launch_tables(b, s) != cudaSuccess) return EH_ERR_CUDA;
+  if (launch_decode(b, s, num_sms) != cudaSuccess) return EH_ERR_CUDA;
+  return EH_OK;
+}
+
+eh_status eh_pages_prepare(const eh_plan_t *plan, const eh_page_store_t *store, void *tables,
+                           uint64_t tables_bytes, void *stream) {
+  if (!plan_ok(plan) || !store || !store->code_len || !store->code || !tables) return EH_ERR_INVALID_ARG;
+  if (((uintptr_t)tables & 255u) != 0) return EH_ERR_INVALID_ARG;
+  if (tables_bytes < kHeader + kLutBytes) return EH_ERR_NOMEM;
+  uint8_t *t = (uint8_t *)tables;
+  Batch b;
+  std::memset(&b, 0, sizeof(b));
+  b.k = 1;
+  b.chunk_elems = plan->chunk_elems;
+  b.dtype = plan->dtype;
+  b.max_code_len = plan->max_code_len;
+  b.status = (uint32_t *)t;
+  b.ticket = (uint32_t *)(t + 4);
+  Item &it = b.item[0];
+  it.n = plan->chunk_elems;  // pages hold values: a codebook without codes is invalid
+  it.code_len = const_cast<uint8_t *>(store->code_len);
+  it.code = const_cast<uint32_t *>(store->code);
+  it.lut = t + kHeader;
+  int num_sms = 0;
+  if (device_setup(&num_sms) != cudaSuccess) return EH_ERR_CUDA;
+  if (launch_tables(b, (cudaStream_t)stream) != cudaSuccess) return EH_ERR_CUDA;
+  return EH_OK;
+}
+
+eh_status eh_pages_read_prepared(const eh_plan_t *plan, const eh_page_store_t *store, const void *tables,
+                                 const uint32_t *slot_ids, uint32_t n_pages, void *out, void *workspace,
+                                 uint64_t workspace_bytes, void *stream) {
+  if (!plan_ok(plan) || !store || !tables || !workspace) return EH_ERR_INVALID_ARG;
+  if (((uintptr_t)workspace & 255u) != 0 || ((uintptr_t)tables & 255u) != 0) return EH_ERR_INVALID_ARG;
+  if (workspace_bytes < kHeader) return EH_ERR_NOMEM;
+  if (n_pages == 0) return EH_OK;
+  if (!page_read_args_ok(plan, store, slot_ids, out)) return EH_ERR_INVALID_ARG;
+  uint8_t *ws = (uint8_t *)workspace;
+  Batch b;
+  page_read_batch(plan, store, slot_ids, n_pages, out, ws, (const uint8_t *)tables + kHeader, &b);
+  int num_sms = 0;
+  if (device_setup(&num_sms) != cudaSuccess) return EH_ERR_CUDA;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (cudaMemsetAsync(ws, 0, 8, s) != cudaSuccess) return EH_ERR_CUDA;  // this call's status starts clean
   if (launch_decode(b, s, num_sms) != cudaSuccess) return EH_ERR_CUDA;
   return EH_OK;
 }

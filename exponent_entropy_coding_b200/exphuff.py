@@ -33,7 +33,7 @@ EXPORTED = ["eh_plan", "eh_compress_bound", "eh_compress_batch_workspace", "eh_c
             "eh_compress_batch", "eh_compress_shard_begin", "eh_compress_shard_finish",
             "eh_decompress_workspace", "eh_decompress", "eh_decompress_batch",
             "eh_decompress_chunks", "eh_decompress_batch_noalloc", "eh_codebook_from_counts",
-            "eh_pages_append", "eh_pages_read",
+            "eh_pages_append", "eh_pages_read", "eh_pages_prepare", "eh_pages_read_prepared",
             "eh_prefetch_workspace", "eh_prefetch_create", "eh_prefetch_submit",
             "eh_prefetch_acquire", "eh_prefetch_release", "eh_prefetch_status",
             "eh_prefetch_destroy",
@@ -108,6 +108,8 @@ def lib():
             "eh_codebook_from_counts": [P(eh_plan_t), vp, vp, vp, vp, u64, vp],
             "eh_pages_append": [P(eh_plan_t), P(eh_page_store_t), vp, u32, vp, vp, u64, vp],
             "eh_pages_read": [P(eh_plan_t), P(eh_page_store_t), vp, u32, vp, vp, u64, vp],
+            "eh_pages_prepare": [P(eh_plan_t), P(eh_page_store_t), vp, u64, vp],
+            "eh_pages_read_prepared": [P(eh_plan_t), P(eh_page_store_t), vp, vp, u32, vp, vp, u64, vp],
             "eh_prefetch_workspace": [P(eh_plan_t), C.c_int, P(u64)],
             "eh_prefetch_create": [P(eh_plan_t), C.c_int, P(vp), u64, vp, u64, vp, u32, P(vp)],
             "eh_prefetch_submit": [vp, C.c_int, P(eh_compressed_t), P(u64), P(C.c_int)],
@@ -492,6 +494,7 @@ class PageStore:
         self.raw_pool = torch.empty(max(raw_cap, 1) * n, dtype=torch.uint8, device=dev)
         self.raw_used = torch.zeros(1, dtype=torch.int32, device=dev)
         self.workspace = torch.empty(max(256, decompress_workspace(p, 1)), dtype=torch.uint8, device=dev)
+        self.tables = None  # decode tables built once by prepare()
 
     def struct(self) -> eh_page_store_t:
         s = eh_page_store_t()
@@ -518,6 +521,14 @@ class PageStore:
         _check(rc, "eh_pages_append")
         return ids
 
+    def prepare(self, stream=None):
+        """Builds the frozen codebook's decode tables once; later reads use
+        them (eh_pages_read_prepared) instead of building them every call."""
+        self.tables = torch.empty(decompress_workspace(self.plan, 1), dtype=torch.uint8, device=self.slots.device)
+        st = self.struct()
+        _check(lib().eh_pages_prepare(C.byref(self.plan), C.byref(st), C.c_void_p(self.tables.data_ptr()),
+                                      self.tables.numel(), _stream_ptr(stream)), "eh_pages_prepare")
+
     def read(self, slot_ids: torch.Tensor, out: Optional[torch.Tensor] = None, stream=None,
              check: bool = True) -> torch.Tensor:
         ids = slot_ids.to(device=self.slots.device, dtype=torch.int32).contiguous()
@@ -525,10 +536,17 @@ class PageStore:
         if out is None:
             out = torch.empty(n, dtype=_elem_dtype(self.plan.dtype), device=self.slots.device)
         st = self.struct()
-        rc = lib().eh_pages_read(C.byref(self.plan), C.byref(st), C.c_void_p(ids.data_ptr()), ids.numel(),
-                                 C.c_void_p(out.data_ptr()), C.c_void_p(self.workspace.data_ptr()),
-                                 self.workspace.numel(), _stream_ptr(stream))
-        _check(rc, "eh_pages_read")
+        if self.tables is not None:
+            rc = lib().eh_pages_read_prepared(C.byref(self.plan), C.byref(st), C.c_void_p(self.tables.data_ptr()),
+                                              C.c_void_p(ids.data_ptr()), ids.numel(), C.c_void_p(out.data_ptr()),
+                                              C.c_void_p(self.workspace.data_ptr()), self.workspace.numel(),
+                                              _stream_ptr(stream))
+            _check(rc, "eh_pages_read_prepared")
+        else:
+            rc = lib().eh_pages_read(C.byref(self.plan), C.byref(st), C.c_void_p(ids.data_ptr()), ids.numel(),
+                                     C.c_void_p(out.data_ptr()), C.c_void_p(self.workspace.data_ptr()),
+                                     self.workspace.numel(), _stream_ptr(stream))
+            _check(rc, "eh_pages_read")
         if check:
             _check(get_status(self.workspace, stream), "eh_pages_read (device status)")
         return out

@@ -284,6 +284,20 @@ EH_API eh_status eh_pages_read(const eh_plan_t *plan, const eh_page_store_t *sto
                                const uint32_t *slot_ids, uint32_t n_pages, void *out,
                                void *workspace, uint64_t workspace_bytes, void *stream);
 
+/* The store's codebook is frozen, so its decode tables can be built once:
+ * eh_pages_prepare builds them into `tables` (device, 256-byte aligned,
+ * eh_decompress_workspace(plan, 1) bytes; an invalid codebook is recorded
+ * there and every read with these tables reports EH_ERR_CORRUPT), and
+ * eh_pages_read_prepared reads pages with them instead of rebuilding them
+ * every call (workspace: 256 bytes, the call's status word).  The tables
+ * must be prepared again if store->code_len or store->code change. */
+EH_API eh_status eh_pages_prepare(const eh_plan_t *plan, const eh_page_store_t *store,
+                                  void *tables, uint64_t tables_bytes, void *stream);
+EH_API eh_status eh_pages_read_prepared(const eh_plan_t *plan, const eh_page_store_t *store,
+                                        const void *tables, const uint32_t *slot_ids,
+                                        uint32_t n_pages, void *out, void *workspace,
+                                        uint64_t workspace_bytes, void *stream);
+
 /* ---- Prefetcher: decompression straight into the operand buffers of the
  * next consumer (a GEMM), on a decode stream that runs ahead of the consumer
  * stream.  The DFloat11 article ("方法介绍") decompresses a whole transformer

@@ -113,6 +113,31 @@ def test_pages_one_cta_per_page(eh, oracle, smooth):
     assert np.array_equal(y.cpu().numpy().view(np.uint16), new)
 
 
+def test_prepared_tables(eh, oracle):
+    # The frozen codebook's decode tables built once (eh_pages_prepare) serve
+    # every later read (eh_pages_read_prepared), in any page order; tables
+    # prepared from an invalid codebook make reads report corruption.
+    p, book, prefill, new = _setup(eh, oracle, n_new=12)
+    store = eh.PageStore(p, book.code_len, book.code, n_slots=16, slot_bytes=28 * 1024, raw_cap=4,
+                         device="cuda")
+    slot_ids = np.random.default_rng(5).permutation(16)[:12]
+    store.append(torch.from_numpy(new.view(np.int16)).cuda(), torch.from_numpy(slot_ids))
+    assert store.status() == eh.EH_OK
+    store.prepare()
+    rng = np.random.default_rng(6)
+    for _ in range(3):
+        order = rng.permutation(12)[: rng.integers(1, 13)]
+        y = store.read(torch.from_numpy(slot_ids[order]))
+        want = np.concatenate([new[i * PAGE:(i + 1) * PAGE] for i in order])
+        assert np.array_equal(y.cpu().numpy().view(np.uint16), want)
+    good = store.code_len
+    store.code_len = torch.ones_like(good)  # every symbol 1 bit long: Kraft sum far above 1
+    store.prepare()
+    store.code_len = good
+    store.read(torch.from_numpy(slot_ids[:2]), check=False)
+    assert store.status() == eh.EH_ERR_CORRUPT
+
+
 def test_small_slots_go_raw(eh, oracle):
     p, book, prefill, new = _setup(eh, oracle, n_new=8)
     store = eh.PageStore(p, book.code_len, book.code, n_slots=8, slot_bytes=16 * 1024, raw_cap=8,
