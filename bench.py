@@ -34,7 +34,7 @@ FALLBACK_HBM_GBS = 6650.0
 # DRAM traffic per decode launch on the full block, from one ncu capture
 # (dram__bytes_read.sum + dram__bytes_write.sum), valid only for the decoder
 # source it was taken on.
-DECODE_TRAFFIC = {"bytes": 301516544 + 377785600, "source_sha": "77a2c177e5c386a7"}
+DECODE_TRAFFIC = {"bytes": 301308928 + 377901312, "source_sha": "6ceea4ebebfb7656"}
 
 
 def decoder_source_sha():

@@ -625,7 +625,9 @@ __device__ __forceinline__ void ring_or64(uint32_t *ring, uint32_t pos, uint32_t
 // of gs.  The ring must be zero on entry and is zero on return.  Words that
 // the range shares with its neighbours are OR-ed into (pre-cleared) stream
 // words unless `exclusive`, when the range owns every word it touches.
-template <int DT, int NT>
+// kIndex: the value index is written (into vindex); without it the encoding
+// loop carries no index code at all.
+template <int DT, int NT, bool kIndex = false>
 __device__ void encode_range(const uint2 *tab, const uint8_t *in, uint32_t cnt, uint64_t bit0, uint64_t bit1,
                              uint32_t *gs, uint32_t *ring, uint32_t *wsum, bool exclusive,
                              uint32_t *vindex = nullptr, uint8_t *smo = nullptr) {
@@ -671,7 +673,7 @@ __device__ void encode_range(const uint2 *tab, const uint8_t *in, uint32_t cnt, 
     uint32_t pos = tile_base + excl;
     // value index: where every kIndexStride-th value's code starts, from the
     // range's first bit
-    if (vindex && (idx % kIndexStride) == 0 && idx < cnt) vindex[idx / kIndexStride] = pos - r0;
+    if (kIndex && (idx % kIndexStride) == 0 && idx < cnt) vindex[idx / kIndexStride] = pos - r0;
     #pragma unroll
     for (int h = 0; h < 2; h++) {
       if (tot[h] == 0) continue;
@@ -714,7 +716,9 @@ __device__ __forceinline__ void load_code_table(uint2 *tab, const uint8_t *code_
   }
 }
 
-template <int DT, int NT>
+// kIndex: some tensor of the call has a value index (a separate kernel, so
+// that the common case's encoding loop has no index code).
+template <int DT, int NT, bool kIndex>
 __global__ void __launch_bounds__(NT, Enc<NT>::kMinBlocks) encode_kernel(const __grid_constant__ Batch b) {
   constexpr int A = DT == EH_FP8_E4M3 ? 16 : 256;
   extern __shared__ uint32_t ring[];  // Enc<NT>::kRingWords words, code bits in MSB-first order
@@ -730,10 +734,15 @@ __global__ void __launch_bounds__(NT, Enc<NT>::kMinBlocks) encode_kernel(const _
   load_code_table<DT>(tab, I.code_len, I.code);
   const uint8_t *in = (const uint8_t *)I.in + i0 * (DT == EH_BF16 ? 2 : 1);
   __syncthreads();
-  uint32_t *vindex = I.vindex ? I.vindex + (uint64_t)c * (b.chunk_elems / kIndexStride) : nullptr;
   uint8_t *smo = DT == EH_BF16 ? I.sm + i0 : (DT == EH_FP8_E4M3 ? I.sm + i0 / 2 : nullptr);
-  encode_range<DT, NT>(tab, in, cnt, I.off[c], I.off[c + 1], (uint32_t *)I.stream, ring, wsum, false, vindex, smo);
-  if (vindex) {
+  if (!kIndex || !I.vindex) {
+    encode_range<DT, NT>(tab, in, cnt, I.off[c], I.off[c + 1], (uint32_t *)I.stream, ring, wsum, false, nullptr, smo);
+    return;
+  }
+  uint32_t *vindex = I.vindex + (uint64_t)c * (b.chunk_elems / kIndexStride);
+  encode_range<DT, NT, true>(tab, in, cnt, I.off[c], I.off[c + 1], (uint32_t *)I.stream, ring, wsum, false, vindex,
+                             smo);
+  {
     // entries past a short last chunk's end: the chunk's bit count
     const uint32_t bits = (uint32_t)(I.off[c + 1] - I.off[c]);
     for (uint32_t k = (cnt + kIndexStride - 1) / kIndexStride + threadIdx.x; k < b.chunk_elems / kIndexStride;
@@ -962,12 +971,23 @@ cudaError_t configure_encode() {
   const int small = Enc<kEncSmall>::kRingWords * (int)sizeof(uint32_t);
   const int large = Enc<kEncLarge>::kRingWords * (int)sizeof(uint32_t);
   const cudaFuncAttribute dyn = cudaFuncAttributeMaxDynamicSharedMemorySize;
-  cudaError_t e = cudaFuncSetAttribute(encode_kernel<EH_BF16, kEncSmall>, dyn, small);
-  if (e == cudaSuccess) e = cudaFuncSetAttribute(encode_kernel<EH_BYTES, kEncSmall>, dyn, small);
-  if (e == cudaSuccess) e = cudaFuncSetAttribute(encode_kernel<EH_FP8_E4M3, kEncSmall>, dyn, small);
-  if (e == cudaSuccess) e = cudaFuncSetAttribute(encode_kernel<EH_BF16, kEncLarge>, dyn, large);
-  if (e == cudaSuccess) e = cudaFuncSetAttribute(encode_kernel<EH_BYTES, kEncLarge>, dyn, large);
-  if (e == cudaSuccess) e = cudaFuncSetAttribute(encode_kernel<EH_FP8_E4M3, kEncLarge>, dyn, large);
+  cudaError_t e = cudaSuccess;
+  const void *small_k[] = {(const void *)encode_kernel<EH_BF16, kEncSmall, false>,
+                           (const void *)encode_kernel<EH_BYTES, kEncSmall, false>,
+                           (const void *)encode_kernel<EH_FP8_E4M3, kEncSmall, false>,
+                           (const void *)encode_kernel<EH_BF16, kEncSmall, true>,
+                           (const void *)encode_kernel<EH_BYTES, kEncSmall, true>,
+                           (const void *)encode_kernel<EH_FP8_E4M3, kEncSmall, true>};
+  const void *large_k[] = {(const void *)encode_kernel<EH_BF16, kEncLarge, false>,
+                           (const void *)encode_kernel<EH_BYTES, kEncLarge, false>,
+                           (const void *)encode_kernel<EH_FP8_E4M3, kEncLarge, false>,
+                           (const void *)encode_kernel<EH_BF16, kEncLarge, true>,
+                           (const void *)encode_kernel<EH_BYTES, kEncLarge, true>,
+                           (const void *)encode_kernel<EH_FP8_E4M3, kEncLarge, true>};
+  for (const void *k : small_k)
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(k, dyn, small);
+  for (const void *k : large_k)
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(k, dyn, large);
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(page_append_kernel<EH_BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
@@ -1001,13 +1021,20 @@ cudaError_t launch_page_append(const PageLaunch &pl, cudaStream_t s) {
   return cudaGetLastError();
 }
 
-template <int NT>
-cudaError_t launch_encode_nt(const Batch &b, cudaStream_t s) {
+template <int NT, bool kIndex>
+cudaError_t launch_encode_nti(const Batch &b, cudaStream_t s) {
   const size_t smem = Enc<NT>::kRingWords * sizeof(uint32_t);
   const dim3 grid(b.total_chunks), block(NT);
-  if (b.dtype == EH_BF16) return launch_pdl(encode_kernel<EH_BF16, NT>, grid, block, smem, s, b);
-  if (b.dtype == EH_BYTES) return launch_pdl(encode_kernel<EH_BYTES, NT>, grid, block, smem, s, b);
-  return launch_pdl(encode_kernel<EH_FP8_E4M3, NT>, grid, block, smem, s, b);
+  if (b.dtype == EH_BF16) return launch_pdl(encode_kernel<EH_BF16, NT, kIndex>, grid, block, smem, s, b);
+  if (b.dtype == EH_BYTES) return launch_pdl(encode_kernel<EH_BYTES, NT, kIndex>, grid, block, smem, s, b);
+  return launch_pdl(encode_kernel<EH_FP8_E4M3, NT, kIndex>, grid, block, smem, s, b);
+}
+
+template <int NT>
+cudaError_t launch_encode_nt(const Batch &b, cudaStream_t s) {
+  bool index = false;
+  for (uint32_t i = 0; i < b.k; i++) index |= b.item[i].vindex != nullptr;
+  return index ? launch_encode_nti<NT, true>(b, s) : launch_encode_nti<NT, false>(b, s);
 }
 
 cudaError_t launch_encode(const Batch &b, cudaStream_t s) {

@@ -836,7 +836,7 @@ __device__ __forceinline__ uint32_t fp8_merge4(uint32_t nib16, uint32_t e4) {
   return ((t << 4) & 0x80808080u) | (t & 0x07070707u) | (e4 << 3);
 }
 
-template <int DT>
+template <int DT, bool kPlain>
 __device__ __forceinline__ ChunkInfo chunk_info(const Batch &b, uint32_t g) {
   ChunkInfo ci;
   ci.item = find_item(b, g);
@@ -844,7 +844,7 @@ __device__ __forceinline__ ChunkInfo chunk_info(const Batch &b, uint32_t g) {
   ci.c = I.first_chunk + (g - I.chunk0);
   ci.raw = 0;
   uint64_t B0, B1, Bt, i0;
-  if (I.page_meta) {
+  if (!kPlain && I.page_meta) {
     // page store: the page's codes start at bit 0 of its own slot
     const uint32_t slot = I.slot_ids[ci.c];
     ci.cnt = b.chunk_elems;
@@ -1015,7 +1015,9 @@ __device__ __forceinline__ void merge_region(const Item &I, const ChunkInfo &ci,
 // run the two groups take alternate chunks.  The last warp of a group to
 // finish writing a chunk's exponents (and so reading its stage) starts the
 // copy of the group's next chunk; every warp then merges its own region.
-template <int DT>
+// kPlain: no tensor of the call is a page store or has a value index (a
+// separate kernel, so that the common case carries none of their code).
+template <int DT, bool kPlain>
 __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_constant__ Batch b) {
   extern __shared__ __align__(128) uint8_t smem_raw[];
   DecodeSmem &S = *reinterpret_cast<DecodeSmem *>(smem_raw);
@@ -1047,7 +1049,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
     ChunkInfo ci;
     ci.fits = false;
     if (g < seg_end) {
-      ci = chunk_info<DT>(b, g);
+      ci = chunk_info<DT, kPlain>(b, g);
       if (ci.fits && gtid == 0) issue_stage(G, b.item[ci.item].stream + ci.lo, ci.bytes);
     }
     {
@@ -1075,7 +1077,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
       bool ok = ci.ok && !terr && !S.abort_flag;
       if (gtid == 0) {
         const uint32_t gn = g + kNumGroups;
-        if (gn < seg_end) G.next[j] = chunk_info<DT>(b, gn);
+        if (gn < seg_end) G.next[j] = chunk_info<DT, kPlain>(b, gn);
         else G.next[j].fits = false;
       }
 
@@ -1085,8 +1087,9 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
       // group never drift more than a chunk apart, and a chunk read from
       // global memory (no copy to wait for) cannot overwrite the end bits
       // that a slow warp of the previous chunk still reads.
-      const uint32_t *vidx = (ok && I.vindex && !I.page_meta) ? I.vindex + (uint64_t)ci.c * (b.chunk_elems / kIndexStride)
-                                                            : nullptr;
+      const uint32_t *vidx = (!kPlain && ok && I.vindex && !I.page_meta)
+                                 ? I.vindex + (uint64_t)ci.c * (b.chunk_elems / kIndexStride)
+                                 : nullptr;
       bool late = false;
       if (ci.fits) {
         late = !mbar_wait_bounded(&G.mbar, parity);
@@ -1095,7 +1098,8 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
           landed++;
         }
       }
-      if (!ok || ci.raw || vidx || !ci.fits) {
+      const bool raw_page = !kPlain && ci.raw;
+      if (!ok || raw_page || vidx || !ci.fits) {
         if (gsync_or(id, late)) {
           if (gtid == 0) {
             set_status(b.status, kFlagTimeout);
@@ -1106,7 +1110,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
       }
       uint32_t r0 = 0, r1 = 0;  // this warp's region of the chunk's values
       const uint8_t *raw = nullptr;
-      if (ok && ci.raw) {
+      if (ok && raw_page) {
         // page stored raw: the merge reads its exponent bytes from the pool
         raw = I.raw_pool + (uint64_t)(ci.raw - 1) * b.chunk_elems;
         const uint32_t per_warp = (cnt + kGroupWarps * 16 - 1) / (kGroupWarps * 16) * 16;
@@ -1115,7 +1119,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
       } else if (ok) {
         const uint32_t per = b.chunk_elems / kIndexStride;
         const uint32_t *gw = (const uint32_t *)(I.stream + ci.lo);
-        if (vidx) {
+        if (!kPlain && vidx) {
           const bool wok = ci.fits ? decode_chunk_indexed<true>(G, S.tabs, G.stage, ci.rel0, ci.nbits, cnt, gtid,
                                                                 vidx, per, &r0, &r1)
                                    : decode_chunk_indexed<false>(G, S.tabs, gw, ci.rel0, ci.nbits, cnt, gtid,
@@ -1150,7 +1154,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
 
       // 6. merge this warp's region with the sign/mantissa bytes
       if (ok && r1 > r0) {
-        if (raw) merge_region<DT, true>(I, ci, G.exps, raw, r0, r1, lane);
+        if (!kPlain && raw) merge_region<DT, true>(I, ci, G.exps, raw, r0, r1, lane);
         else merge_region<DT, false>(I, ci, G.exps, raw, r0, r1, lane);
       }
       // no barrier here: the next chunk's barriers order these reads of the
@@ -1175,18 +1179,28 @@ cudaError_t launch_decode(const Batch &b, cudaStream_t s, int num_sms) {
   const size_t smem = sizeof(DecodeSmem) + 128;
   uint32_t grid = (uint32_t)num_sms;
   if (grid > b.total_chunks) grid = b.total_chunks;
-  if (b.dtype == EH_BF16) return launch_pdl(decode_kernel<EH_BF16>, dim3(grid), dim3(kDecThreads), smem, s, b);
-  if (b.dtype == EH_BYTES) return launch_pdl(decode_kernel<EH_BYTES>, dim3(grid), dim3(kDecThreads), smem, s, b);
-  return launch_pdl(decode_kernel<EH_FP8_E4M3>, dim3(grid), dim3(kDecThreads), smem, s, b);
+  bool plain = true;
+  for (uint32_t i = 0; i < b.k; i++) plain &= !b.item[i].page_meta && !b.item[i].vindex;
+  const dim3 g(grid), t(kDecThreads);
+  if (plain) {
+    if (b.dtype == EH_BF16) return launch_pdl(decode_kernel<EH_BF16, true>, g, t, smem, s, b);
+    if (b.dtype == EH_BYTES) return launch_pdl(decode_kernel<EH_BYTES, true>, g, t, smem, s, b);
+    return launch_pdl(decode_kernel<EH_FP8_E4M3, true>, g, t, smem, s, b);
+  }
+  if (b.dtype == EH_BF16) return launch_pdl(decode_kernel<EH_BF16, false>, g, t, smem, s, b);
+  if (b.dtype == EH_BYTES) return launch_pdl(decode_kernel<EH_BYTES, false>, g, t, smem, s, b);
+  return launch_pdl(decode_kernel<EH_FP8_E4M3, false>, g, t, smem, s, b);
 }
 
 cudaError_t configure_decode() {
   const int smem = (int)(sizeof(DecodeSmem) + 128);
-  cudaError_t e = cudaFuncSetAttribute(decode_kernel<EH_BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(decode_kernel<EH_BYTES>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  if (e != cudaSuccess) return e;
-  return cudaFuncSetAttribute(decode_kernel<EH_FP8_E4M3>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  const void *kernels[] = {(const void *)decode_kernel<EH_BF16, true>, (const void *)decode_kernel<EH_BYTES, true>,
+                           (const void *)decode_kernel<EH_FP8_E4M3, true>, (const void *)decode_kernel<EH_BF16, false>,
+                           (const void *)decode_kernel<EH_BYTES, false>, (const void *)decode_kernel<EH_FP8_E4M3, false>};
+  cudaError_t e = cudaSuccess;
+  for (const void *k : kernels)
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  return e;
 }
 
 }  // namespace eh
