@@ -673,3 +673,64 @@ def test_container_layout(oracle, dtype, n, chunk, with_index):
         pos = end
     assert len(buf) == pos
     assert struct.unpack_from("<II", buf, 184) == (zlib.crc32(buf[:184]), 0)
+
+
+# ------------------------------------------------------------ randomized
+# Random tensors of the three alphabets with skewed (geometric) exponent
+# distributions, random sizes, chunk sizes and code-length limits: the stored
+# form must obey its definition and round-trip.
+
+from hypothesis import HealthCheck, given, settings, strategies as st  # noqa: E402
+
+
+def _skewed(dtype, n, rng):
+    g = rng.geometric(0.35, n)
+    if dtype == 0:
+        e = np.clip(121 - g, 0, 255).astype(np.uint16)
+        return ((rng.integers(0, 2, n).astype(np.uint16) << 15) | (e << 7)
+                | rng.integers(0, 128, n).astype(np.uint16)).astype(np.uint16)
+    if dtype == 1:
+        e = np.clip(9 - g, 0, 15).astype(np.uint8)
+        m = rng.integers(0, 8, n).astype(np.uint8)
+        m = np.where((e == 15) & (m == 7), 6, m).astype(np.uint8)  # no NaN patterns
+        return ((rng.integers(0, 2, n).astype(np.uint8) << 7) | (e << 3) | m).astype(np.uint8)
+    return np.clip(100 - g, 0, 255).astype(np.uint8)
+
+
+@settings(max_examples=60, deadline=None, suppress_health_check=[HealthCheck.function_scoped_fixture])
+@given(dtype=st.sampled_from([0, 1, 2]), n=st.integers(0, 5000), chunk=st.sampled_from([1024, 2048, 4096]),
+       lmax=st.integers(8, 32), seed=st.integers(0, 2 ** 31 - 1))
+def test_random_tensors(oracle, dtype, n, chunk, lmax, seed):
+    x = _skewed(dtype, n, np.random.default_rng(seed))
+    c = oracle.compress(dtype, x, chunk=chunk, lmax=lmax)
+    lens = c.code_len.astype(np.int64)
+    used = lens[lens > 0]
+    assert used.size == 0 or used.max() <= lmax
+    if used.size >= 2:
+        assert np.sum(2.0 ** -used) == 1.0  # a complete prefix code
+    # symbols and their code lengths, straight from the definition
+    if dtype == 0:
+        e = (x.astype(np.int64) >> 7) & 0xFF
+    elif dtype == 1:
+        e = (x.astype(np.int64) >> 3) & 0xF
+    else:
+        e = x.astype(np.int64)
+    assert np.all(lens[e] > 0)
+    per_value = lens[e]
+    C = -(-n // chunk)
+    off = c.chunk_bit_off.astype(np.int64)
+    assert off.size == C + 1 and off[0] == 0
+    for k in range(C):
+        assert off[k + 1] - off[k] == per_value[k * chunk:(k + 1) * chunk].sum()
+    assert c.bits == per_value.sum() and c.stream.size == (c.bits + 7) // 8
+    # sign and mantissa, stored raw
+    xi = x.astype(np.int64)
+    if dtype == 0:
+        assert np.array_equal(c.sign_mant, (((xi >> 8) & 0x80) | (xi & 0x7F)).astype(np.uint8))
+    elif dtype == 1:
+        nib = ((xi >> 4) & 0x8) | (xi & 0x7)
+        nib = np.concatenate([nib, np.zeros(n % 2, np.int64)])
+        assert np.array_equal(c.sign_mant, (nib[0::2] | (nib[1::2] << 4)).astype(np.uint8))
+    else:
+        assert c.sign_mant.size == 0
+    assert np.array_equal(oracle.decompress(c), x)
