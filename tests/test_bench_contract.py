@@ -41,3 +41,19 @@ def test_reference_arm_line():
 
 def test_reference_arm_other_ranks_are_silent():
     assert _run({"RANK": "1"}) == []
+
+
+def test_clock_summary():
+    # the bench line's `clocks`: median SM clock, highest max clock, every
+    # throttle reason seen in the timed region, sample count and source
+    sys.path.insert(0, ROOT)
+    import bench
+    c = bench.ClockSampler(0)
+    c.source = "test"
+    c.samples = [(1965.0, 1965.0, set()), (1900.0, 1965.0, {"sw_power_cap"}), (1965.0, 1965.0, set()),
+                 (1800.0, 1965.0, {"hw_slowdown"})]
+    d = c.summary()
+    assert d == {"sm_mhz": 1932.5, "sm_max_mhz": 1965.0, "reasons": ["hw_slowdown", "sw_power_cap"],
+                 "samples": 4, "source": "test"}
+    c.samples = []
+    assert c.summary()["samples"] == 0 and c.summary()["sm_mhz"] is None
